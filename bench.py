@@ -1,0 +1,425 @@
+"""Benchmark of the LSA hot path on B200: LSA decode queries/s and achieved HBM bandwidth.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl lsa|reference]
+
+A step is one pass of the whole path over one batch of synthetic input already resident
+in HBM: indexer (flat, or HI block scores -> recall -> fine scores), top-k with sinks and
+SI window, then sparse attention for every layer / draft step sharing the index, with
+split-KV merge.  Default workload: batched decode at 64K-128K context with cross-layer
+index reuse (32 sequences, 2 layers).  Multi-GPU (torchrun): every rank runs its own
+batch (weak scaling, no collective on the data path); value = all ranks' queries / the
+slowest rank's time.  ``--impl reference`` times the float64 CPU oracle on a bounded
+sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from lsa_synth import workloads as W  # noqa: E402
+
+METRIC = "LSA decode queries/s at 128K & 1M ctx; achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ the GPU arm
+
+def build_step(w, wt, pi, n_split):
+    from long_context_sparse_indexer_b200 import lsa
+    pt = wt.passes[pi]
+    p = w.passes[pi]
+    T = pt.q_idx.shape[0]
+    dev = pt.q_idx.device
+    batch = lsa.Batch(wt.seq_len, pt.q_seq, pt.q_pos, wt.L_alloc, q_group=p.q_per_seq)
+    layers = []
+    for L in pt.layers:
+        o = torch.empty((T, w.H, w.Dv), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((T, w.H), dtype=torch.float32, device=dev)
+        layers.append(lsa.Layer(L["q"], lsa.Cache(L["kv"], L["kv_scale"]), o, lse,
+                                lsa.Cache(L["v"]) if L["v"] is not None else None))
+    kbar = None
+    if w.hi:
+        nblk = (wt.L_alloc + w.block_size - 1) // w.block_size
+        kbar = torch.empty((w.B, nblk, w.d_I), dtype=torch.float32, device=dev)
+        lsa.block_keys(batch, lsa.Cache(pt.k_idx, pt.k_scale), w.block_size, kbar)
+    idx = torch.empty((T, w.cap), dtype=torch.int32, device=dev)
+    cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+    step = lsa.DecodeStep(batch, pt.q_idx, pt.w, lsa.Cache(pt.k_idx, pt.k_scale), w.k, w.n_sink, w.window, layers,
+                          w.H, w.D, w.Dv, w.sm_scale, n_split=n_split, hi=w.hi, block_size=w.block_size,
+                          n_recall=w.n_recall, kbar=kbar, idx_out=idx, count_out=cnt)
+    ws = torch.empty(max(256, step.workspace_size()), dtype=torch.uint8, device=dev)
+    return dict(step=step, ws=ws, idx=idx, cnt=cnt, layers=layers, batch=batch, kbar=kbar, T=T, n_split=n_split)
+
+
+def launches_per_step(w, n_split):
+    per = 0
+    for p in w.passes:
+        per += 4 if w.hi else 2
+        per += len(p.layers) * (2 if n_split > 1 else 1)
+    return per
+
+
+def algorithmic_bytes(w, wt, steps_data):
+    """Bytes the method must move per step (see the design notes): indexer keys once per pass, HI
+    block keys + recalled keys, selected KV rows once per layer (union over a sequence's tokens),
+    q / w / o / lse.  Returns (total, indexer_bytes_of_first_pass)."""
+    lens = W.lengths(w)
+    kb = w.d_I * (1 if w.idx_fp8 else 2) + (4 if w.idx_fp8 else 0)
+    rowb = w.D * (1 if w.kv_fp8 else 2) + (4 if w.kv_fp8 else 0)
+    total = 0
+    idx_first = 0
+    for pi, p in enumerate(w.passes):
+        sd = steps_data[pi]
+        T = sd["T"]
+        _, q_pos = W.query_rows(w, p)
+        qw = T * (w.H_I * w.d_I * 2 + w.H_I * 4)
+        if w.hi:
+            vis_blocks = sum(int(q_pos[t]) // w.block_size + 1 for t in range(T))
+            ib = vis_blocks * w.d_I * 4 + T * w.n_recall * w.block_size * kb + qw
+        else:
+            seq_max = {}
+            for t in range(T):
+                b = int(t // p.q_per_seq)
+                seq_max[b] = max(seq_max.get(b, 0), int(q_pos[t]) + 1)
+            ib = sum(seq_max.values()) * kb + qw
+        if pi == 0:
+            idx_first = ib
+        total += ib
+        idx = sd["idx"].cpu().numpy()
+        cnt = sd["cnt"].cpu().numpy()
+        rows = 0
+        for b in range(w.B):
+            toks = range(b * p.q_per_seq, (b + 1) * p.q_per_seq)
+            u = np.unique(np.concatenate([idx[t, :cnt[t]] for t in toks]))
+            rows += u.size
+        kvb = rows * rowb
+        distinct_kv = len({L.tid_kv for L in p.layers})
+        per_layer_io = T * (w.H * w.D * 2 + w.H * w.Dv * 2 + w.H * 4)
+        total += kvb * distinct_kv + per_layer_io * len(p.layers)
+        if distinct_kv < len(p.layers):   # draft steps: same rows, read again by each step's query
+            total += kvb * (len(p.layers) - distinct_kv)
+    return total, idx_first
+
+
+def time_region(fn, steps, stream):
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_gpu(args, rank, world, local_rank):
+    from lsa_synth import device as D
+    from long_context_sparse_indexer_b200 import launch, lsa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS[args.workload]
+    if world > 1:
+        w = W.scaled(args.workload, seed=w.seed + 1000 * rank)
+    wt = D.build_workload(w, dev)
+    stream = torch.cuda.current_stream()
+    sds = [build_step(w, wt, pi, launch.split_for(w.T(p), w.H)) for pi, p in enumerate(w.passes)]
+
+    def step():
+        for sd in sds:
+            sd["step"](sd["ws"], stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    graph = None
+    if not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    for sd in sds:
+                        sd["step"](sd["ws"], stream=s)
+            torch.cuda.synchronize()
+            graph = g
+        except Exception as e:  # capture unsupported: eager launches
+            print(f"[bench] graph capture failed, timing eager launches: {e}", file=sys.stderr)
+            graph = None
+    fn = (lambda: graph.replay()) if graph is not None else step
+    for _ in range(3):
+        fn()
+
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize()
+        ms = time_region(fn, args.steps, stream)
+    if world > 1:
+        dist.barrier()
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    q_per_step = w.queries_per_step()
+    value = q_per_step * world / (ms / 1e3)
+    total_bytes, idx_bytes = algorithmic_bytes(w, wt, sds)
+
+    # Dominant kernel: the indexer of the first pass, timed alone on the same inputs.
+    sd0 = sds[0]
+    pt0 = wt.passes[0]
+    k_cache = lsa.Cache(pt0.k_idx, pt0.k_scale)
+    if not w.hi:
+        ld = (wt.L_alloc + 3) // 4 * 4
+        sc = torch.empty((sd0["T"], ld), dtype=torch.float32, device=dev)
+        idx_fn = lambda: lsa.index_score(sd0["batch"], pt0.q_idx, pt0.w, k_cache, sc, n_cols=wt.L_alloc,  # noqa
+                                         stream=stream)
+        kern = "index_score (flat indexer)"
+    else:
+        nblk = (wt.L_alloc + w.block_size - 1) // w.block_size
+        sc = torch.empty((sd0["T"], (nblk + 3) // 4 * 4), dtype=torch.float32, device=dev)
+        idx_fn = lambda: lsa.block_score(sd0["batch"], pt0.q_idx, pt0.w, sd0["kbar"], w.block_size, sc, nblk,  # noqa
+                                         stream=stream)
+        kern = "block_score (HI coarse scores)"
+        lens = W.lengths(w)
+        idx_bytes = sum((int(l) - 1) // w.block_size + 1 for l in lens) * w.d_I * 4
+    for _ in range(3):
+        idx_fn()
+    kms = time_region(idx_fn, max(10, args.steps), stream)
+    hbm, src = peaks()
+    achieved = idx_bytes / (kms / 1e3) / 1e9
+
+    # End to end through the public API: H2D of the step's queries from pinned host memory, the
+    # fused calls, D2H of every layer's output.
+    h_in, d_in, h_out, d_out = [], [], [], []
+    for pi, pt in enumerate(wt.passes):
+        for t in [pt.q_idx, pt.w] + [L["q"] for L in pt.layers]:
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            h.copy_(t)
+            h_in.append(h)
+            d_in.append(t)
+        for L in sds[pi]["layers"]:
+            h_out.append(torch.empty(L.o.shape, dtype=L.o.dtype, pin_memory=True))
+            d_out.append(L.o)
+
+    def e2e():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        step()
+        for h, d in zip(h_out, d_out):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        e2e()
+    e2e_ms = time_region(e2e, args.steps, stream)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(h.numel() * h.element_size() for h in h_in)
+    d2h = sum(h.numel() * h.element_size() for h in h_out)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16+fp8", "data": "synthetic (seeded counter-based generator)",
+        "config": {"workload": w.name, "description": w.description, "batch": w.B,
+                   "queries_per_step_per_gpu": q_per_step, "ctx": [int(W.lengths(w).min()), int(W.lengths(w).max())],
+                   "k": w.k, "n_sink": w.n_sink, "window": w.window, "hi": w.hi,
+                   "layers_per_index": [len(p.layers) for p in w.passes],
+                   "n_split": [sd["n_split"] for sd in sds], "parallelism": f"replicas x{world} (batch per GPU)",
+                   "launch": "cuda_graph" if graph is not None else "eager",
+                   "l2": "inputs larger than L2 (indexer keys + selected KV rows per step >> 126 MB)"},
+        "algorithmic_gb_per_step": total_bytes / 1e9,
+        "step_hbm_gbs": total_bytes / (ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "peak_source": f"{src} hbm_gbs",
+                     "launch_ms": kms, "algorithmic_bytes_per_launch": idx_bytes},
+        "e2e": {"value": q_per_step * world / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step(w, sds[0]["n_split"]) * args.steps,
+        "clocks": clk.summary(),
+    }
+    return res, w, wt
+
+
+# ------------------------------------------------------------------ the CPU oracle (baseline / reference arm)
+
+def oracle_sample(w, n_tokens=1, layers_all=True):
+    """Times the float64 oracle's compute (selection + attention) on pre-decoded inputs of sampled tokens."""
+    from oracle import formats, lsa as olsa, run
+    p = w.passes[0]
+    T = w.T(p)
+    toks = sorted(set(np.linspace(0, T - 1, n_tokens).astype(int).tolist()))
+    plan = W.plant_plan(w, p) if (w.plant_frac or w.plant_blocks) else None
+    prepared = []
+    for t in toks:
+        b, pos, L, qi, wi = run.query_context(w, p, t)
+        K = run.index_keys(w, p, b, np.arange(L if w.hi else pos + 1), plan)
+        prepared.append((t, b, pos, L, qi, wi, K))
+    t0 = time.perf_counter()
+    for (t, b, pos, L, qi, wi, K) in prepared:
+        idx, _ = olsa.select(qi, wi, K, pos, w.k, w.n_sink, w.window, hi=w.hi, length=L, block_size=w.block_size,
+                             n_recall=w.n_recall)
+        for layer in p.layers:
+            q = formats.bf16_to_f64(W.attn_q_bits(w, layer, [t])[0])
+            Kr, Vr = run.kv_decoded(w, layer, b, idx)
+            olsa.attention(q, Kr, Vr, w.sm_scale)
+    dt = time.perf_counter() - t0
+    return len(toks), dt
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    w = W.WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        oracle_sample(w, 1)
+    n_q, tot = 0, 0.0
+    for _ in range(args.steps):
+        n, dt = oracle_sample(w, 1)
+        n_q += n
+        tot += dt
+    v = n_q / tot
+    cores = cpu_cores()
+    sample = (f"{args.steps} step(s) of 1 query token of {w.name} (all of its layers), inputs decoded "
+              f"beforehand; float64 numpy/BLAS")
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "queries/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded counter-based generator)",
+            "config": {"workload": w.name, "description": w.description},
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": v, "unit": "queries/s"},
+            "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_cli_128k", choices=list(W.WORKLOADS))
+    ap.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    res, w, wt = run_gpu(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            n, dt = oracle_sample(W.WORKLOADS[args.workload], 2)
+            res["cpu_baseline"] = {"value": n / dt, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+                                   "sample": f"{n} query tokens of {w.name} (all layers), float64 numpy/BLAS, "
+                                             f"inputs decoded beforehand; {dt:.2f} s"}
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

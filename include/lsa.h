@@ -1,0 +1,226 @@
+/*
+ * lsa.h -- C ABI of the LSA (LongCat Sparse Attention) hot path for NVIDIA B200 (sm_100a).
+ *
+ * Sources.  The operations follow the LongCat-2.0 pages:
+ *   [release]   "美团大模型LongCat-2.0 正式发布，总参数量达 1.6 万亿，使用国产算力集群",
+ *               section "LongCat 稀疏注意力" (SI, CLI and HI bullets; MTP paragraph) and
+ *               section "确定性与可靠性" (deterministic operators, tree reductions);
+ *   [explainer] "如何在 5 万张国产芯片训练出 1.6T 万亿参数模型？", section
+ *               "① LSA：从“每个 Query 全量扫”改成“先索引、再稀疏读”" and section
+ *               "③ KVP 解码切分示意" (partial attention per KV shard, then merged).
+ * The pages give no formula; the indexer score is the DSA form
+ *   I(t,s) = sum_h w[t,h] * ReLU(q[t,h,:] . k[s,:]),
+ * and the top-k order is (score descending, position ascending).
+ *
+ * Conventions for every entry point.
+ *   - All tensor pointers are DEVICE pointers, allocated and owned by the caller; the
+ *     library allocates, frees and synchronises nothing on these paths.  Structs
+ *     (lsa_batch, lsa_cache, lsa_layer, lsa_decode_params) are read on the host during
+ *     the call and may be discarded when it returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued
+ *     asynchronously; outputs are valid once the stream reaches that point.
+ *   - Host-side argument validation fails with a status and launches nothing.
+ *     A launch failure returns LSA_ERR_CUDA.
+ *   - Bad DEVICE data (q_pos >= seq_len, an index outside 0..seq_len-1, a NaN score,
+ *     a sequence id outside 0..B-1) is detected in the kernels: the offending access is
+ *     skipped and, when `dev_status` is not NULL, an lsa_status code is stored there
+ *     (the first error wins).  `dev_status` points to one int32 in device memory that
+ *     the caller zeroes before use; read it with lsa_read_device_status.  Kernels never
+ *     trap.
+ *   - Deterministic: identical inputs and parameters (including n_split) give bitwise
+ *     identical outputs.  No floating-point atomics are used; every reduction has a
+ *     fixed order.
+ *   - Element strides are counted in elements of the cache's dtype.
+ *   - No exception crosses this boundary.  Calls on different streams may run
+ *     concurrently as long as their output buffers do not overlap.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LSA_OK = 0,
+    LSA_ERR_INVALID_ARG = 1,   /* host validation: null pointer, bad size, misalignment */
+    LSA_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels implement */
+    LSA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the *_workspace_size result */
+    LSA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    LSA_ERR_DEVICE_DATA = 5,   /* (device) bad lengths / positions / indices, NaN score */
+    LSA_ERR_TIMEOUT = 6        /* (device) a bounded wait gave up */
+} lsa_status;
+
+typedef enum { LSA_BF16 = 0, LSA_FP8_E4M3 = 1, LSA_FP32 = 2 } lsa_dtype;
+
+/* lsa_topk flags */
+#define LSA_TOPK_RAW (1u << 0) /* output the selected COLUMN ids, no sink/window union (HI recall) */
+
+/* A per-sequence cache: row r of sequence b starts at
+ *   data + b * seq_stride + r * tok_stride            (elements of `dtype`),
+ * and its FP8 scale (one float per row, FP8 caches only) at
+ *   scale[b * scale_seq_stride + r].
+ * A row's value is data (BF16) or scale * data (FP8 e4m3, OCP definition). */
+typedef struct {
+    const void*  data;
+    const float* scale;            /* FP8: per-token scale (> 0); BF16: NULL */
+    int32_t      dtype;            /* LSA_BF16 or LSA_FP8_E4M3 */
+    int32_t      dim;              /* elements per row */
+    int64_t      seq_stride;       /* elements between sequences */
+    int64_t      tok_stride;       /* elements between rows (>= dim) */
+    int64_t      scale_seq_stride; /* floats between sequences in `scale` */
+} lsa_cache;
+
+/* The query tokens of one call.  Token t belongs to sequence q_seq[t] and sits at
+ * position q_pos[t]; it sees keys 0..q_pos[t] (causal).  Tokens are grouped in runs of
+ * `q_group` consecutive tokens of the same sequence (1 for plain decode, the verify
+ * length for speculative decoding, the chunk length for prefill); kernels read a
+ * sequence's keys once per group. */
+typedef struct {
+    int32_t        B;          /* sequences */
+    int32_t        T;          /* query tokens, a multiple of q_group */
+    int32_t        q_group;    /* consecutive tokens sharing a sequence */
+    int32_t        L_alloc;    /* rows allocated per sequence in the caches */
+    const int32_t* seq_len;    /* device [B], 1 <= seq_len[b] <= L_alloc */
+    const int32_t* q_seq;      /* device [T], 0 <= q_seq[t] < B */
+    const int32_t* q_pos;      /* device [T], 0 <= q_pos[t] < seq_len[q_seq[t]] */
+} lsa_batch;
+
+/* ---------------------------------------------------------------- a1 / a4: indexer
+ * Indexer scores  I(t,s) = sum_h w[t,h] * ReLU(q_idx[t,h,:] . k(s))  for the key rows k(s)
+ * of the indexer cache ([release] "LongCat 稀疏注意力": the lightweight indexer that
+ * scores keys for each query; DSA form).  FP8 keys contribute scale(s) * code(s).
+ *   q_idx  [T][H_I][d_I] BF16, d_I = k_idx->dim (64 or 128);  w [T][H_I] float.
+ *   Flat (cand_blocks == NULL): scores[t * ld_scores + s] for s < n_cols, the score when
+ *     s <= q_pos[t], -INFINITY otherwise.
+ *   Fine stage of HI (cand_blocks != NULL): cand_blocks [T][n_cand] int32 block ids
+ *     (ascending, -1 = unused); column c < n_cand * block_size is position
+ *     cand_blocks[t][c / block_size] * block_size + c % block_size; its score, or
+ *     -INFINITY when the block id is -1 or the position is beyond q_pos[t].
+ *   Requires H_I % 8 == 0, H_I <= 128, ld_scores >= number of columns, 16-byte aligned
+ *   q_idx / data / rows. */
+lsa_status lsa_index_score(const lsa_batch* batch, const void* q_idx, const float* w, int H_I,
+                           const lsa_cache* k_idx, const int32_t* cand_blocks, int n_cand,
+                           int block_size, float* scores, int64_t ld_scores, int n_cols,
+                           int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- a2: HI block keys
+ * Block key of block j of sequence b = arithmetic mean of the dequantised indexer keys
+ * of rows j*block_size .. min(seq_len[b], (j+1)*block_size) - 1 ([release] HI bullet:
+ * block-level approximate scoring; the mean is this library's block summary).
+ *   kbar [B][*][d_I] float, sequence b at kbar + b * kbar_seq_stride; blocks
+ *   0 .. ceil(seq_len[b] / block_size) - 1 are written.  Cache maintenance: rerun for the
+ *   blocks whose rows changed (here: all). */
+lsa_status lsa_block_keys(const lsa_batch* batch, const lsa_cache* k_idx, int block_size,
+                          float* kbar, int64_t kbar_seq_stride, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- a2: HI block scores
+ * J(t,j) = sum_h w[t,h] * ReLU(q_idx[t,h,:] . kbar[q_seq[t], j, :]) for block columns
+ * j < n_cols: the score when block j is visible (j * block_size <= q_pos[t]), else
+ * -INFINITY.  d_I = dimension of q_idx rows (64 or 128). */
+lsa_status lsa_block_score(const lsa_batch* batch, const void* q_idx, const float* w, int H_I, int d_I,
+                           const float* kbar, int64_t kbar_seq_stride, int block_size,
+                           float* scores, int64_t ld_scores, int n_cols,
+                           int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- a3 / a5: top-k and union
+ * Per query row t: candidates are the columns c < n_cols with scores[t * ld + c] != -inf.
+ * The k candidates ranked first by (score desc, column asc) are selected (all of them if
+ * fewer); -0 ranks equal to +0; a NaN score sets LSA_ERR_DEVICE_DATA and is ignored.
+ *   Default: columns map to positions (identity, or through cand_blocks as in
+ *   lsa_index_score); the output is the ascending, de-duplicated union of the selected
+ *   positions, the sinks 0..n_sink-1 and the SI window q_pos-window+1..q_pos, all clipped
+ *   to 0..q_pos ([explainer] "① LSA": top-k keys plus a few fixed sink tokens; [release]
+ *   SI bullet: a contiguous, hardware-aligned window beside the dynamic picks).
+ *   LSA_TOPK_RAW: the output is the selected column ids, ascending (HI coarse recall);
+ *   n_sink and window must be 0.
+ *   idx [T][ld_idx] int32, entries beyond count[t] set to -1; count [T] int32.
+ *   ld_idx >= k + n_sink + window. */
+lsa_status lsa_topk(const lsa_batch* batch, const float* scores, int64_t ld_scores, int n_cols,
+                    const int32_t* cand_blocks, int n_cand, int block_size,
+                    int k, int n_sink, int window, uint32_t flags,
+                    int32_t* idx, int64_t ld_idx, int32_t* count,
+                    int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- a7 / a8: sparse attention
+ * For each query token t and head h, softmax attention over the rows idx[t][0..count[t]-1]
+ * of sequence q_seq[t] ([explainer] "① LSA": attention reads only the selected keys):
+ *   z_j = sm_scale * q[t,h,:] . K_j,  o[t,h,:] = sum_j softmax(z)_j V_j,
+ *   lse[t,h] = log sum_j exp(z_j)  (natural log; -inf and o = 0 for an empty list).
+ * K_j is row j of `kv` (dim = Dqk).  V_j is row j of `v` (dim = Dv) or, when v == NULL,
+ * the first Dv elements of K_j (MLA absorbed layout).  FP8 rows are scale * code.
+ * The list is cut into n_split contiguous chunks processed in parallel; the partial
+ * results are merged with the log-sum-exp rule in a fixed binary tree ([explainer]
+ * "③ KVP 解码切分示意": partial attention per KV shard, then merged -- here the shards are
+ * chunks of one GPU's work).
+ *   q [T][H][Dqk] BF16, o [T][H][Dv] BF16, lse [T][H] float (may be NULL).
+ *   Supported: (Dqk, Dv) = (576, 512) with H % 32 == 0, or (128, 128) with H % 16 == 0;
+ *   1 <= n_split <= 64.  ws: lsa_attn_workspace_size(T, H, Dv, n_split) bytes (0 when
+ *   n_split == 1; ws may then be NULL). */
+lsa_status lsa_sparse_attn(const lsa_batch* batch, const void* q, int H, int Dqk,
+                           const lsa_cache* kv, const lsa_cache* v, int Dv,
+                           const int32_t* idx, int64_t ld_idx, const int32_t* count,
+                           float sm_scale, int n_split, void* o, float* lse,
+                           void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+size_t lsa_attn_workspace_size(int T, int H, int Dv, int n_split);
+
+/* ---------------------------------------------------------------- fused decode / prefill step
+ * One attention layer consuming a shared index list (cross-layer indexing: [release] CLI
+ * bullet, one index serves consecutive layers; MTP paragraph, draft steps 2 and 3 reuse
+ * step 1's index). */
+typedef struct {
+    const void* q;         /* [T][H][Dqk] BF16 */
+    lsa_cache   kv;        /* K rows (and V = first Dv dims when v.data == NULL) */
+    lsa_cache   v;         /* separate V cache, or v.data == NULL */
+    void*       o;         /* [T][H][Dv] BF16 */
+    float*      lse;       /* [T][H] or NULL */
+} lsa_layer;
+
+typedef struct {
+    lsa_batch        batch;
+    /* indexer */
+    const void*      q_idx;      /* [T][H_I][d_I] BF16 */
+    const float*     w;          /* [T][H_I] */
+    int32_t          H_I;
+    lsa_cache        k_idx;
+    /* selection */
+    int32_t          k, n_sink, window;
+    /* hierarchical indexing (hi != 0): block keys kbar from lsa_block_keys */
+    int32_t          hi, block_size, n_recall;
+    const float*     kbar;
+    int64_t          kbar_seq_stride;
+    /* attention layers sharing the index */
+    int32_t          H, Dqk, Dv;
+    float            sm_scale;
+    int32_t          n_split;
+    int32_t          n_layers;
+    const lsa_layer* layers;     /* host array [n_layers] */
+    /* optional: the index list and its counts are also written here ([T][idx_ld], [T]) */
+    int32_t*         idx_out;
+    int64_t          idx_ld;
+    int32_t*         count_out;
+} lsa_decode_params;
+
+/* Runs indexer (flat, or HI: block scores -> recall -> fine scores), top-k + union, then
+ * attention for every layer, all on `stream`, with no host synchronisation.  Scores,
+ * index lists and split partials live in `ws` (lsa_decode_workspace_size bytes). */
+lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_bytes,
+                            int32_t* dev_status, void* stream);
+
+size_t lsa_decode_workspace_size(const lsa_decode_params* p);
+
+/* ---------------------------------------------------------------- helpers
+ * Synchronises `stream`, then returns the status stored at dev_status (LSA_OK when 0),
+ * or LSA_ERR_CUDA if the copy fails. */
+lsa_status  lsa_read_device_status(const int32_t* dev_status, void* stream);
+const char* lsa_status_string(lsa_status s);
+int         lsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LSA_H_ */

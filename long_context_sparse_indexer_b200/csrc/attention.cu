@@ -1,0 +1,355 @@
+// Sparse attention over the selected rows, split-KV partials and their log-sum-exp merge.
+//
+// Explainer page ("如何在 5 万张国产芯片训练出 1.6T 万亿参数模型？"), section "① LSA": attention
+// reads only the top-k keys and the sink tokens the indexer selected; the model's
+// attention is MLA in absorbed form, so all heads of a query share one latent KV row
+// (K = the 576-dim row, V = its first 512 dims).  Section "③ KVP 解码切分示意": each KV
+// shard computes a partial attention and the partial results are merged; here the shards
+// are contiguous chunks of one query's index list (n_split), merged in a fixed binary
+// tree, as the release post's section "确定性与可靠性" asks of reductions.
+//
+// CTA = (split, group of 16*MT heads, query token).  Warps 0..4*MT-1: warp w owns head
+// tile (w % MT) and quarter (w / MT).  For S = Q K^T each quarter computes a partial over
+// a quarter of the QK dims; the four partials meet in shared memory and are summed in a
+// fixed order.  Every warp then runs the same online softmax on its head tile and
+// accumulates P V for its quarter of the V dims.  FP8 rows are widened exactly to BF16;
+// their per-row scale multiplies the scores and the probabilities.
+#include "kernels.cuh"
+
+namespace lsa {
+
+constexpr int kNR = 32;          // rows per tile
+
+template <int DQK, int DV, int MT, bool KV_FP8, bool SEP_V>
+struct AttnCfg {
+    static constexpr int WARPS = 4 * MT;
+    static constexpr int THREADS = WARPS * 32;
+    static constexpr int KLD = DQK + 8;              // padded smem row (elements): 16 B shift per row
+    static constexpr int VLD = DV + 8;
+    static constexpr int KQ = DQK / 4 / 16;          // k16 steps per quarter
+    static constexpr int NV = DV / 4 / 8;            // n8 tiles of V per quarter
+    static constexpr size_t K_BYTES = (size_t)kNR * KLD * 2;
+    static constexpr size_t V_BYTES = SEP_V ? (size_t)kNR * VLD * 2 : 0;
+    static constexpr size_t SP_BYTES = (size_t)4 * MT * 16 * kNR * 4;
+    static constexpr size_t SMEM = K_BYTES + V_BYTES + SP_BYTES + 3 * kNR * 4;
+};
+
+template <int DQK, int DV, int MT, bool KV_FP8, bool SEP_V>
+__global__ void __launch_bounds__(AttnCfg<DQK, DV, MT, KV_FP8, SEP_V>::THREADS)
+sparse_attn_kernel(AttnArgs a) {
+    using C = AttnCfg<DQK, DV, MT, KV_FP8, SEP_V>;
+    static_assert(DQK % 64 == 0 && DV % 64 == 0, "dims");
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint16_t* sK = reinterpret_cast<uint16_t*>(smem);
+    uint16_t* sV = SEP_V ? reinterpret_cast<uint16_t*>(smem + C::K_BYTES) : sK;
+    float* sP = reinterpret_cast<float*>(smem + C::K_BYTES + C::V_BYTES);          // [4][MT][16][kNR]
+    float* sKs = reinterpret_cast<float*>(smem + C::K_BYTES + C::V_BYTES + C::SP_BYTES);  // [kNR] K scale
+    float* sVs = sKs + kNR;                                                         // [kNR] V scale
+    int* sOk = reinterpret_cast<int*>(sVs + kNR);                                   // [kNR] row valid
+    const int vld = SEP_V ? C::VLD : C::KLD;
+
+    const int split = blockIdx.x, hg = blockIdx.y, t = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int mw = warp % MT, qw = warp / MT;
+    const int h0 = hg * 16 * MT + mw * 16;             // first head of this warp's tile
+
+    const int b = a.q_seq[t];
+    int len = 0;
+    bool ok = b >= 0 && b < a.B;
+    if (ok) { len = a.seq_len[b]; ok = len >= 1 && len <= a.L_alloc; }
+    int n = ok ? a.count[t] : 0;
+    if (n < 0 || n > a.ld_idx) { ok = false; n = 0; }
+    if (!ok && threadIdx.x == 0 && split == 0 && hg == 0) report(a.status, LSA_ERR_DEVICE_DATA);
+    const int per = (n + a.n_split - 1) / a.n_split;
+    const int r_beg = min(n, split * per), r_end = min(n, r_beg + per);
+    const int32_t* irow = a.idx + (size_t)t * a.ld_idx;
+    const uint8_t* kvb = a.kv + (size_t)max(b, 0) * a.kv_seq_b;
+    const float* kvs = KV_FP8 ? a.kv_scale + (size_t)max(b, 0) * a.kv_scale_seq : nullptr;
+    const uint8_t* vb = SEP_V ? a.v + (size_t)max(b, 0) * a.v_seq_b : nullptr;
+
+    // Q fragments for this warp's head tile and QK quarter (A operand, row-major).
+    uint32_t qf[C::KQ][4];
+    {
+        const uint16_t* q0 = a.q + ((size_t)t * a.H + h0 + g) * DQK + qw * (DQK / 4);
+        const uint16_t* q8 = q0 + (size_t)8 * DQK;
+#pragma unroll
+        for (int s = 0; s < C::KQ; ++s) {
+            qf[s][0] = *reinterpret_cast<const uint32_t*>(q0 + s * 16 + 2 * c);
+            qf[s][1] = *reinterpret_cast<const uint32_t*>(q8 + s * 16 + 2 * c);
+            qf[s][2] = *reinterpret_cast<const uint32_t*>(q0 + s * 16 + 8 + 2 * c);
+            qf[s][3] = *reinterpret_cast<const uint32_t*>(q8 + s * 16 + 8 + 2 * c);
+        }
+    }
+    float oacc[C::NV][4];
+#pragma unroll
+    for (int i = 0; i < C::NV; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[i][e] = 0.f;
+    float m_run[2] = {kNegInf, kNegInf}, l_run[2] = {0.f, 0.f};
+
+    for (int r0 = r_beg; r0 < r_end; r0 += kNR) {
+        const int nr = min(kNR, r_end - r0);
+        // ---- gather the tile's rows into shared memory
+        if (!KV_FP8) {
+            constexpr int CPR = DQK * 2 / 16;           // 16-byte chunks per row
+            for (int i = threadIdx.x; i < kNR * CPR; i += C::THREADS) {
+                const int r = i / CPR, ch = i % CPR;
+                int row = r < nr ? irow[r0 + r] : -1;
+                bool valid = row >= 0 && row < len;
+                if (r < nr && !valid) report(a.status, LSA_ERR_DEVICE_DATA);
+                cp_async16(sK + (size_t)r * C::KLD + ch * 8, kvb + (size_t)(valid ? row : 0) * a.kv_tok_b + ch * 16, valid);
+            }
+            if (SEP_V) {
+                constexpr int CPV = DV * 2 / 16;
+                for (int i = threadIdx.x; i < kNR * CPV; i += C::THREADS) {
+                    const int r = i / CPV, ch = i % CPV;
+                    int row = r < nr ? irow[r0 + r] : -1;
+                    bool valid = row >= 0 && row < len;
+                    cp_async16(sV + (size_t)r * C::VLD + ch * 8, vb + (size_t)(valid ? row : 0) * a.v_tok_b + ch * 16, valid);
+                }
+            }
+            cp_async_commit();
+            if (threadIdx.x < kNR) {
+                const int r = threadIdx.x;
+                const int row = r < nr ? irow[r0 + r] : -1;
+                sKs[r] = 1.f;
+                sVs[r] = 1.f;
+                sOk[r] = row >= 0 && row < len;
+            }
+            cp_async_wait<0>();
+        } else {
+            constexpr int CPR = DQK / 16;               // 16 codes per chunk
+            for (int i = threadIdx.x; i < kNR * CPR; i += C::THREADS) {
+                const int r = i / CPR, ch = i % CPR;
+                int row = r < nr ? irow[r0 + r] : -1;
+                bool valid = row >= 0 && row < len;
+                if (r < nr && !valid) report(a.status, LSA_ERR_DEVICE_DATA);
+                uint4 raw = valid ? ldg_nc16(kvb + (size_t)row * a.kv_tok_b + ch * 16) : make_uint4(0, 0, 0, 0);
+                const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw);
+                uint32_t outw[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    outw[2 * j] = e4m3x2_to_bf16x2((uint16_t)(wd[j] & 0xffff));
+                    outw[2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(wd[j] >> 16));
+                }
+                uint4* dst = reinterpret_cast<uint4*>(sK + (size_t)r * C::KLD + ch * 16);
+                dst[0] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+                dst[1] = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+            }
+            if (threadIdx.x < kNR) {
+                const int r = threadIdx.x;
+                int row = r < nr ? irow[r0 + r] : -1;
+                bool valid = row >= 0 && row < len;
+                const float s = valid ? kvs[row] : 0.f;
+                sKs[r] = s;
+                sVs[r] = s;
+                sOk[r] = valid;
+            }
+        }
+        __syncthreads();
+
+        // ---- partial S over this warp's QK quarter: [16 heads] x [32 rows]
+        float sacc[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[j][e] = 0.f;
+#pragma unroll
+        for (int s = 0; s < C::KQ; ++s) {
+            const int k0 = qw * (DQK / 4) + s * 16;
+#pragma unroll
+            for (int jp = 0; jp < 2; ++jp) {              // pairs of n8 row tiles
+                uint32_t bf[4];
+                const int mi = lane >> 3, ri = lane & 7;
+                const int row = jp * 16 + (mi >> 1) * 8 + ri;
+                const int col = k0 + (mi & 1) * 8;
+                ldmatrix_x4(bf, sK + (size_t)row * C::KLD + col);
+                mma_bf16_16816(sacc[2 * jp], qf[s], bf[0], bf[1]);
+                mma_bf16_16816(sacc[2 * jp + 1], qf[s], bf[2], bf[3]);
+            }
+        }
+        float* myP = sP + ((size_t)(qw * MT + mw) * 16) * kNR;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            *reinterpret_cast<float2*>(myP + g * kNR + j * 8 + 2 * c) = make_float2(sacc[j][0], sacc[j][1]);
+            *reinterpret_cast<float2*>(myP + (g + 8) * kNR + j * 8 + 2 * c) = make_float2(sacc[j][2], sacc[j][3]);
+        }
+        __syncthreads();
+
+        // ---- full S (fixed order), mask, online softmax
+        float sv[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int hr = g + 8 * (e >> 1), col = j * 8 + 2 * c + (e & 1);
+                const float* base = sP + (size_t)mw * 16 * kNR + hr * kNR + col;
+                const size_t qs = (size_t)MT * 16 * kNR;
+                const float x = (base[0] + base[qs]) + (base[2 * qs] + base[3 * qs]);
+                sv[j][e] = sOk[col] ? x * sKs[col] * a.sm_scale_log2 : kNegInf;
+            }
+        float alpha[2];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            float mx = kNegInf;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) mx = fmaxf(mx, fmaxf(sv[j][2 * hf], sv[j][2 * hf + 1]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run[hf], mx);
+            alpha[hf] = (m_new == kNegInf) ? 1.f : exp2f(m_run[hf] - m_new);
+            float ls = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float p = (m_new == kNegInf) ? 0.f : exp2f(sv[j][2 * hf + e] - m_new);
+                    sv[j][2 * hf + e] = p;
+                    ls += p;
+                }
+            ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+            ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+            l_run[hf] = l_run[hf] * alpha[hf] + ls;
+            m_run[hf] = m_new;
+        }
+#pragma unroll
+        for (int i = 0; i < C::NV; ++i) {
+            oacc[i][0] *= alpha[0]; oacc[i][1] *= alpha[0];
+            oacc[i][2] *= alpha[1]; oacc[i][3] *= alpha[1];
+        }
+        // ---- P (times the V scale) as the A operand; O += P V for this warp's V quarter
+        uint32_t pf[2][4];
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const int ca = kk * 16 + 2 * c, cb = ca + 8;
+            const float v0 = sVs[ca], v1 = sVs[ca + 1], v2 = sVs[cb], v3 = sVs[cb + 1];
+            pf[kk][0] = pack_bf16x2(sv[2 * kk][0] * v0, sv[2 * kk][1] * v1);
+            pf[kk][1] = pack_bf16x2(sv[2 * kk][2] * v0, sv[2 * kk][3] * v1);
+            pf[kk][2] = pack_bf16x2(sv[2 * kk + 1][0] * v2, sv[2 * kk + 1][1] * v3);
+            pf[kk][3] = pack_bf16x2(sv[2 * kk + 1][2] * v2, sv[2 * kk + 1][3] * v3);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+            for (int np = 0; np < C::NV / 2; ++np) {
+                uint32_t bf[4];
+                const int mi = lane >> 3, ri = lane & 7;
+                const int row = kk * 16 + (mi & 1) * 8 + ri;
+                const int col = qw * (DV / 4) + (2 * np + (mi >> 1)) * 8;
+                ldmatrix_x4_trans(bf, sV + (size_t)row * vld + col);
+                mma_bf16_16816(oacc[2 * np], pf[kk], bf[0], bf[1]);
+                mma_bf16_16816(oacc[2 * np + 1], pf[kk], bf[2], bf[3]);
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- epilogue
+    const float kLn2 = 0.69314718055994530942f;
+    float inv[2], lse_v[2];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        inv[hf] = l_run[hf] > 0.f ? 1.f / l_run[hf] : 0.f;
+        lse_v[hf] = l_run[hf] > 0.f ? (m_run[hf] + log2f(l_run[hf])) * kLn2 : kNegInf;
+    }
+    const int dv0 = qw * (DV / 4);
+    if (a.n_split == 1) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int h = h0 + g + 8 * hf;
+            uint16_t* orow = a.o + ((size_t)t * a.H + h) * DV + dv0;
+#pragma unroll
+            for (int i = 0; i < C::NV; ++i)
+                *reinterpret_cast<uint32_t*>(orow + i * 8 + 2 * c) =
+                    pack_bf16x2(oacc[i][2 * hf] * inv[hf], oacc[i][2 * hf + 1] * inv[hf]);
+            if (a.lse && qw == 0 && c == 0) a.lse[(size_t)t * a.H + h] = lse_v[hf];
+        }
+    } else {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int h = h0 + g + 8 * hf;
+            float* prow = a.part_o + (((size_t)t * a.n_split + split) * a.H + h) * DV + dv0;
+#pragma unroll
+            for (int i = 0; i < C::NV; ++i)
+                *reinterpret_cast<float2*>(prow + i * 8 + 2 * c) =
+                    make_float2(oacc[i][2 * hf] * inv[hf], oacc[i][2 * hf + 1] * inv[hf]);
+            if (qw == 0 && c == 0) a.part_lse[((size_t)t * a.n_split + split) * a.H + h] = lse_v[hf];
+        }
+    }
+}
+
+// Merge of split partials: a fixed pairwise tree in binary-counter order (the balanced tree
+// when n_split is a power of two).  Thread = 4 consecutive V dims of one (token, head).
+__device__ __forceinline__ void lse_combine(float4& o1, float& l1, const float4& o2, float l2) {
+    const float m = fmaxf(l1, l2);
+    if (m == kNegInf) { o1 = make_float4(0.f, 0.f, 0.f, 0.f); l1 = kNegInf; return; }
+    const float w1 = expf(l1 - m), w2 = expf(l2 - m);
+    const float s = w1 + w2, r = 1.f / s;
+    o1.x = (w1 * o1.x + w2 * o2.x) * r;
+    o1.y = (w1 * o1.y + w2 * o2.y) * r;
+    o1.z = (w1 * o1.z + w2 * o2.z) * r;
+    o1.w = (w1 * o1.w + w2 * o2.w) * r;
+    l1 = m + logf(s);
+}
+
+__global__ void merge_kernel(const float* part_o, const float* part_lse, int n_split, int H, int DV,
+                             uint16_t* o, float* lse) {
+    const int t = blockIdx.y, h = blockIdx.x, d = threadIdx.x * 4;
+    if (d >= DV) return;
+    float4 st_o[7];
+    float st_l[7];
+    for (int s = 0; s < n_split; ++s) {
+        const size_t base = ((size_t)t * n_split + s) * H + h;
+        float4 v = *reinterpret_cast<const float4*>(part_o + base * DV + d);
+        float l = part_lse[base];
+        int lvl = 0;
+        for (int m = s; m & 1; m >>= 1, ++lvl) {
+            float4 acc = st_o[lvl];
+            float la = st_l[lvl];
+            lse_combine(acc, la, v, l);
+            v = acc;
+            l = la;
+        }
+        st_o[lvl] = v;
+        st_l[lvl] = l;
+    }
+    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+    float tl = kNegInf;
+    bool have = false;
+    for (int lvl = 0; lvl < 7; ++lvl)
+        if ((n_split >> lvl) & 1) {
+            if (!have) { tot = st_o[lvl]; tl = st_l[lvl]; have = true; }
+            else { float4 acc = st_o[lvl]; float la = st_l[lvl]; lse_combine(acc, la, tot, tl); tot = acc; tl = la; }
+        }
+    uint16_t* orow = o + ((size_t)t * H + h) * DV + d;
+    *reinterpret_cast<uint2*>(orow) = make_uint2(pack_bf16x2(tot.x, tot.y), pack_bf16x2(tot.z, tot.w));
+    if (lse && d == 0) lse[(size_t)t * H + h] = tl;
+}
+
+template <int DQK, int DV, int MT, bool KV_FP8, bool SEP_V>
+static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
+    using C = AttnCfg<DQK, DV, MT, KV_FP8, SEP_V>;
+    auto kern = sparse_attn_kernel<DQK, DV, MT, KV_FP8, SEP_V>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.n_split, a.H / (16 * MT), a.T);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.n_split == 1) return e;
+    dim3 mg(a.H, a.T);
+    merge_kernel<<<mg, DV / 4, 0, st>>>(a.part_o, a.part_lse, a.n_split, a.H, DV, a.o, a.lse);
+    return cudaGetLastError();
+}
+
+// Supported: (576, 512) MLA layout, BF16 or FP8 rows, H % 32 == 0; (128, 128) with a
+// separate BF16 V cache, H % 16 == 0.
+cudaError_t launch_sparse_attn(const AttnArgs& a, int DQK, int DV, bool kv_fp8, bool sep_v, cudaStream_t st) {
+    if (a.T <= 0) return cudaSuccess;
+    if (DQK == 576 && DV == 512 && !sep_v)
+        return kv_fp8 ? launch_attn_t<576, 512, 2, true, false>(a, st) : launch_attn_t<576, 512, 2, false, false>(a, st);
+    if (DQK == 128 && DV == 128 && sep_v && !kv_fp8) return launch_attn_t<128, 128, 1, false, true>(a, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace lsa

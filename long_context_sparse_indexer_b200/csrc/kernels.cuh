@@ -1,0 +1,104 @@
+// Internal kernel interfaces of the LSA library (argument blocks and host launchers).
+#pragma once
+
+#include "common.cuh"
+
+namespace lsa {
+
+struct IndexArgs {
+    const int32_t* seq_len;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    int B, T, q_group, L_alloc;
+    const uint16_t* q;       // bf16 bits [T][H_I][D_I]
+    const float* w;          // [T][H_I]
+    const uint8_t* kdata;    // cache base (bytes)
+    const float* kscale;     // per-token scale or NULL
+    int64_t seq_stride_b, tok_stride_b, scale_seq_stride;
+    const int32_t* cand;     // [T][n_cand] or NULL
+    int n_cand, block_size;
+    float* scores;
+    int64_t ld;
+    int n_cols;              // columns to write
+    int group;               // tokens per CTA (<= 4)
+    int32_t* status;
+};
+
+struct BlockKeyArgs {
+    const int32_t* seq_len;
+    int B, L_alloc;
+    const uint8_t* kdata;
+    const float* kscale;
+    int64_t seq_stride_b, tok_stride_b, scale_seq_stride;
+    int d_I, block_size;
+    bool fp8;
+    float* kbar;
+    int64_t kbar_seq_stride;
+    int32_t* status;
+};
+
+struct BlockScoreArgs {
+    const int32_t* seq_len;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    int B, T, L_alloc;
+    const uint16_t* q;   // bf16 [T][H_I][d_I]
+    const float* w;      // [T][H_I]
+    const float* kbar;
+    int64_t kbar_seq_stride;
+    int d_I, block_size;
+    float* scores;
+    int64_t ld;
+    int n_cols;
+    int32_t* status;
+};
+
+struct TopkArgs {
+    const int32_t* seq_len;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    int B, T, L_alloc;
+    const float* scores;
+    int64_t ld;
+    int n_cols;
+    const int32_t* cand;
+    int n_cand, block_size;
+    int k, n_sink, window;
+    bool raw;
+    int32_t* idx;
+    int64_t ld_idx;
+    int32_t* count;
+    int32_t* status;
+};
+
+struct AttnArgs {
+    const int32_t* seq_len;
+    const int32_t* q_seq;
+    int B, T, L_alloc;
+    const uint16_t* q;          // [T][H][DQK] bf16
+    int H;
+    const uint8_t* kv;          // bytes
+    const float* kv_scale;
+    int64_t kv_seq_b, kv_tok_b, kv_scale_seq;
+    const uint8_t* v;           // separate V cache or NULL
+    const float* v_scale;
+    int64_t v_seq_b, v_tok_b, v_scale_seq;
+    const int32_t* idx;
+    int64_t ld_idx;
+    const int32_t* count;
+    float sm_scale_log2;        // sm_scale * log2(e)
+    int n_split;
+    uint16_t* o;                // [T][H][DV] bf16
+    float* lse;                 // [T][H] or NULL
+    float* part_o;              // [T][n_split][H][DV] (n_split > 1)
+    float* part_lse;            // [T][n_split][H]
+    int32_t* status;
+};
+
+cudaError_t launch_index_score(IndexArgs a, int H_I, int D_I, bool fp8, cudaStream_t st);
+cudaError_t launch_block_keys(const BlockKeyArgs& a, cudaStream_t st);
+cudaError_t launch_block_score(const BlockScoreArgs& a, int H_I, cudaStream_t st);
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
+cudaError_t launch_sparse_attn(const AttnArgs& a, int DQK, int DV, bool kv_fp8, bool sep_v, cudaStream_t st);
+
+}  // namespace lsa

@@ -1,0 +1,252 @@
+"""Python binding of the LSA C ABI (include/lsa.h): argument marshalling only.
+
+Every computation runs in the CUDA library ``_lsa.so``; this module turns torch tensors
+into the pointers, strides and structs the C functions take, and raises ``LsaError`` on
+a non-OK status.  There is no fallback: importing this module on a machine without the
+built library fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"LSA CUDA library not built: {LIB_PATH} (run python -m long_context_sparse_indexer_b200.build)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_DATA, ERR_TIMEOUT = range(7)
+BF16, FP8_E4M3, FP32 = 0, 1, 2
+TOPK_RAW = 1
+
+c_i32, c_i64, c_u32, c_f32, c_vp, c_size = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float,
+                                             ctypes.c_void_p, ctypes.c_size_t)
+
+
+class LsaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = _lib.lsa_status_string(status).decode()
+        super().__init__(f"{what}: {msg} (status {status})" if what else f"{msg} (status {status})")
+
+
+class CCache(ctypes.Structure):
+    _fields_ = [("data", c_vp), ("scale", c_vp), ("dtype", c_i32), ("dim", c_i32),
+                ("seq_stride", c_i64), ("tok_stride", c_i64), ("scale_seq_stride", c_i64)]
+
+
+class CBatch(ctypes.Structure):
+    _fields_ = [("B", c_i32), ("T", c_i32), ("q_group", c_i32), ("L_alloc", c_i32),
+                ("seq_len", c_vp), ("q_seq", c_vp), ("q_pos", c_vp)]
+
+
+class CLayer(ctypes.Structure):
+    _fields_ = [("q", c_vp), ("kv", CCache), ("v", CCache), ("o", c_vp), ("lse", c_vp)]
+
+
+class CDecodeParams(ctypes.Structure):
+    _fields_ = [("batch", CBatch), ("q_idx", c_vp), ("w", c_vp), ("H_I", c_i32), ("k_idx", CCache),
+                ("k", c_i32), ("n_sink", c_i32), ("window", c_i32),
+                ("hi", c_i32), ("block_size", c_i32), ("n_recall", c_i32), ("kbar", c_vp),
+                ("kbar_seq_stride", c_i64),
+                ("H", c_i32), ("Dqk", c_i32), ("Dv", c_i32), ("sm_scale", c_f32), ("n_split", c_i32),
+                ("n_layers", c_i32), ("layers", ctypes.POINTER(CLayer)),
+                ("idx_out", c_vp), ("idx_ld", c_i64), ("count_out", c_vp)]
+
+
+_P = ctypes.POINTER
+_lib.lsa_index_score.argtypes = [_P(CBatch), c_vp, c_vp, c_i32, _P(CCache), c_vp, c_i32, c_i32, c_vp, c_i64,
+                                 c_i32, c_vp, c_vp]
+_lib.lsa_block_keys.argtypes = [_P(CBatch), _P(CCache), c_i32, c_vp, c_i64, c_vp, c_vp]
+_lib.lsa_block_score.argtypes = [_P(CBatch), c_vp, c_vp, c_i32, c_i32, c_vp, c_i64, c_i32, c_vp, c_i64, c_i32,
+                                 c_vp, c_vp]
+_lib.lsa_topk.argtypes = [_P(CBatch), c_vp, c_i64, c_i32, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_u32, c_vp,
+                          c_i64, c_vp, c_vp, c_vp]
+_lib.lsa_sparse_attn.argtypes = [_P(CBatch), c_vp, c_i32, c_i32, _P(CCache), _P(CCache), c_i32, c_vp, c_i64, c_vp,
+                                 c_f32, c_i32, c_vp, c_vp, c_vp, c_size, c_vp, c_vp]
+_lib.lsa_attn_workspace_size.argtypes = [c_i32, c_i32, c_i32, c_i32]
+_lib.lsa_attn_workspace_size.restype = c_size
+_lib.lsa_decode_fused.argtypes = [_P(CDecodeParams), c_vp, c_size, c_vp, c_vp]
+_lib.lsa_decode_workspace_size.argtypes = [_P(CDecodeParams)]
+_lib.lsa_decode_workspace_size.restype = c_size
+_lib.lsa_read_device_status.argtypes = [c_vp, c_vp]
+_lib.lsa_status_string.argtypes = [c_i32]
+_lib.lsa_status_string.restype = ctypes.c_char_p
+_lib.lsa_version.restype = c_i32
+for _f in ("lsa_index_score", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
+           "lsa_decode_fused", "lsa_read_device_status"):
+    getattr(_lib, _f).restype = c_i32
+
+EXPORTS = ("lsa_index_score", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
+           "lsa_attn_workspace_size", "lsa_decode_fused", "lsa_decode_workspace_size", "lsa_read_device_status",
+           "lsa_status_string", "lsa_version")
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise LsaError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ------------------------------------------------------------------ descriptors
+
+@dataclass
+class Batch:
+    """Query tokens: q_seq / q_pos / seq_len are int32 device tensors."""
+    seq_len: torch.Tensor
+    q_seq: torch.Tensor
+    q_pos: torch.Tensor
+    L_alloc: int
+    q_group: int = 1
+
+    def c(self) -> CBatch:
+        return CBatch(int(self.seq_len.numel()), int(self.q_seq.numel()), int(self.q_group), int(self.L_alloc),
+                      _ptr(self.seq_len), _ptr(self.q_seq), _ptr(self.q_pos))
+
+
+@dataclass
+class Cache:
+    """A per-sequence cache [B, L_alloc, dim]: uint8 FP8 codes (+ float scale [B, L_alloc]) or bf16."""
+    data: torch.Tensor
+    scale: Optional[torch.Tensor] = None
+
+    @property
+    def dtype(self) -> int:
+        if self.data.dtype == torch.uint8 or self.data.dtype == torch.float8_e4m3fn:
+            return FP8_E4M3
+        if self.data.dtype == torch.bfloat16:
+            return BF16
+        raise ValueError(f"unsupported cache dtype {self.data.dtype}")
+
+    def c(self) -> CCache:
+        d = self.data
+        assert d.dim() == 3 and d.stride(2) == 1
+        sc = self.scale
+        sss = int(sc.stride(0)) if sc is not None else 0
+        return CCache(_ptr(d), _ptr(sc), self.dtype, int(d.shape[2]), int(d.stride(0)), int(d.stride(1)), sss)
+
+
+_EMPTY_CACHE = CCache(None, None, 0, 0, 0, 0, 0)
+
+
+# ------------------------------------------------------------------ entry points
+
+def index_score(batch: Batch, q_idx: torch.Tensor, w: torch.Tensor, k_idx: Cache, scores: torch.Tensor,
+                n_cols: int = 0, cand_blocks: Optional[torch.Tensor] = None, block_size: int = 0,
+                dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """lsa_index_score: flat scores (cand_blocks None) or HI fine scores over recalled blocks."""
+    cb, ck = batch.c(), k_idx.c()
+    n_cand = int(cand_blocks.shape[1]) if cand_blocks is not None else 0
+    _check(_lib.lsa_index_score(ctypes.byref(cb), _ptr(q_idx), _ptr(w), int(q_idx.shape[1]), ctypes.byref(ck),
+                                _ptr(cand_blocks), n_cand, int(block_size), _ptr(scores), int(scores.stride(0)),
+                                int(n_cols), _ptr(dev_status), _stream(stream)), "lsa_index_score")
+
+
+def block_keys(batch: Batch, k_idx: Cache, block_size: int, kbar: torch.Tensor,
+               dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    cb, ck = batch.c(), k_idx.c()
+    _check(_lib.lsa_block_keys(ctypes.byref(cb), ctypes.byref(ck), int(block_size), _ptr(kbar), int(kbar.stride(0)),
+                               _ptr(dev_status), _stream(stream)), "lsa_block_keys")
+
+
+def block_score(batch: Batch, q_idx: torch.Tensor, w: torch.Tensor, kbar: torch.Tensor, block_size: int,
+                scores: torch.Tensor, n_cols: int, dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    cb = batch.c()
+    _check(_lib.lsa_block_score(ctypes.byref(cb), _ptr(q_idx), _ptr(w), int(q_idx.shape[1]), int(q_idx.shape[2]),
+                                _ptr(kbar), int(kbar.stride(0)), int(block_size), _ptr(scores), int(scores.stride(0)),
+                                int(n_cols), _ptr(dev_status), _stream(stream)), "lsa_block_score")
+
+
+def topk(batch: Batch, scores: torch.Tensor, n_cols: int, k: int, n_sink: int, window: int, idx: torch.Tensor,
+         count: torch.Tensor, cand_blocks: Optional[torch.Tensor] = None, block_size: int = 0, raw: bool = False,
+         dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    cb = batch.c()
+    n_cand = int(cand_blocks.shape[1]) if cand_blocks is not None else 0
+    _check(_lib.lsa_topk(ctypes.byref(cb), _ptr(scores), int(scores.stride(0)), int(n_cols), _ptr(cand_blocks),
+                         n_cand, int(block_size), int(k), int(n_sink), int(window), TOPK_RAW if raw else 0,
+                         _ptr(idx), int(idx.stride(0)), _ptr(count), _ptr(dev_status), _stream(stream)), "lsa_topk")
+
+
+def attn_workspace_size(T: int, H: int, Dv: int, n_split: int) -> int:
+    return int(_lib.lsa_attn_workspace_size(T, H, Dv, n_split))
+
+
+def sparse_attn(batch: Batch, q: torch.Tensor, kv: Cache, idx: torch.Tensor, count: torch.Tensor, sm_scale: float,
+                o: torch.Tensor, lse: Optional[torch.Tensor] = None, v: Optional[Cache] = None, Dv: int = 0,
+                n_split: int = 1, ws: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                stream=None) -> None:
+    cb, ck = batch.c(), kv.c()
+    cv = v.c() if v is not None else None
+    H, Dqk = int(q.shape[1]), int(q.shape[2])
+    Dv = int(Dv or o.shape[2])
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.lsa_sparse_attn(ctypes.byref(cb), _ptr(q), H, Dqk, ctypes.byref(ck),
+                                ctypes.byref(cv) if cv is not None else None, Dv, _ptr(idx), int(idx.stride(0)),
+                                _ptr(count), float(sm_scale), int(n_split), _ptr(o), _ptr(lse), _ptr(ws), wsb,
+                                _ptr(dev_status), _stream(stream)), "lsa_sparse_attn")
+
+
+@dataclass
+class Layer:
+    q: torch.Tensor
+    kv: Cache
+    o: torch.Tensor
+    lse: Optional[torch.Tensor] = None
+    v: Optional[Cache] = None
+
+
+class DecodeStep:
+    """Marshalled parameters of lsa_decode_fused (built once, launched many times)."""
+
+    def __init__(self, batch: Batch, q_idx: torch.Tensor, w: torch.Tensor, k_idx: Cache, k: int, n_sink: int,
+                 window: int, layers: Sequence[Layer], H: int, Dqk: int, Dv: int, sm_scale: float, n_split: int = 1,
+                 hi: bool = False, block_size: int = 64, n_recall: int = 0, kbar: Optional[torch.Tensor] = None,
+                 idx_out: Optional[torch.Tensor] = None, count_out: Optional[torch.Tensor] = None):
+        self._keep = (batch, q_idx, w, k_idx, list(layers), kbar, idx_out, count_out)
+        arr = (CLayer * max(1, len(layers)))()
+        for i, L in enumerate(layers):
+            arr[i] = CLayer(_ptr(L.q), L.kv.c(), L.v.c() if L.v is not None else _EMPTY_CACHE, _ptr(L.o), _ptr(L.lse))
+        self._layers = arr
+        self.p = CDecodeParams(batch.c(), _ptr(q_idx), _ptr(w), int(q_idx.shape[1]), k_idx.c(), int(k), int(n_sink),
+                               int(window), int(bool(hi)), int(block_size), int(n_recall), _ptr(kbar),
+                               int(kbar.stride(0)) if kbar is not None else 0, int(H), int(Dqk), int(Dv),
+                               float(sm_scale), int(n_split), len(layers), arr, _ptr(idx_out),
+                               int(idx_out.stride(0)) if idx_out is not None else 0, _ptr(count_out))
+
+    def workspace_size(self) -> int:
+        return int(_lib.lsa_decode_workspace_size(ctypes.byref(self.p)))
+
+    def __call__(self, ws: torch.Tensor, dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+        _check(_lib.lsa_decode_fused(ctypes.byref(self.p), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _ptr(dev_status), _stream(stream)), "lsa_decode_fused")
+
+
+def read_device_status(dev_status: torch.Tensor, stream=None) -> int:
+    return int(_lib.lsa_read_device_status(_ptr(dev_status), _stream(stream)))
+
+
+def status_string(status: int) -> str:
+    return _lib.lsa_status_string(status).decode()
+
+
+def version() -> int:
+    return int(_lib.lsa_version())

@@ -1,0 +1,118 @@
+"""The C ABI without a GPU: every symbol of include/lsa.h is exported, host validation rejects bad calls."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from long_context_sparse_indexer_b200 import lsa
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "lsa.h")
+
+
+def declared():
+    txt = open(HDR).read()
+    return sorted(set(re.findall(r"^\s*(?:lsa_status|size_t|const char\*|int)\s+(lsa_\w+)\s*\(", txt, re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared()
+    assert len(names) >= 11
+    lib = lsa.library()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(lsa.EXPORTS)
+
+
+def test_status_strings_and_version():
+    assert lsa.version() == 1
+    for s in range(7):
+        assert lsa.status_string(s)
+    assert "unknown" in lsa.status_string(99)
+
+
+def _batch(T=1, B=1, q_group=1, L=100):
+    return lsa.CBatch(B, T, q_group, L, 16, 16, 16)        # fake device pointers: never dereferenced
+
+
+def _cache(dtype=lsa.FP8_E4M3, dim=128, scale=16, data=4096):
+    return lsa.CCache(data, scale, dtype, dim, 100 * dim, dim, 100)
+
+
+def test_index_score_rejects_bad_arguments():
+    lib = lsa.library()
+    b, c = _batch(), _cache()
+    call = lambda bb, cc, H_I=64, ld=100, n=100, q=16, w=16, sc=16: lib.lsa_index_score(  # noqa: E731
+        ctypes.byref(bb), q, w, H_I, ctypes.byref(cc), None, 0, 0, sc, ld, n, None, None)
+    assert call(b, c, H_I=48) == lsa.ERR_UNSUPPORTED
+    assert call(b, _cache(dim=96)) == lsa.ERR_UNSUPPORTED
+    assert call(b, _cache(scale=None)) == lsa.ERR_INVALID_ARG              # FP8 without scale
+    assert call(b, _cache(data=4097)) == lsa.ERR_INVALID_ARG               # misaligned rows
+    assert call(b, c, n=101) == lsa.ERR_INVALID_ARG                        # n_cols > ld
+    assert call(_batch(T=3, q_group=2), c) == lsa.ERR_INVALID_ARG          # T not a multiple of q_group
+    assert call(b, c, q=None) == lsa.ERR_INVALID_ARG
+    assert call(b, _cache(dtype=7)) == lsa.ERR_UNSUPPORTED
+    assert lib.lsa_index_score(None, 16, 16, 64, ctypes.byref(c), None, 0, 0, 16, 100, 100, None, None) \
+        == lsa.ERR_INVALID_ARG
+
+
+def test_topk_rejects_bad_arguments():
+    lib = lsa.library()
+    b = _batch()
+    call = lambda k=10, ns=4, win=8, ld_idx=22, flags=0, cand=None: lib.lsa_topk(  # noqa: E731
+        ctypes.byref(b), 16, 100, 100, cand, 1 if cand else 0, 64 if cand else 0, k, ns, win, flags, 16, ld_idx, 16,
+        None, None)
+    assert call(ld_idx=21) == lsa.ERR_INVALID_ARG                          # capacity below k + sinks + window
+    assert call(k=-1) == lsa.ERR_INVALID_ARG
+    assert call(flags=lsa.TOPK_RAW) == lsa.ERR_INVALID_ARG                 # raw mode takes no sinks/window
+    assert call(flags=8) == lsa.ERR_UNSUPPORTED
+
+
+def test_attention_rejects_bad_arguments():
+    lib = lsa.library()
+    b = _batch()
+    kv = _cache(dtype=lsa.BF16, dim=576, scale=None)
+    call = lambda H=128, Dqk=576, Dv=512, ns=1, ws=None, wsb=0, scale=0.04, kvc=kv: lib.lsa_sparse_attn(  # noqa
+        ctypes.byref(b), 4096, H, Dqk, ctypes.byref(kvc), None, Dv, 16, 100, 16, scale, ns, 4096, 16, ws, wsb, None,
+        None)
+    assert call(H=100) == lsa.ERR_UNSUPPORTED
+    assert call(Dv=256) == lsa.ERR_UNSUPPORTED
+    assert call(ns=0) == lsa.ERR_INVALID_ARG
+    assert call(ns=65) == lsa.ERR_INVALID_ARG
+    assert call(scale=float("nan")) == lsa.ERR_INVALID_ARG
+    assert call(ns=4) == lsa.ERR_WORKSPACE                                 # split partials need a workspace
+    need = lsa.attn_workspace_size(1, 128, 512, 4)
+    assert need >= 4 * 128 * 512 * 4
+    assert call(ns=4, ws=4096, wsb=need - 1) == lsa.ERR_WORKSPACE
+    assert lsa.attn_workspace_size(5, 128, 512, 1) == 0
+
+
+def test_fused_rejects_bad_arguments():
+    lib = lsa.library()
+    p = lsa.CDecodeParams()
+    p.batch = _batch()
+    p.k, p.n_sink, p.window = 10, 4, 8
+    p.H_I = 64
+    p.k_idx = _cache()
+    p.n_layers = 1
+    p.layers = None
+    assert lib.lsa_decode_fused(ctypes.byref(p), 4096, 1 << 30, None, None) == lsa.ERR_INVALID_ARG
+    p.n_layers = 0
+    p.hi, p.block_size, p.n_recall = 1, 64, 0
+    assert lib.lsa_decode_fused(ctypes.byref(p), 4096, 1 << 30, None, None) == lsa.ERR_INVALID_ARG
+    p.hi = 0
+    need = lib.lsa_decode_workspace_size(ctypes.byref(p))
+    assert need > 0
+    assert lib.lsa_decode_fused(ctypes.byref(p), 4096, need - 1, None, None) == lsa.ERR_WORKSPACE
+    assert lib.lsa_decode_fused(ctypes.byref(p), 4097, need, None, None) == lsa.ERR_WORKSPACE
+
+
+def test_binding_refuses_to_run_without_cuda_library_on_missing_build(tmp_path, monkeypatch):
+    import importlib
+    import long_context_sparse_indexer_b200.lsa as mod
+    monkeypatch.setattr(os.path, "exists", lambda p: False if p.endswith("_lsa.so") else os.path.isfile(p))
+    with pytest.raises(ImportError):
+        importlib.reload(mod)
+    monkeypatch.undo()
+    importlib.reload(mod)

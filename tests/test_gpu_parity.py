@@ -1,0 +1,359 @@
+"""GPU parity: the CUDA library against the float64 CPU oracle on the same seeded inputs.
+
+Tolerances (from the definitions of the path and its precision):
+* indexer / block scores: relative 1e-3, with a floor at 1% of the row's RMS score for
+  entries near zero (ReLU sums of cancelling dot products);
+* top-k: exact index lists when the selection runs on identical scores; >= 99.9% overlap
+  against the oracle's own float64 scores;
+* attention (BF16 output): max-abs 1e-2 and relative L2 5e-3;
+* determinism: bitwise identical outputs across runs at a fixed n_split.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from lsa_synth import device as D
+from lsa_synth import gen
+from lsa_synth import workloads as W
+from oracle import formats, lsa as olsa, run
+
+from long_context_sparse_indexer_b200 import lsa
+
+from . import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny_decode": W.WORKLOADS["tiny_decode"],
+    "cli_small": W.scaled("decode_cli_128k", B=3, len_lo=2500, len_hi=5200),
+    "mtp_small": W.scaled("mtp_256k", B=2, len_lo=3001, len_hi=3001),
+    "prefill_small": W.scaled("prefill_32k", len_lo=3000, len_hi=3000, passes=(W._target_pass(64, 1),)),
+    "hi_small": W.scaled("decode_hi_1m", B=2, len_lo=20000, len_hi=20000),
+}
+FLAT = ["tiny_decode", "cli_small", "mtp_small", "prefill_small"]
+
+_cache = {}
+
+
+def wt_of(name):
+    if name not in _cache:
+        _cache[name] = D.build_workload(SMALL[name], "cuda")
+    return _cache[name]
+
+
+def tokens_to_check(w, p, limit=6):
+    T = w.T(p)
+    if T <= limit:
+        return list(range(T))
+    return sorted({0, 1, T // 2, T - 2, T - 1})
+
+
+# ------------------------------------------------------------------ inputs
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_device_inputs_match_host_generator(cuda, name):
+    w = SMALL[name]
+    wt = wt_of(name)
+    plan = None
+    for pi, p in enumerate(w.passes):
+        pt = wt.passes[pi]
+        T = w.T(p)
+        assert np.array_equal(pt.q_idx.view(torch.int16).cpu().numpy().view(np.uint16), W.idx_q_bits(w, p))
+        assert np.array_equal(pt.w.cpu().numpy(), W.idx_w(w, p))
+        if p.name == "target" and (w.plant_frac or w.plant_blocks):
+            plan = W.plant_plan(w, p)
+        for b in range(w.B):
+            L = int(W.lengths(w)[b])
+            rows = np.unique(np.concatenate([np.arange(0, 70), np.arange(L - 70, L),
+                                             plan[0][b][:50] if plan is not None and p.name == "target"
+                                             else np.zeros(0, np.int64)]))
+            data, scale = W.idx_key_rows(w, p, b, rows, plan if p.name == "target" else None)
+            got = pt.k_idx[b, torch.from_numpy(rows).cuda()].cpu()
+            if scale is None:
+                assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), data)
+            else:
+                assert np.array_equal(got.numpy(), data)
+                assert np.array_equal(pt.k_scale[b, torch.from_numpy(rows).cuda()].cpu().numpy(), scale)
+            for li, layer in enumerate(p.layers):
+                kd, ks = W.kv_rows(w, layer.tid_kv, b, rows[:20], w.D)
+                g = pt.layers[li]["kv"][b, torch.from_numpy(rows[:20]).cuda()].cpu()
+                if ks is None:
+                    assert np.array_equal(g.view(torch.int16).numpy().view(np.uint16), kd)
+                else:
+                    assert np.array_equal(g.numpy(), kd)
+        toks = [0, T - 1]
+        for li, layer in enumerate(p.layers):
+            got = pt.layers[li]["q"][toks].view(torch.int16).cpu().numpy().view(np.uint16)
+            assert np.array_equal(got, W.attn_q_bits(w, layer, toks))
+
+
+# ------------------------------------------------------------------ indexer scores
+
+@pytest.mark.parametrize("name", FLAT)
+def test_flat_index_scores(cuda, name):
+    w = SMALL[name]
+    wt = wt_of(name)
+    for pi, p in enumerate(w.passes):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sc = H.flat_scores(wt, pi, st).cpu().numpy().astype(np.float64)
+        assert lsa.read_device_status(st) == lsa.OK
+        q_seq, q_pos = W.query_rows(w, p)
+        plan = W.plant_plan(w, p) if p.name == "target" and (w.plant_frac or w.plant_blocks) else None
+        for t in tokens_to_check(w, p):
+            b, pos, L, qi, wi = run.query_context(w, p, t)
+            K = run.index_keys(w, p, b, np.arange(pos + 1), plan)
+            ref = olsa.indexer_scores(qi, wi, K)
+            assert H.score_close(sc[t, :pos + 1], ref) < 1e-3
+            assert np.all(np.isneginf(sc[t, pos + 1:wt.L_alloc]))
+
+
+def test_block_keys_and_block_scores(cuda):
+    w = SMALL["hi_small"]
+    wt = wt_of("hi_small")
+    p = w.passes[0]
+    kbar_dev = H.block_keys(wt)
+    kbar = kbar_dev.cpu().numpy().astype(np.float64)
+    plan = W.plant_plan(w, p)
+    nblk = kbar.shape[1]
+    bsc = torch.empty((w.B, (nblk + 3) // 4 * 4), dtype=torch.float32, device="cuda")
+    lsa.block_score(H.batch_of(wt), wt.passes[0].q_idx, wt.passes[0].w, kbar_dev, w.block_size, bsc, nblk)
+    bsc = bsc.cpu().numpy().astype(np.float64)
+    for t in range(w.T(p)):
+        b, pos, L, qi, wi = run.query_context(w, p, t)
+        ref_kbar = run.block_keys_of_sequence(w, p, b, L, plan)
+        rel = np.abs(kbar[b, :ref_kbar.shape[0]] - ref_kbar).max() / np.abs(ref_kbar).max()
+        assert rel < 1e-5
+        nvis = pos // w.block_size + 1
+        J = olsa.indexer_scores(qi, wi, ref_kbar[:nvis])
+        assert H.score_close(bsc[t, :nvis], J) < 1e-3
+        assert np.all(np.isneginf(bsc[t, nvis:nblk]))
+
+
+# ------------------------------------------------------------------ top-k in isolation
+
+def _host_score_rows(rng, T, n_cols, tie_levels):
+    s = rng.integers(0, tie_levels, size=(T, n_cols)).astype(np.float32) * np.float32(0.25)
+    s[:, ::7] = rng.normal(size=(T, (n_cols + 6) // 7)).astype(np.float32)
+    s[:, 3::11] = -0.0
+    s[:, 5::13] = -np.inf
+    return s
+
+
+@pytest.mark.parametrize("n_cols,k,n_sink,window,tie_levels", [
+    (5000, 256, 4, 128, 3), (5000, 256, 4, 128, 1000), (3000, 2048, 4, 512, 5), (100, 300, 4, 16, 2),
+    (70000, 2048, 4, 512, 50), (4097, 0, 4, 128, 3), (4097, 33, 0, 0, 4),
+])
+def test_topk_matches_oracle_exactly(cuda, n_cols, k, n_sink, window, tie_levels):
+    rng = np.random.default_rng(n_cols + k)
+    T = 5
+    s = _host_score_rows(rng, T, n_cols, tie_levels)
+    pos = np.array([n_cols - 1, n_cols // 2, 10, min(n_cols - 1, 3), n_cols - 2])
+    s_masked = s.copy()
+    for t in range(T):
+        s_masked[t, pos[t] + 1:] = -np.inf
+    batch = lsa.Batch(torch.tensor([n_cols], dtype=torch.int32, device="cuda"),
+                      torch.zeros(T, dtype=torch.int32, device="cuda"),
+                      torch.from_numpy(pos.astype(np.int32)).cuda(), n_cols)
+    cap = k + n_sink + window
+    idx = torch.empty((T, max(cap, 1)), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(T, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.topk(batch, torch.from_numpy(s_masked).cuda(), n_cols, k, n_sink, window, idx, cnt, dev_status=st)
+    assert lsa.read_device_status(st) == lsa.OK
+    got = H.index_lists(idx, cnt)
+    for t in range(T):
+        valid = ~np.isneginf(s_masked[t])
+        cols = np.nonzero(valid)[0]
+        picks = olsa.topk(s_masked[t, cols].astype(np.float64), cols, k)
+        want = olsa.union_fixed(picks, int(pos[t]), n_sink, window)
+        assert got[t].tolist() == want.tolist()
+        assert np.all(idx[t, cnt[t]:].cpu().numpy() == -1)
+
+
+def test_topk_raw_and_candidate_blocks(cuda):
+    rng = np.random.default_rng(1)
+    T, bs, n_cand = 3, 64, 40
+    blocks = np.stack([np.sort(rng.choice(500, size=n_cand, replace=False)) for _ in range(T)])
+    blocks[2, -5:] = -1                                     # unused tail
+    pos = np.array([500 * 64 - 1, 250 * 64 + 17, 30000])
+    s = rng.integers(0, 20, size=(T, n_cand * bs)).astype(np.float32)
+    for t in range(T):
+        p_of_col = (blocks[t][:, None] * bs + np.arange(bs)[None, :]).reshape(-1)
+        bad = (np.repeat(blocks[t], bs) < 0) | (p_of_col > pos[t])
+        s[t, bad] = -np.inf
+    batch = lsa.Batch(torch.tensor([500 * 64], dtype=torch.int32, device="cuda"),
+                      torch.zeros(T, dtype=torch.int32, device="cuda"), torch.from_numpy(pos.astype(np.int32)).cuda(),
+                      500 * 64)
+    cb = torch.from_numpy(blocks.astype(np.int32)).cuda()
+    k, ns, win = 300, 4, 100
+    idx = torch.empty((T, k + ns + win), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(T, dtype=torch.int32, device="cuda")
+    sd = torch.from_numpy(s).cuda()
+    lsa.topk(batch, sd, n_cand * bs, k, ns, win, idx, cnt, cand_blocks=cb, block_size=bs)
+    got = H.index_lists(idx, cnt)
+    raw_idx = torch.empty((T, 50), dtype=torch.int32, device="cuda")
+    lsa.topk(batch, sd, n_cand * bs, 50, 0, 0, raw_idx, cnt, raw=True)
+    got_raw = H.index_lists(raw_idx, cnt)
+    for t in range(T):
+        p_of_col = (blocks[t][:, None] * bs + np.arange(bs)[None, :]).reshape(-1)
+        valid = ~np.isneginf(s[t])
+        picks = olsa.topk(s[t, valid].astype(np.float64), p_of_col[valid], k)
+        assert got[t].tolist() == olsa.union_fixed(picks, int(pos[t]), ns, win).tolist()
+        cols = np.nonzero(valid)[0]
+        assert got_raw[t].tolist() == sorted(olsa.topk(s[t, valid].astype(np.float64), cols, 50).tolist())
+
+
+# ------------------------------------------------------------------ attention in isolation
+
+@pytest.mark.parametrize("name", ["tiny_decode", "cli_small", "mtp_small"])
+@pytest.mark.parametrize("n_split", [1, 3, 7])
+def test_attention_on_oracle_index(cuda, name, n_split):
+    w = SMALL[name]
+    wt = wt_of(name)
+    p = w.passes[0]
+    toks = tokens_to_check(w, p, limit=4)
+    T = w.T(p)
+    plan = W.plant_plan(w, p) if (w.plant_frac or w.plant_blocks) else None
+    lists = {t: run.index_list(w, p, t, plan)[0] for t in toks}
+    cap = w.cap
+    idx = torch.full((T, cap), -1, dtype=torch.int32)
+    cnt = torch.zeros(T, dtype=torch.int32)
+    for t, l in lists.items():
+        idx[t, :len(l)] = torch.from_numpy(l.astype(np.int32))
+        cnt[t] = len(l)
+    idx, cnt = idx.cuda(), cnt.cuda()
+    batch = H.batch_of(wt)
+    for li, layer in enumerate(p.layers):
+        kv, v = H.kv_cache(wt, 0, li)
+        q = wt.passes[0].layers[li]["q"]
+        o = torch.empty((T, w.H, w.Dv), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
+        ws = torch.empty(max(256, lsa.attn_workspace_size(T, w.H, w.Dv, n_split)), dtype=torch.uint8, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        lsa.sparse_attn(batch, q, kv, idx, cnt, w.sm_scale, o, lse, v=v, n_split=n_split, ws=ws, dev_status=st)
+        assert lsa.read_device_status(st) == lsa.OK
+        on, ln = H.bf16_to_np(o), lse.cpu().numpy()
+        for t in toks:
+            o_ref, lse_ref = run.attend(w, p, layer, t, lists[t])
+            mx, rl2 = H.attn_errors(on[t], o_ref)
+            assert mx < 1e-2 and rl2 < 5e-3, (t, mx, rl2)
+            assert np.abs(ln[t] - lse_ref).max() < 1e-3 * max(1.0, np.abs(lse_ref).max())
+
+
+# ------------------------------------------------------------------ whole path
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_fused_path_end_to_end(cuda, name):
+    w = SMALL[name]
+    wt = wt_of(name)
+    for pi, p in enumerate(w.passes):
+        step, ws, idx, cnt, layers = H.decode_step(wt, pi, n_split=3)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        step(ws, st)
+        assert lsa.read_device_status(st) == lsa.OK
+        got = H.index_lists(idx, cnt)
+        plan = W.plant_plan(w, p) if p.name == "target" and (w.plant_frac or w.plant_blocks) else None
+        outs = [(H.bf16_to_np(L.o), L.lse.cpu().numpy()) for L in layers]
+        for t in tokens_to_check(w, p, limit=4):
+            ref = run.run_query(w, p, t, plan)
+            a, b = set(got[t].tolist()), set(ref["idx"].tolist())
+            assert len(a & b) >= 0.999 * len(b) and len(a) == len(b), (t, len(a), len(b), len(a & b))
+            assert np.all(np.diff(got[t]) > 0)
+            if a == b:
+                for li, (o_ref, lse_ref) in enumerate(ref["layers"]):
+                    mx, rl2 = H.attn_errors(outs[li][0][t], o_ref)
+                    assert mx < 1e-2 and rl2 < 5e-3, (t, li, mx, rl2)
+
+
+@pytest.mark.parametrize("name", FLAT)
+def test_oracle_selection_on_gpu_scores_is_bit_exact(cuda, name):
+    """The oracle's top-k + union, run on the GPU's own scores, gives the GPU's index list exactly."""
+    w = SMALL[name]
+    wt = wt_of(name)
+    for pi, p in enumerate(w.passes):
+        sc = H.flat_scores(wt, pi).cpu().numpy().astype(np.float64)
+        step, ws, idx, cnt, _ = H.decode_step(wt, pi)
+        step(ws)
+        got = H.index_lists(idx, cnt)
+        _, q_pos = W.query_rows(w, p)
+        for t in range(w.T(p)):
+            pos = int(q_pos[t])
+            picks = olsa.topk(sc[t, :pos + 1], np.arange(pos + 1), w.k)
+            assert got[t].tolist() == olsa.union_fixed(picks, pos, w.n_sink, w.window).tolist()
+
+
+@pytest.mark.parametrize("name", ["cli_small", "hi_small", "mtp_small"])
+def test_two_runs_bitwise_identical(cuda, name):
+    wt = wt_of(name)
+    res = []
+    for _ in range(2):
+        step, ws, idx, cnt, layers = H.decode_step(wt, 0, n_split=4)
+        step(ws)
+        torch.cuda.synchronize()
+        res.append([idx.cpu(), cnt.cpu()] + [L.o.cpu() for L in layers] + [L.lse.cpu() for L in layers])
+    for x, y in zip(*res):
+        assert torch.equal(x.view(torch.uint8) if x.dtype == torch.bfloat16 else x,
+                           y.view(torch.uint8) if y.dtype == torch.bfloat16 else y)
+
+
+def test_split_count_invariance(cuda):
+    wt = wt_of("cli_small")
+    outs = {}
+    for ns in (1, 2, 5, 16):
+        step, ws, idx, cnt, layers = H.decode_step(wt, 0, n_split=ns)
+        step(ws)
+        outs[ns] = [H.bf16_to_np(L.o) for L in layers]
+    for ns in (2, 5, 16):
+        for a, b in zip(outs[1], outs[ns]):
+            mx, rl2 = H.attn_errors(a, b.astype(np.float64))
+            assert mx < 1e-2 and rl2 < 5e-3
+
+
+def test_hi_with_every_block_recalled_equals_flat(cuda):
+    base = SMALL["hi_small"]
+    w_all = W.scaled("decode_hi_1m", B=2, len_lo=20000, len_hi=20000, n_recall=400)
+    w_flat = W.scaled("decode_hi_1m", B=2, len_lo=20000, len_hi=20000, hi=False)
+    wt = wt_of("hi_small")
+    res = []
+    for w in (w_all, w_flat):
+        wt2 = D.WorkloadTensors(w, wt.L_alloc, wt.seq_len, wt.passes)
+        step, ws, idx, cnt, _ = H.decode_step(wt2, 0)
+        step(ws)
+        res.append(H.index_lists(idx, cnt))
+    assert all(a.tolist() == b.tolist() for a, b in zip(*res))
+    assert base.n_recall == 256
+
+
+# ------------------------------------------------------------------ device-side data errors
+
+def test_device_data_errors_are_reported(cuda):
+    wt = wt_of("cli_small")
+    pt = wt.passes[0]
+    bad_pos = pt.q_pos.clone()
+    bad_pos[1] = wt.L_alloc + 5
+    batch = lsa.Batch(wt.seq_len, pt.q_seq, bad_pos, wt.L_alloc)
+    sc = torch.empty((pt.q_idx.shape[0], wt.L_alloc), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.index_score(batch, pt.q_idx, pt.w, H.idx_cache(wt), sc, n_cols=wt.L_alloc, dev_status=st)
+    assert lsa.read_device_status(st) == lsa.ERR_DEVICE_DATA
+    # NaN score
+    good = H.batch_of(wt)
+    sc = H.flat_scores(wt)
+    sc[0, 3] = float("nan")
+    idx = torch.empty((sc.shape[0], 2564), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc.shape[0], dtype=torch.int32, device="cuda")
+    st.zero_()
+    lsa.topk(good, sc, wt.L_alloc, 2048, 4, 512, idx, cnt, dev_status=st)
+    assert lsa.read_device_status(st) == lsa.ERR_DEVICE_DATA
+    # index outside the sequence
+    st.zero_()
+    sc = H.flat_scores(wt)
+    lsa.topk(good, sc, wt.L_alloc, 2048, 4, 512, idx, cnt)
+    idx[0, 5] = 10 ** 7
+    kv, _ = H.kv_cache(wt, 0, 0)
+    o = torch.empty((sc.shape[0], 128, 512), dtype=torch.bfloat16, device="cuda")
+    lsa.sparse_attn(good, pt.layers[0]["q"], kv, idx, cnt, 0.04, o, dev_status=st)
+    assert lsa.read_device_status(st) == lsa.ERR_DEVICE_DATA
+    torch.cuda.synchronize()
