@@ -127,9 +127,9 @@ def build_step(w, wt, pi, n_split):
     return dict(step=step, ws=ws, idx=idx, cnt=cnt, layers=layers, batch=batch, kbar=kbar, T=T, n_split=n_split)
 
 
-def launches_per_step(w, n_split):
+def launches_per_step(w, splits):
     per = 0
-    for p in w.passes:
+    for p, n_split in zip(w.passes, splits):
         per += 4 if w.hi else 2
         per += len(p.layers) * (2 if n_split > 1 else 1)
     return per
@@ -196,8 +196,10 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = W.WORKLOADS[args.workload]
+    if args.batch:
+        w = W.scaled(args.workload, B=args.batch)
     if world > 1:
-        w = W.scaled(args.workload, seed=w.seed + 1000 * rank)
+        w = W.scaled(args.workload, B=w.B, seed=w.seed + 1000 * rank)
     wt = D.build_workload(w, dev)
     stream = torch.cuda.current_stream()
     sds = [build_step(w, wt, pi, launch.split_for(w.T(p), w.H)) for pi, p in enumerate(w.passes)]
@@ -317,7 +319,7 @@ def run_gpu(args, rank, world, local_rank):
                      "launch_ms": kms, "algorithmic_bytes_per_launch": idx_bytes},
         "e2e": {"value": q_per_step * world / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": launches_per_step(w, sds[0]["n_split"]) * args.steps,
+        "gpu_launches": launches_per_step(w, [sd["n_split"] for sd in sds]) * args.steps,
         "clocks": clk.summary(),
     }
     return res, w, wt
@@ -388,6 +390,7 @@ def main():
     ap.add_argument("--workload", default="decode_cli_128k", choices=list(W.WORKLOADS))
     ap.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the sequence count (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

@@ -168,6 +168,31 @@ lsa_status lsa_sparse_attn(const lsa_batch* batch, const void* q, int H, int Dqk
 
 size_t lsa_attn_workspace_size(int T, int H, int Dv, int n_split);
 
+/* ---------------------------------------------------------------- sparse attention without allocation
+ * The pages have no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory (a serving runtime whose memory pool forbids new allocations, a
+ * plugin host that owns every cudaMalloc) and so cannot provide lsa_sparse_attn's
+ * workspace.  Same arguments, results and determinism as lsa_sparse_attn, minus the
+ * workspace: the split-KV partials live in one static device array of
+ * LSA_NOALLOC_SCRATCH_BYTES inside this library, which every GPU that loads the library
+ * holds until the process exits.  The call allocates nothing.
+ *   - Returns LSA_ERR_WORKSPACE when lsa_attn_workspace_size(T, H, Dv, n_split) exceeds
+ *     LSA_NOALLOC_SCRATCH_BYTES (at Dv = 512: T * n_split * H at most 16,352);
+ *     n_split == 1 needs no scratch.
+ *   - The first call with n_split > 1 on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents; nothing in
+ *     it needs to start at zero (each call writes every partial it reads).  Calls whose
+ *     execution overlaps on the GPU (other streams, other threads, concurrent graphs)
+ *     race on the array and corrupt each other's results: serialise them. */
+#define LSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+lsa_status lsa_sparse_attn_noalloc(const lsa_batch* batch, const void* q, int H, int Dqk,
+                                   const lsa_cache* kv, const lsa_cache* v, int Dv,
+                                   const int32_t* idx, int64_t ld_idx, const int32_t* count,
+                                   float sm_scale, int n_split, void* o, float* lse,
+                                   int32_t* dev_status, void* stream);
+
 /* ---------------------------------------------------------------- fused decode / prefill step
  * One attention layer consuming a shared index list (cross-layer indexing: [release] CLI
  * bullet, one index serves consecutive layers; MTP paragraph, draft steps 2 and 3 reuse

@@ -70,6 +70,8 @@ _lib.lsa_topk.argtypes = [_P(CBatch), c_vp, c_i64, c_i32, c_vp, c_i32, c_i32, c_
                           c_i64, c_vp, c_vp, c_vp]
 _lib.lsa_sparse_attn.argtypes = [_P(CBatch), c_vp, c_i32, c_i32, _P(CCache), _P(CCache), c_i32, c_vp, c_i64, c_vp,
                                  c_f32, c_i32, c_vp, c_vp, c_vp, c_size, c_vp, c_vp]
+_lib.lsa_sparse_attn_noalloc.argtypes = [_P(CBatch), c_vp, c_i32, c_i32, _P(CCache), _P(CCache), c_i32, c_vp, c_i64,
+                                         c_vp, c_f32, c_i32, c_vp, c_vp, c_vp, c_vp]
 _lib.lsa_attn_workspace_size.argtypes = [c_i32, c_i32, c_i32, c_i32]
 _lib.lsa_attn_workspace_size.restype = c_size
 _lib.lsa_decode_fused.argtypes = [_P(CDecodeParams), c_vp, c_size, c_vp, c_vp]
@@ -80,11 +82,11 @@ _lib.lsa_status_string.argtypes = [c_i32]
 _lib.lsa_status_string.restype = ctypes.c_char_p
 _lib.lsa_version.restype = c_i32
 for _f in ("lsa_index_score", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
-           "lsa_decode_fused", "lsa_read_device_status"):
+           "lsa_sparse_attn_noalloc", "lsa_decode_fused", "lsa_read_device_status"):
     getattr(_lib, _f).restype = c_i32
 
 EXPORTS = ("lsa_index_score", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
-           "lsa_attn_workspace_size", "lsa_decode_fused", "lsa_decode_workspace_size", "lsa_read_device_status",
+           "lsa_sparse_attn_noalloc", "lsa_attn_workspace_size", "lsa_decode_fused", "lsa_decode_workspace_size", "lsa_read_device_status",
            "lsa_status_string", "lsa_version")
 
 
@@ -203,6 +205,28 @@ def sparse_attn(batch: Batch, q: torch.Tensor, kv: Cache, idx: torch.Tensor, cou
                                 ctypes.byref(cv) if cv is not None else None, Dv, _ptr(idx), int(idx.stride(0)),
                                 _ptr(count), float(sm_scale), int(n_split), _ptr(o), _ptr(lse), _ptr(ws), wsb,
                                 _ptr(dev_status), _stream(stream)), "lsa_sparse_attn")
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def sparse_attn_noalloc(batch: Batch, q: torch.Tensor, kv: Cache, idx: torch.Tensor, count: torch.Tensor,
+                        sm_scale: float, o: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                        v: Optional[Cache] = None, Dv: int = 0, n_split: int = 1,
+                        dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """lsa_sparse_attn_noalloc: sparse_attn for callers that cannot allocate device memory.
+
+    The split partials live in the library's static device scratch array (32 MiB per GPU,
+    shared by every call, so calls must not overlap on the GPU); nothing is allocated.
+    """
+    cb, ck = batch.c(), kv.c()
+    cv = v.c() if v is not None else None
+    H, Dqk = int(q.shape[1]), int(q.shape[2])
+    Dv = int(Dv or o.shape[2])
+    _check(_lib.lsa_sparse_attn_noalloc(ctypes.byref(cb), _ptr(q), H, Dqk, ctypes.byref(ck),
+                                        ctypes.byref(cv) if cv is not None else None, Dv, _ptr(idx),
+                                        int(idx.stride(0)), _ptr(count), float(sm_scale), int(n_split), _ptr(o),
+                                        _ptr(lse), _ptr(dev_status), _stream(stream)), "lsa_sparse_attn_noalloc")
 
 
 @dataclass
