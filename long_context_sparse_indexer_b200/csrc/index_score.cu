@@ -268,6 +268,7 @@ cudaError_t launch_index_score(IndexArgs a, int H_I, int D_I, bool fp8, cudaStre
     else a.group = a.q_group < kIdxMaxGroup ? a.q_group : (a.q_group % kIdxMaxGroup == 0 ? kIdxMaxGroup
                                                            : (a.q_group % 2 == 0 ? 2 : 1));
     if (a.n_cols <= 0 || a.T <= 0) return cudaSuccess;
+    if (index_score_tc_supported(a, H_I, D_I, fp8)) return launch_index_score_tc(a, H_I, st);
     if (fp8) return D_I == 64 ? launch_index_d<true, 64>(a, H_I, st) : launch_index_d<true, 128>(a, H_I, st);
     return D_I == 64 ? launch_index_d<false, 64>(a, H_I, st) : launch_index_d<false, 128>(a, H_I, st);
 }

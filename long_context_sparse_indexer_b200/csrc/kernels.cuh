@@ -96,6 +96,8 @@ struct AttnArgs {
 };
 
 cudaError_t launch_index_score(IndexArgs a, int H_I, int D_I, bool fp8, cudaStream_t st);
+bool index_score_tc_supported(const IndexArgs& a, int H_I, int D_I, bool fp8);
+cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st);
 cudaError_t launch_block_keys(const BlockKeyArgs& a, cudaStream_t st);
 cudaError_t launch_block_score(const BlockScoreArgs& a, int H_I, cudaStream_t st);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
