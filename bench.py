@@ -202,7 +202,7 @@ def run_gpu(args, rank, world, local_rank):
         w = W.scaled(args.workload, B=w.B, seed=w.seed + 1000 * rank)
     wt = D.build_workload(w, dev)
     stream = torch.cuda.current_stream()
-    sds = [build_step(w, wt, pi, launch.split_for(w.T(p), w.H)) for pi, p in enumerate(w.passes)]
+    sds = [build_step(w, wt, pi, launch.split_for(w.T(p), w.H, w.cap)) for pi, p in enumerate(w.passes)]
 
     def step():
         for sd in sds:

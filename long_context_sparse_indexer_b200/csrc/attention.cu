@@ -346,6 +346,13 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
 // separate BF16 V cache, H % 16 == 0.
 cudaError_t launch_sparse_attn(const AttnArgs& a, int DQK, int DV, bool kv_fp8, bool sep_v, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
+    if (sparse_attn_tc_supported(a, DQK, DV, sep_v)) {
+        cudaError_t e = launch_sparse_attn_tc(a, kv_fp8, st);
+        if (e != cudaSuccess || a.n_split == 1) return e;
+        dim3 mg(a.H, a.T);
+        merge_kernel<<<mg, DV / 4, 0, st>>>(a.part_o, a.part_lse, a.n_split, a.H, DV, a.o, a.lse);
+        return cudaGetLastError();
+    }
     if (DQK == 576 && DV == 512 && !sep_v)
         return kv_fp8 ? launch_attn_t<576, 512, 2, true, false>(a, st) : launch_attn_t<576, 512, 2, false, false>(a, st);
     if (DQK == 128 && DV == 128 && sep_v && !kv_fp8) return launch_attn_t<128, 128, 1, false, true>(a, st);

@@ -102,5 +102,7 @@ cudaError_t launch_block_keys(const BlockKeyArgs& a, cudaStream_t st);
 cudaError_t launch_block_score(const BlockScoreArgs& a, int H_I, cudaStream_t st);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int DQK, int DV, bool kv_fp8, bool sep_v, cudaStream_t st);
+bool sparse_attn_tc_supported(const AttnArgs& a, int DQK, int DV, bool sep_v);
+cudaError_t launch_sparse_attn_tc(const AttnArgs& a, bool kv_fp8, cudaStream_t st);
 
 }  // namespace lsa

@@ -119,6 +119,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// 32 lanes x 16 columns of 32-bit.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+           "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 // ---------------------------------------------------------------- UMMA descriptors and issue
 
 // Instruction descriptor of kind::f16: D f32, A/B f16 (fmt 0) or bf16 (fmt 1), both K-major.
@@ -128,6 +138,22 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_fmt) {
          | ((uint32_t)ab_fmt << 10)            // B format
          | ((uint32_t)(N >> 3) << 17)          // N / 8
          | ((uint32_t)(M >> 4) << 24);         // M / 16
+}
+
+// Instruction descriptor of kind::f16 with B in MN-major layout (A K-major, from TMEM or smem).
+__host__ __device__ constexpr uint32_t idesc_f16_bmn(int M, int N, int ab_fmt) {
+    return idesc_f16(M, N, ab_fmt) | (1u << 16);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, explicit leading / stride byte offsets.
+__device__ __forceinline__ uint64_t sdesc_sw128_lbo(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
 }
 
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups 1024 B apart.
