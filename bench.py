@@ -59,7 +59,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -236,6 +236,7 @@ def run_gpu(args, rank, world, local_rank):
         dist.barrier()
     with ClockSampler(local_rank) as clk:
         torch.cuda.synchronize()
+        time.sleep(0.05)                     # let the sampler start before the timed region
         ms = time_region(fn, args.steps, stream)
     if world > 1:
         dist.barrier()
@@ -385,7 +386,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode_cli_128k", choices=list(W.WORKLOADS))
     ap.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
