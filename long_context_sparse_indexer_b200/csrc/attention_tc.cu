@@ -9,10 +9,12 @@
 // the duplicated QK^T keeps every CTA independent (no cross-CTA exchange) at 1.53x the
 // minimum tensor work.
 //
-//   warps 0..2 : gather -- the rows idx[t][...] of the split, 32 per tile, copied with 16-byte
-//                cp.async into a 2-stage ring in the 128-byte-swizzled K-major layout (FP8
-//                rows are widened to BF16 on the way, exactly); per-row scale and validity.
-//   warp 3     : MMA issuer -- S_j = Q K_j^T into TMEM (36 MMAs, N = 32), then after the
+//   warps 0..3 : gather -- two groups of two warps, group g fills stage g with the tiles
+//                j = g, g+2, ...: the tile's 32 row indices (prefetched one tile ahead) are
+//                staged in shared memory, then the rows are copied with 16-byte cp.async into
+//                the 128-byte-swizzled K-major layout (FP8 rows are widened to BF16 on the way,
+//                exactly); per-row scale and validity.  The two groups overlap their copies.
+//   warp 8     : MMA issuer -- S_j = Q K_j^T into TMEM (36 MMAs, N = 32), then after the
 //                softmax O += P_j V_j (2 MMAs, N = 256) with P read from TMEM and the same
 //                shared-memory tile read as an MN-major B operand.
 //   warps 4..7 : softmax -- thread = head (TMEM lane): online max / sum with lazy rescaling
@@ -27,19 +29,20 @@ namespace lsa {
 
 namespace {
 
-constexpr int kAThreads = 256;
+constexpr int kAThreads = 288;
 constexpr int kRows = 32;                    // KV rows per tile
 constexpr int kD = 576, kDv = 512, kHalf = 256;
 constexpr int kAtoms = kD / 64;              // 64-element (128-byte) K atoms
 constexpr int kTileBytes = kAtoms * kRows * 128;     // 36 KB
 constexpr int kQBytes = kAtoms * 128 * 128;          // 144 KB
-constexpr int kProdThreads = 96;
+constexpr int kGroupThreads = 64;            // threads of one gather group
 
 struct AttnSmem {
     alignas(1024) uint8_t q[kQBytes];
     alignas(1024) uint8_t kv[2][kTileBytes];
     float kscale[2][kRows];
     int valid[2][kRows];
+    int rows[2][kRows];
     uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done;
     uint32_t tmem_base;
     int abort;
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&sm.kv_full[i], kProdThreads);
+            tc::mbar_init(&sm.kv_full[i], kGroupThreads);
             tc::mbar_init(&sm.kv_empty[i], 1);
             tc::mbar_init(&sm.s_full[i], 1);
             tc::mbar_init(&sm.p_full[i], 128);
@@ -98,57 +101,80 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
     const uint32_t tmem = sm.tmem_base;
     const uint32_t o_col = tmem, s_col = tmem + 256, p_col = tmem + 320;
 
-    if (warp < 3) {
-        // ---------------- gather producer
-        const int pt = threadIdx.x;                       // 0..95
-        for (int j = 0; j < n_tiles; ++j) {
-            const int s = j & 1;
-            if (!tc::mbar_wait(&sm.kv_empty[s], ((j >> 1) + 1) & 1, abort_flag)) break;
+    if (warp < 4) {
+        // ---------------- gather producers: group g owns stage g and the tiles j = g, g + 2, ...
+        const int g = warp >> 1;
+        const int gt = threadIdx.x - g * kGroupThreads;          // 0..63
+        auto fetch_row = [&](int j) -> int {
+            if (j >= n_tiles || gt >= kRows) return -1;
+            const int r0 = r_beg + j * kRows;
+            return gt < min(kRows, r_end - r0) ? irow[r0 + gt] : -1;
+        };
+        int nxt = fetch_row(g);
+        for (int j = g; j < n_tiles; j += 2) {
+            const int cur = nxt;
+            nxt = fetch_row(j + 2);                                // prefetch the group's next tile
+            if (!tc::mbar_wait(&sm.kv_empty[g], ((j >> 1) + 1) & 1, abort_flag)) break;
             const int r0 = r_beg + j * kRows;
             const int nr = min(kRows, r_end - r0);
-            if (pt < kRows) {
-                const int row = pt < nr ? irow[r0 + pt] : -1;
-                const bool v = row >= 0 && row < len;
-                if (pt < nr && !v) report(a.status, LSA_ERR_DEVICE_DATA);
-                sm.valid[s][pt] = v;
-                sm.kscale[s][pt] = KV_FP8 ? (v ? kvs[row] : 0.f) : 1.f;
+            if (gt < kRows) {
+                const bool v = cur >= 0 && cur < len;
+                if (gt < nr && !v) report(a.status, LSA_ERR_DEVICE_DATA);
+                sm.rows[g][gt] = v ? cur : -1;
+                sm.valid[g][gt] = v;
+                sm.kscale[g][gt] = KV_FP8 ? (v ? kvs[cur] : 0.f) : 1.f;
             }
-            uint8_t* tile = sm.kv[s];
+            asm volatile("bar.sync %0, %1;" :: "r"(1 + g), "r"(kGroupThreads) : "memory");
+            uint8_t* tile = sm.kv[g];
             if (!KV_FP8) {
-                for (int i = pt; i < kRows * (kD / 8); i += kProdThreads) {
+                for (int i = gt; i < kRows * (kD / 8); i += kGroupThreads) {
                     const int r = i / (kD / 8), c = i % (kD / 8);
-                    const int row = r < nr ? irow[r0 + r] : -1;
-                    const bool v = row >= 0 && row < len;
+                    const int row = sm.rows[g][r];
                     uint8_t* dst = tile + (c >> 3) * (kRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-                    cp_async16(dst, kvb + (size_t)(v ? row : 0) * a.kv_tok_b + c * 16, v);
+                    cp_async16(dst, kvb + (size_t)(row >= 0 ? row : 0) * a.kv_tok_b + c * 16, row >= 0);
                 }
                 cp_async_commit();
                 cp_async_wait<0>();
             } else {
-                for (int i = pt; i < kRows * (kD / 16); i += kProdThreads) {
-                    const int r = i / (kD / 16), c = i % (kD / 16);      // 16 codes -> two 16-byte bf16 chunks
-                    const int row = r < nr ? irow[r0 + r] : -1;
-                    const bool v = row >= 0 && row < len;
-                    const uint4 raw = v ? ldg_nc16(kvb + (size_t)row * a.kv_tok_b + c * 16) : make_uint4(0, 0, 0, 0);
-                    const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw);
-                    uint32_t ow[8];
+                constexpr int kChunks = kRows * (kD / 16);             // 16 codes per chunk
+                constexpr int kBatch = 6;
+                for (int i0 = gt; i0 < kChunks; i0 += kGroupThreads * kBatch) {
+                    uint4 raw[kBatch];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        ow[2 * u] = e4m3x2_to_bf16x2((uint16_t)(wd[u] & 0xffff));
-                        ow[2 * u + 1] = e4m3x2_to_bf16x2((uint16_t)(wd[u] >> 16));
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int i = i0 + u * kGroupThreads;
+                        raw[u] = make_uint4(0, 0, 0, 0);
+                        if (i < kChunks) {
+                            const int row = sm.rows[g][i / (kD / 16)];
+                            if (row >= 0) raw[u] = ldg_nc16(kvb + (size_t)row * a.kv_tok_b + (i % (kD / 16)) * 16);
+                        }
                     }
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int cb = 2 * c + hh;                          // bf16 chunk index (8 dims)
-                        uint8_t* dst = tile + (cb >> 3) * (kRows * 128) + r * 128 + (((cb & 7) ^ (r & 7)) << 4);
-                        *reinterpret_cast<uint4*>(dst) = make_uint4(ow[4 * hh], ow[4 * hh + 1], ow[4 * hh + 2], ow[4 * hh + 3]);
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int i = i0 + u * kGroupThreads;
+                        if (i >= kChunks) break;
+                        const int r = i / (kD / 16), c = i % (kD / 16);
+                        const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw[u]);
+                        uint32_t ow[8];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            ow[2 * q] = e4m3x2_to_bf16x2((uint16_t)(wd[q] & 0xffff));
+                            ow[2 * q + 1] = e4m3x2_to_bf16x2((uint16_t)(wd[q] >> 16));
+                        }
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int cb = 2 * c + hh;                  // bf16 chunk index (8 dims)
+                            uint8_t* dst = tile + (cb >> 3) * (kRows * 128) + r * 128 + (((cb & 7) ^ (r & 7)) << 4);
+                            *reinterpret_cast<uint4*>(dst) =
+                                make_uint4(ow[4 * hh], ow[4 * hh + 1], ow[4 * hh + 2], ow[4 * hh + 3]);
+                        }
                     }
                 }
             }
             tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&sm.kv_full[s]);
+            tc::mbar_arrive(&sm.kv_full[g]);
         }
-    } else if (warp == 3) {
+    } else if (warp == 8) {
         // ---------------- MMA issuer
         const uint32_t idesc_s = tc::idesc_f16(128, kRows, 1);
         const uint32_t idesc_o = tc::idesc_f16_bmn(128, kHalf, 1);

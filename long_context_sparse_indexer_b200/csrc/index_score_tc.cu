@@ -5,14 +5,15 @@
 // restated for sm_100a.  One CTA owns 2048 score columns of a group of G <= 4 query tokens
 // of one sequence, so every key row is read from HBM once per group.
 //
-//   warp 0      : TMA producer -- 128-key tiles (two 64-row boxes, 128-byte swizzle) into a
-//                 4-stage shared-memory ring; allocates / frees TMEM.
+//   warp 0      : TMA producer -- 128-key tiles (two 64-row boxes, 128-byte swizzle) and their
+//                 per-token scales into a 4-stage shared-memory ring; allocates / frees TMEM.
 //   warp 1      : MMA issuer -- per tile, 8 x tcgen05.mma kind::f16 (M = 128 keys, N = G*H_I,
 //                 K = 16) with A read from TMEM and B (the queries) from shared memory.
-//   warps 2..5  : converters / epilogue -- thread = key row (= TMEM lane): widen the row's 128
-//                 FP8 codes to f16 (exact) and store them as the A operand in TMEM; for the
-//                 previous tile, load the accumulator row (G*H_I scores), apply ReLU, the
-//                 weighted head sum (fixed order) and the token's FP8 scale, store.
+//   warps 2..5  : converters -- thread = key row (= TMEM lane): widen the row's 128 FP8 codes
+//                 to f16 (exact) and store them as the A operand in TMEM.
+//   warps 6..9  : epilogue -- thread = key row: load the accumulator row (G*H_I scores), apply
+//                 ReLU, the weighted head sum (four partial sums combined in a fixed order)
+//                 and the token's FP8 scale, store.
 //
 // Queries are scaled per head by a power of two into f16 range (exact for all values within
 // 2^28 of the head's maximum); the inverse power is folded into the head weight.  Products
@@ -28,7 +29,7 @@ namespace lsa {
 
 namespace {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;
 constexpr int kTcCols = 2048;          // score columns per CTA
 constexpr int kTile = 128;             // keys per MMA tile
 constexpr int kStages = 4;             // key-tile ring
@@ -44,7 +45,8 @@ template <int N>
 struct TcSmem {
     alignas(1024) uint8_t keys[kStages][kKeyTileBytes];
     alignas(1024) uint8_t q[2][N * 128];          // B operand: two 64-element K atoms, SW128
-    float w[N];                                   // head weights (inverse query scale folded in)
+    alignas(16) float scl[kStages][kTile];        // per-token FP8 scales of each key tile
+    alignas(16) float w[N];                       // head weights (inverse query scale folded in)
     uint64_t full_k[kStages], empty_k[kStages];
     uint64_t a_full[2], a_empty[2];
     uint64_t d_full[2], d_empty[2];
@@ -55,8 +57,9 @@ struct TcSmem {
 };
 
 template <int N>
-__global__ void __launch_bounds__(kTcThreads, 1)
-index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs ta) {
+__global__ void __launch_bounds__(kTcThreads, (N <= 128 ? 2 : 1))
+index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap smap,
+                      TcArgs ta) {
     extern __shared__ uint8_t smem_raw[];
     TcSmem<N>& sm = *reinterpret_cast<TcSmem<N>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const IndexArgs& a = ta.a;
@@ -70,7 +73,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs ta) {
 
     // ---- set-up: barriers, TMEM, query group validity
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full_k[s], 1); tc::mbar_init(&sm.empty_k[s], 128); }
+        // A stage is free once the converters have read its keys and the epilogue its scales.
+        for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full_k[s], 1); tc::mbar_init(&sm.empty_k[s], 256); }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.a_full[i], 128); tc::mbar_init(&sm.a_empty[i], 1);
             tc::mbar_init(&sm.d_full[i], 1); tc::mbar_init(&sm.d_empty[i], 128);
@@ -78,6 +82,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs ta) {
         sm.abort = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&tmap);
+        tc::prefetch_tmap(&smap);
     }
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, ta.tmem_cols);
     const int bseq = a.q_seq[t0];
@@ -144,7 +149,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs ta) {
                 const int s = j % kStages;
                 if (!tc::mbar_wait(&sm.empty_k[s], ((j / kStages) + 1) & 1, abort_flag)) break;
                 ++issued;
-                tc::mbar_expect_tx(&sm.full_k[s], kKeyTileBytes);
+                tc::mbar_expect_tx(&sm.full_k[s], kKeyTileBytes + kTile * 4);
                 const int c = col_beg + j * kTile;
                 int r0 = c, r1 = c + 64;
                 if (hi) {
@@ -156,6 +161,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs ta) {
                 }
                 tc::tma_load_3d(sm.keys[s], &tmap, &sm.full_k[s], 0, r0, max(bseq, 0));
                 tc::tma_load_3d(sm.keys[s] + kKeyTileBytes / 2, &tmap, &sm.full_k[s], 0, r1, max(bseq, 0));
+                tc::tma_load_2d(sm.scl[s], &smap, &sm.full_k[s], r0, max(bseq, 0));
+                tc::tma_load_2d(sm.scl[s] + 64, &smap, &sm.full_k[s], r1, max(bseq, 0));
             }
             // Drain: every issued tile has landed before the CTA can exit (bounded; already true
             // unless the consumers gave up early).
@@ -189,54 +196,20 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs ta) {
                 tc::mbar_wait(&sm.d_full[last % DS], (last / DS) & 1, &drain_abort);
             }
         }
-    } else {
-        // ---------------- converters / epilogue: thread = TMEM lane = key row of the tile
+    } else if (warp < 6) {
+        // ---------------- converters: thread = TMEM lane = key row of the tile
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const float* sseq = a.kscale ? a.kscale + (size_t)max(bseq, 0) * a.scale_seq_stride : nullptr;
-
-        auto epilogue = [&](int j) -> bool {
-            const int db = j % DS;
-            if (!tc::mbar_wait(&sm.d_full[db], (j / DS) & 1, abort_flag)) return false;
-            tc::tc_fence_after();
-            const int col = col_beg + j * kTile + r;
-            int row = col;
-            if (hi) {
-                const int bi = col / 64;
-                const int blk = (col < a.n_cols && bi < a.n_cand) ? a.cand[(size_t)t0 * a.n_cand + bi] : -1;
-                row = blk >= 0 ? blk * 64 + (col & 63) : -1;
-            }
-            const float ks = (sseq && row >= 0 && row <= max_pos) ? sseq[row] : 1.f;
-            for (int gi = 0; gi < G; ++gi) {
-                float acc = 0.f;
-                for (int h0 = 0; h0 < H_I; h0 += 32) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(d_col + db * N + gi * H_I + h0 + lane_off, v);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc = fmaf(sm.w[gi * H_I + h0 + i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
-                }
-                if (col < col_end) {
-                    const bool vis = sm.ok[gi] && row >= 0 && row <= sm.pos[gi];
-                    a.scores[(size_t)(t0 + gi) * a.ld + col] = vis ? acc * ks : kNegInf;
-                }
-            }
-            tc::tc_fence_before();
-            tc::mbar_arrive(&sm.d_empty[db]);
-            return true;
-        };
-
-        bool alive = true;
-        for (int j = 0; j < n_active && alive; ++j) {
+        for (int j = 0; j < n_active; ++j) {
             const int s = j % kStages, ab = j & 1;
-            if (!tc::mbar_wait(&sm.full_k[s], (j / kStages) & 1, abort_flag)) { alive = false; break; }
+            if (!tc::mbar_wait(&sm.full_k[s], (j / kStages) & 1, abort_flag)) break;
             const uint8_t* rowp = sm.keys[s] + r * 128;          // 128-byte rows, 16-byte chunks XOR-swizzled
             uint4 ch[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) ch[c] = *reinterpret_cast<const uint4*>(rowp + ((c ^ (r & 7)) << 4));
             tc::mbar_arrive(&sm.empty_k[s]);
-            if (!tc::mbar_wait(&sm.a_empty[ab], ((j >> 1) + 1) & 1, abort_flag)) { alive = false; break; }
+            if (!tc::mbar_wait(&sm.a_empty[ab], ((j >> 1) + 1) & 1, abort_flag)) break;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t wv[32];
@@ -254,9 +227,52 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs ta) {
             tc::tmem_wait_st();
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.a_full[ab]);
-            if (j > 0 && !epilogue(j - 1)) { alive = false; break; }
         }
-        if (alive && n_active > 0) epilogue(n_active - 1);
+    } else {
+        // ---------------- epilogue: thread = TMEM lane = key row of the tile
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const bool fp8 = a.kscale != nullptr;
+        for (int j = 0; j < n_active; ++j) {
+            const int s = j % kStages, db = j % DS;
+            if (!tc::mbar_wait(&sm.full_k[s], (j / kStages) & 1, abort_flag)) break;
+            const float ks = fp8 ? sm.scl[s][r] : 1.f;
+            tc::mbar_arrive(&sm.empty_k[s]);
+            if (!tc::mbar_wait(&sm.d_full[db], (j / DS) & 1, abort_flag)) break;
+            tc::tc_fence_after();
+            const int col = col_beg + j * kTile + r;
+            int row = col;
+            if (hi) {
+                const int bi = col / 64;
+                const int blk = (col < a.n_cols && bi < a.n_cand) ? a.cand[(size_t)t0 * a.n_cand + bi] : -1;
+                row = blk >= 0 ? blk * 64 + (col & 63) : -1;
+            }
+            for (int gi = 0; gi < G; ++gi) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int h0 = 0; h0 < H_I; h0 += 32) {
+                    uint32_t v[32];
+                    tc::tmem_ld32(d_col + db * N + gi * H_I + h0 + lane_off, v);
+                    tc::tmem_wait_ld();
+                    const float4* wp = reinterpret_cast<const float4*>(sm.w + gi * H_I + h0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 ww = wp[i];
+                        acc[0] = fmaf(ww.x, fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), acc[0]);
+                        acc[1] = fmaf(ww.y, fmaxf(__uint_as_float(v[4 * i + 1]), 0.f), acc[1]);
+                        acc[2] = fmaf(ww.z, fmaxf(__uint_as_float(v[4 * i + 2]), 0.f), acc[2]);
+                        acc[3] = fmaf(ww.w, fmaxf(__uint_as_float(v[4 * i + 3]), 0.f), acc[3]);
+                    }
+                }
+                const float total = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                if (col < col_end) {
+                    const bool vis = sm.ok[gi] && row >= 0 && row <= sm.pos[gi];
+                    a.scores[(size_t)(t0 + gi) * a.ld + col] = vis ? total * ks : kNegInf;
+                }
+            }
+            tc::tc_fence_before();
+            tc::mbar_arrive(&sm.d_empty[db]);
+        }
         // Columns of the chunk past the active tiles see no visible key.
         for (int col = col_beg + n_active * kTile + r; col < col_end; col += 128)
             for (int gi = 0; gi < G; ++gi) a.scores[(size_t)(t0 + gi) * a.ld + col] = kNegInf;
@@ -289,7 +305,7 @@ EncodeTiled encode_fn() {
 }
 
 template <int N>
-cudaError_t launch_n(const CUtensorMap& m, const TcArgs& ta, cudaStream_t st) {
+cudaError_t launch_n(const CUtensorMap& m, const CUtensorMap& sm, const TcArgs& ta, cudaStream_t st) {
     // At least 80 KB so that no more than two CTAs share an SM: two 256-column TMEM
     // allocations fill the SM's 512 columns (a third CTA would wait for one to finish).
     const size_t smem = std::max(sizeof(TcSmem<N>) + 1024, (size_t)80 * 1024);
@@ -297,7 +313,7 @@ cudaError_t launch_n(const CUtensorMap& m, const TcArgs& ta, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((ta.a.n_cols + kTcCols - 1) / kTcCols, ta.a.T / ta.G);
-    kern<<<grid, kTcThreads, smem, st>>>(m, ta);
+    kern<<<grid, kTcThreads, smem, st>>>(m, sm, ta);
     return cudaGetLastError();
 }
 
@@ -310,6 +326,7 @@ bool index_score_tc_supported(const IndexArgs& a, int H_I, int D_I, bool fp8) {
     const int N = G * H_I;
     if (N > 256) return false;
     return ((uintptr_t)a.kdata % 16 == 0) && (a.tok_stride_b % 16 == 0) && (a.seq_stride_b % 16 == 0) &&
+           a.kscale != nullptr && ((uintptr_t)a.kscale % 16 == 0) && (a.scale_seq_stride % 4 == 0) &&
            encode_fn() != nullptr;
 }
 
@@ -334,12 +351,22 @@ cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st) {
                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // Per-token scales: [B][L_alloc] floats, boxes of 64 rows (zero fill past the end).
+    CUtensorMap sc;
+    const cuuint64_t sdims[2] = {(cuuint64_t)a.L_alloc, (cuuint64_t)a.B};
+    const cuuint64_t sstr[1] = {(cuuint64_t)a.scale_seq_stride * 4};
+    const cuuint32_t sbox[2] = {64, 1};
+    const cuuint32_t sestr[2] = {1, 1};
+    r = encode_fn()(&sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(a.kscale), sdims, sstr, sbox, sestr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     switch (ta.N) {
-        case 32: return launch_n<32>(m, ta, st);
-        case 64: return launch_n<64>(m, ta, st);
-        case 128: return launch_n<128>(m, ta, st);
-        case 192: return launch_n<192>(m, ta, st);
-        case 256: return launch_n<256>(m, ta, st);
+        case 32: return launch_n<32>(m, sc, ta, st);
+        case 64: return launch_n<64>(m, sc, ta, st);
+        case 128: return launch_n<128>(m, sc, ta, st);
+        case 192: return launch_n<192>(m, sc, ta, st);
+        case 256: return launch_n<256>(m, sc, ta, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -16,7 +16,8 @@
 // columns first); ranks across CTAs, warps and lanes come from cluster-wide prefix
 // counts, ballots and popcounts.  Positions are written in ascending order and merged
 // with the sinks [0, a) and the window [b, pos], so the list comes out sorted and
-// de-duplicated.
+// de-duplicated.  Segments of up to 40960 columns are first cached in shared memory as
+// order keys (one coalesced read of the row); longer ones are re-read from global memory.
 #include <cooperative_groups.h>
 
 #include "kernels.cuh"
@@ -109,12 +110,17 @@ __device__ int cluster_exclusive(cg::cluster_group& cl, int* slot, int rank, int
     return before;
 }
 
+// Segment length (columns) a CTA caches in shared memory as order keys.
+constexpr int kTopkCacheCols = 40960;
+
+template <bool CACHED>
 __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
 topk_kernel(TopkArgs a) {
     __shared__ int hist[4096];
     __shared__ int hsum[4096];
     __shared__ int s_warp[kTopkWarps];
     __shared__ int s_bin, s_above, s_slot, s_nvalid;
+    extern __shared__ uint32_t s_keys[];          // CACHED: order key of each column of the segment, 0 = invalid
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
     const int t = blockIdx.x / kTopkCluster;
@@ -144,18 +150,47 @@ topk_kernel(TopkArgs a) {
     const int per_warp = ((c1 - c0 + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
     const int w0 = min(c1, c0 + warp * per_warp), w1 = min(c1, w0 + per_warp);
 
-    // ---- pass 1: top 12 bits
+    // Order key of column cc of this warp's segment (0 = not a candidate; valid keys are > 0).
+    auto key_at = [&](int cc) -> uint32_t {
+        if (cc >= w1) return 0u;
+        if (CACHED) return s_keys[cc - c0];
+        const float f = row[cc];
+        return (f != f || f == kNegInf) ? 0u : order_key(f);
+    };
+
+    // ---- pass 1: top 12 bits (and, when cached, the segment's keys into shared memory)
     for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
     if (threadIdx.x == 0) s_nvalid = 0;
+    if (CACHED) {
+        for (int cc = c0 + threadIdx.x * 4; cc < c1; cc += kTopkThreads * 4) {
+            float f[4];
+            if (cc + 3 < c1 && (((uintptr_t)(row + cc)) & 15) == 0) {
+                const float4 v4 = *reinterpret_cast<const float4*>(row + cc);
+                f[0] = v4.x; f[1] = v4.y; f[2] = v4.z; f[3] = v4.w;
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) f[u] = cc + u < c1 ? row[cc + u] : kNegInf;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (cc + u >= c1) break;
+                if (f[u] != f[u]) report(a.status, LSA_ERR_DEVICE_DATA);
+                s_keys[cc + u - c0] = (f[u] != f[u] || f[u] == kNegInf) ? 0u : order_key(f[u]);
+            }
+        }
+    }
     __syncthreads();
     int nvalid = 0;
     for (int c = w0; c < w1; c += 32) {
         const int cc = c + lane;
-        const float f = cc < w1 ? row[cc] : kNegInf;
-        if (f != f) report(a.status, LSA_ERR_DEVICE_DATA);
-        const bool v = !(f != f) && f != kNegInf;
+        if (!CACHED && cc < w1) {
+            const float f = row[cc];
+            if (f != f) report(a.status, LSA_ERR_DEVICE_DATA);
+        }
+        const uint32_t key = key_at(cc);
+        const bool v = key != 0u;
         nvalid += v;
-        hist_add(hist, v ? (int)(order_key(f) >> 20) : 0, v);
+        hist_add(hist, v ? (int)(key >> 20) : 0, v);
     }
     atomicAdd(&s_nvalid, nvalid);
     __syncthreads();
@@ -173,11 +208,8 @@ topk_kernel(TopkArgs a) {
         for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
         __syncthreads();
         for (int c = w0; c < w1; c += 32) {
-            const int cc = c + lane;
-            const float f = cc < w1 ? row[cc] : kNegInf;
-            const bool v = !(f != f) && f != kNegInf;
-            const uint32_t key = v ? order_key(f) : 0u;
-            hist_add(hist, (int)((key >> 8) & 0xfff), v && (key >> 20) == b1);
+            const uint32_t key = key_at(c + lane);
+            hist_add(hist, (int)((key >> 8) & 0xfff), key != 0u && (key >> 20) == b1);
         }
         cluster_threshold(cl, hist, hsum, 4096, a.k - above, s_warp, &s_bin, &s_above);
         const uint32_t b2 = (uint32_t)s_bin;
@@ -187,11 +219,8 @@ topk_kernel(TopkArgs a) {
         for (int i = threadIdx.x; i < 256; i += kTopkThreads) hist[i] = 0;
         __syncthreads();
         for (int c = w0; c < w1; c += 32) {
-            const int cc = c + lane;
-            const float f = cc < w1 ? row[cc] : kNegInf;
-            const bool v = !(f != f) && f != kNegInf;
-            const uint32_t key = v ? order_key(f) : 0u;
-            hist_add(hist, (int)(key & 0xff), v && (key >> 8) == pre);
+            const uint32_t key = key_at(c + lane);
+            hist_add(hist, (int)(key & 0xff), key != 0u && (key >> 8) == pre);
         }
         cluster_threshold(cl, hist, hsum, 256, a.k - above, s_warp, &s_bin, &s_above);
         above += s_above;
@@ -205,11 +234,9 @@ topk_kernel(TopkArgs a) {
     auto classify = [&](int cc, bool& eq, bool& gt, int& p) {
         eq = gt = false;
         p = -1;
-        if (cc >= w1) return;
-        const float f = row[cc];
-        if (f != f || f == kNegInf) return;
+        const uint32_t key = key_at(cc);
+        if (key == 0u) return;
         if (a.k > 0) {
-            const uint32_t key = order_key(f);
             gt = take_all || key > vstar;
             eq = !take_all && key == vstar;
         }
@@ -283,7 +310,16 @@ topk_kernel(TopkArgs a) {
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
-    topk_kernel<<<a.T * kTopkCluster, kTopkThreads, 0, st>>>(a);
+    const int per_cta = ((a.n_cols + kTopkCluster - 1) / kTopkCluster + 31) / 32 * 32;
+    if (per_cta <= kTopkCacheCols) {
+        const size_t smem = (size_t)per_cta * 4;
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kTopkCacheCols * 4);
+        if (e != cudaSuccess) return e;
+        topk_kernel<true><<<a.T * kTopkCluster, kTopkThreads, smem, st>>>(a);
+    } else {
+        topk_kernel<false><<<a.T * kTopkCluster, kTopkThreads, 0, st>>>(a);
+    }
     return cudaGetLastError();
 }
 
