@@ -20,6 +20,7 @@
 // of f16 values are exact in the FP32 accumulator.  All waits are bounded (2 s of wall time);
 // a CTA that gives up reports LSA_ERR_TIMEOUT and returns after freeing its TMEM.
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "kernels.cuh"
@@ -39,6 +40,7 @@ constexpr int kMaxG = 4;
 struct TcArgs {
     IndexArgs a;
     int G, H_I, N, d_stages, tmem_cols;
+    int scale_tma;          // per-token scales arrive by TMA with the keys (else: epilogue reads global)
 };
 
 template <int N>
@@ -82,7 +84,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         sm.abort = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&tmap);
-        tc::prefetch_tmap(&smap);
+        if (ta.scale_tma) tc::prefetch_tmap(&smap);
     }
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, ta.tmem_cols);
     const int bseq = a.q_seq[t0];
@@ -149,7 +151,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                 const int s = j % kStages;
                 if (!tc::mbar_wait(&sm.empty_k[s], ((j / kStages) + 1) & 1, abort_flag)) break;
                 ++issued;
-                tc::mbar_expect_tx(&sm.full_k[s], kKeyTileBytes + kTile * 4);
+                tc::mbar_expect_tx(&sm.full_k[s], kKeyTileBytes + (ta.scale_tma ? kTile * 4 : 0));
                 const int c = col_beg + j * kTile;
                 int r0 = c, r1 = c + 64;
                 if (hi) {
@@ -161,8 +163,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                 }
                 tc::tma_load_3d(sm.keys[s], &tmap, &sm.full_k[s], 0, r0, max(bseq, 0));
                 tc::tma_load_3d(sm.keys[s] + kKeyTileBytes / 2, &tmap, &sm.full_k[s], 0, r1, max(bseq, 0));
-                tc::tma_load_2d(sm.scl[s], &smap, &sm.full_k[s], r0, max(bseq, 0));
-                tc::tma_load_2d(sm.scl[s] + 64, &smap, &sm.full_k[s], r1, max(bseq, 0));
+                if (ta.scale_tma) {
+                    tc::tma_load_2d(sm.scl[s], &smap, &sm.full_k[s], r0, max(bseq, 0));
+                    tc::tma_load_2d(sm.scl[s] + 64, &smap, &sm.full_k[s], r1, max(bseq, 0));
+                }
             }
             // Drain: every issued tile has landed before the CTA can exit (bounded; already true
             // unless the consumers gave up early).
@@ -237,10 +241,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         for (int j = 0; j < n_active; ++j) {
             const int s = j % kStages, db = j % DS;
             if (!tc::mbar_wait(&sm.full_k[s], (j / kStages) & 1, abort_flag)) break;
-            const float ks = fp8 ? sm.scl[s][r] : 1.f;
-            tc::mbar_arrive(&sm.empty_k[s]);
-            if (!tc::mbar_wait(&sm.d_full[db], (j / DS) & 1, abort_flag)) break;
-            tc::tc_fence_after();
             const int col = col_beg + j * kTile + r;
             int row = col;
             if (hi) {
@@ -248,6 +248,14 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                 const int blk = (col < a.n_cols && bi < a.n_cand) ? a.cand[(size_t)t0 * a.n_cand + bi] : -1;
                 row = blk >= 0 ? blk * 64 + (col & 63) : -1;
             }
+            float ks = 1.f;
+            if (fp8) {
+                if (ta.scale_tma) ks = sm.scl[s][r];
+                else if (row >= 0 && row <= max_pos) ks = a.kscale[(size_t)max(bseq, 0) * a.scale_seq_stride + row];
+            }
+            tc::mbar_arrive(&sm.empty_k[s]);
+            if (!tc::mbar_wait(&sm.d_full[db], (j / DS) & 1, abort_flag)) break;
+            tc::tc_fence_after();
             for (int gi = 0; gi < G; ++gi) {
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int h0 = 0; h0 < H_I; h0 += 32) {
@@ -326,8 +334,7 @@ bool index_score_tc_supported(const IndexArgs& a, int H_I, int D_I, bool fp8) {
     const int N = G * H_I;
     if (N > 256) return false;
     return ((uintptr_t)a.kdata % 16 == 0) && (a.tok_stride_b % 16 == 0) && (a.seq_stride_b % 16 == 0) &&
-           a.kscale != nullptr && ((uintptr_t)a.kscale % 16 == 0) && (a.scale_seq_stride % 4 == 0) &&
-           encode_fn() != nullptr;
+           a.kscale != nullptr && encode_fn() != nullptr;
 }
 
 cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st) {
@@ -351,16 +358,21 @@ cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st) {
                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    // Per-token scales: [B][L_alloc] floats, boxes of 64 rows (zero fill past the end).
+    // Per-token scales: [B][L_alloc] floats, boxes of 64 rows (zero fill past the end); TMA needs
+    // a 16-byte aligned base and sequence stride, otherwise the epilogue reads them directly.
+    ta.scale_tma = ((uintptr_t)a.kscale % 16 == 0) && (a.scale_seq_stride % 4 == 0) && a.B * (int64_t)a.scale_seq_stride > 0;
     CUtensorMap sc;
+    memset(&sc, 0, sizeof(sc));
     const cuuint64_t sdims[2] = {(cuuint64_t)a.L_alloc, (cuuint64_t)a.B};
     const cuuint64_t sstr[1] = {(cuuint64_t)a.scale_seq_stride * 4};
     const cuuint32_t sbox[2] = {64, 1};
     const cuuint32_t sestr[2] = {1, 1};
-    r = encode_fn()(&sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(a.kscale), sdims, sstr, sbox, sestr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    if (ta.scale_tma) {
+        r = encode_fn()(&sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(a.kscale), sdims, sstr, sbox,
+                        sestr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) ta.scale_tma = 0;
+    }
     switch (ta.N) {
         case 32: return launch_n<32>(m, sc, ta, st);
         case 64: return launch_n<64>(m, sc, ta, st);

@@ -105,7 +105,7 @@ def build_workload(w: W.Workload, device="cuda", L_alloc: int | None = None) -> 
     build()
     dev = torch.device(device)
     lens = W.lengths(w)
-    L_alloc = int(L_alloc or lens.max())
+    L_alloc = int(L_alloc or -(-int(lens.max()) // 64) * 64)     # rows per sequence, a multiple of 64
     seq_len = torch.from_numpy(lens.astype(np.int32)).to(dev)
     passes = []
     kv_done = {}

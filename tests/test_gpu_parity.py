@@ -31,15 +31,20 @@ SMALL = {
     "mtp_small": W.scaled("mtp_256k", B=2, len_lo=3001, len_hi=3001),
     "prefill_small": W.scaled("prefill_32k", len_lo=3000, len_hi=3000, passes=(W._target_pass(64, 1),)),
     "hi_small": W.scaled("decode_hi_1m", B=2, len_lo=20000, len_hi=20000),
+    # FP8 scales whose per-sequence stride is not 16-byte aligned (the tensor-core indexer
+    # reads them directly instead of by TMA), and a 64-dim FP8 indexer (warp-MMA kernel).
+    "cli_unaligned": W.scaled("decode_cli_128k", B=3, len_lo=2500, len_hi=5200, seed=12),
+    "cli_d64": W.scaled("decode_cli_128k", B=2, len_lo=3000, len_hi=4100, d_I=64, seed=13),
 }
-FLAT = ["tiny_decode", "cli_small", "mtp_small", "prefill_small"]
+FLAT = ["tiny_decode", "cli_small", "mtp_small", "prefill_small", "cli_unaligned", "cli_d64"]
+L_ALLOC = {"cli_unaligned": 5203}
 
 _cache = {}
 
 
 def wt_of(name):
     if name not in _cache:
-        _cache[name] = D.build_workload(SMALL[name], "cuda")
+        _cache[name] = D.build_workload(SMALL[name], "cuda", L_alloc=L_ALLOC.get(name))
     return _cache[name]
 
 
