@@ -9,14 +9,19 @@
 // the duplicated QK^T keeps every CTA independent (no cross-CTA exchange) at 1.53x the
 // minimum tensor work.
 //
-//   warps 0..3 : gather -- two groups of two warps, group g fills stage g with the tiles
-//                j = g, g+2, ...: the tile's 32 row indices (prefetched one tile ahead) are
-//                staged in shared memory, then the rows are copied with 16-byte cp.async into
-//                the 128-byte-swizzled K-major layout (FP8 rows are widened to BF16 on the way,
-//                exactly); per-row scale and validity.  The two groups overlap their copies.
-//   warp 8     : MMA issuer -- S_j = Q K_j^T into TMEM (36 MMAs, N = 32), then after the
-//                softmax O += P_j V_j (2 MMAs, N = 256) with P read from TMEM and the same
-//                shared-memory tile read as an MN-major B operand.
+// Memory plan.  TMEM (512 columns): O half [0,256), S double buffer [256,320), P double
+// buffer [320,352), and Q dims 256..575 [352,512) as the A operand of the last 20 K-steps of
+// S.  Shared memory: Q dims 0..255 (4 swizzled K atoms, 64 KB) as the A operand of the first
+// 16 K-steps, and a 4-stage ring of 32-row KV tiles (36 KB each) in the 128-byte-swizzled
+// K-major layout, read as the B operand of S (K-major) and of P V (MN-major).
+//
+//   warps 0..3 : gather -- warp g fills stage g with the tiles j = g, g+4, ...: the tile's 32
+//                row indices (prefetched one tile ahead) go to shared memory, then the rows
+//                are copied with 16-byte cp.async (FP8 rows are widened to BF16 exactly on the
+//                way); per-row scale and validity.
+//   warp 8     : MMA issuer -- issues whatever is ready, in order per kind: S_j (16 SS + 20 TS
+//                MMAs, N = 32) once tile j has landed and P V_{j-2} has been issued, and
+//                O += P_j V_j (2 TS MMAs, N = 256) once the softmax of tile j is done.
 //   warps 4..7 : softmax -- thread = head (TMEM lane): online max / sum with lazy rescaling
 //                of O (only when the running max grows by more than 2^8; warp-uniform, so
 //                deterministic), P to TMEM as BF16; finally O / l and lse.
@@ -31,22 +36,30 @@ namespace {
 
 constexpr int kAThreads = 288;
 constexpr int kRows = 32;                    // KV rows per tile
+constexpr int kStagesA = 4;                  // KV tile ring
 constexpr int kD = 576, kDv = 512, kHalf = 256;
-constexpr int kAtoms = kD / 64;              // 64-element (128-byte) K atoms
-constexpr int kTileBytes = kAtoms * kRows * 128;     // 36 KB
-constexpr int kQBytes = kAtoms * 128 * 128;          // 144 KB
-constexpr int kGroupThreads = 64;            // threads of one gather group
+constexpr int kAtoms = kD / 64;              // 64-element (128-byte) K atoms of a KV row
+constexpr int kQSmemAtoms = 4;               // Q dims 0..255 in shared memory
+constexpr int kQTmemCols = (kD - kQSmemAtoms * 64) / 2;   // Q dims 256..575 in TMEM: 160 columns
+constexpr int kTileBytes = kAtoms * kRows * 128;          // 36 KB
+constexpr int kQBytes = kQSmemAtoms * 128 * 128;          // 64 KB
 
 struct AttnSmem {
     alignas(1024) uint8_t q[kQBytes];
-    alignas(1024) uint8_t kv[2][kTileBytes];
-    float kscale[2][kRows];
-    int valid[2][kRows];
-    int rows[2][kRows];
-    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done;
+    alignas(1024) uint8_t kv[kStagesA][kTileBytes];
+    alignas(16) float kscale[kStagesA][kRows];   // per-row FP8 scale x softmax scale (0 for masked rows)
+    alignas(16) float vscale[kStagesA][kRows];   // per-row FP8 scale (1 for BF16)
+    int rows[kStagesA][kRows];
+    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[2], p_full[2], o_done[2];
     uint32_t tmem_base;
     int abort;
 };
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 template <bool KV_FP8>
 __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a) {
@@ -69,65 +82,81 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
     const int32_t* irow = a.idx + (size_t)t * a.ld_idx;
     const uint8_t* kvb = a.kv + (size_t)max(b, 0) * a.kv_seq_b;
     const float* kvs = KV_FP8 ? a.kv_scale + (size_t)max(b, 0) * a.kv_scale_seq : nullptr;
+    const uint16_t* qt = a.q + (size_t)t * 128 * kD;
 
     if (threadIdx.x == 0) {
+        for (int i = 0; i < kStagesA; ++i) { tc::mbar_init(&sm.kv_full[i], 32); tc::mbar_init(&sm.kv_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&sm.kv_full[i], kGroupThreads);
-            tc::mbar_init(&sm.kv_empty[i], 1);
             tc::mbar_init(&sm.s_full[i], 1);
             tc::mbar_init(&sm.p_full[i], 128);
+            tc::mbar_init(&sm.o_done[i], 1);
         }
-        tc::mbar_init(&sm.o_done, 1);
         sm.abort = 0;
         tc::fence_barrier_init();
     }
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
-    // Q (all heads, all 576 dims) -> shared memory, K-major, 128-byte swizzle.
-    {
-        const uint16_t* qt = a.q + (size_t)t * 128 * kD;
-        for (int i = threadIdx.x; i < 128 * (kD / 8); i += kAThreads) {
-            const int h = i / (kD / 8), c = i % (kD / 8);
-            const int atom = c >> 3, cc = c & 7;
-            uint8_t* dst = sm.q + atom * (128 * 128) + h * 128 + ((cc ^ (h & 7)) << 4);
-            cp_async16(dst, qt + (size_t)h * kD + c * 8, true);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
+    // Q dims 0..255 -> shared memory (K-major, 128-byte swizzle).
+    for (int i = threadIdx.x; i < 128 * (kQSmemAtoms * 8); i += kAThreads) {
+        const int h = i / (kQSmemAtoms * 8), c = i % (kQSmemAtoms * 8);
+        uint8_t* dst = sm.q + (c >> 3) * (128 * 128) + h * 128 + (((c & 7) ^ (h & 7)) << 4);
+        cp_async16(dst, qt + (size_t)h * kD + c * 8, true);
     }
+    cp_async_commit();
+    cp_async_wait<0>();
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t o_col = tmem, s_col = tmem + 256, p_col = tmem + 320;
+    const uint32_t o_col = tmem, s_col = tmem + 256, p_col = tmem + 320, qt_col = tmem + 352;
+    // Q dims 256..575 -> TMEM (softmax warps: thread = head = lane).
+    if (warp >= 4 && warp < 8) {
+        const int h = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint4* src = reinterpret_cast<const uint4*>(qt + (size_t)h * kD + kQSmemAtoms * 64);
+#pragma unroll 1
+        for (int c = 0; c < kQTmemCols / 32; ++c) {
+            uint32_t v[32];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint4 x = src[c * 8 + u];
+                v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+            }
+            tc::tmem_st32(qt_col + c * 32 + lane_off, v);
+        }
+        tc::tmem_wait_st();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
 
     if (warp < 4) {
-        // ---------------- gather producers: group g owns stage g and the tiles j = g, g + 2, ...
-        const int g = warp >> 1;
-        const int gt = threadIdx.x - g * kGroupThreads;          // 0..63
+        // ---------------- gather producers: warp g owns stage g and the tiles j = g, g + 4, ...
+        const int g = warp;
         auto fetch_row = [&](int j) -> int {
-            if (j >= n_tiles || gt >= kRows) return -1;
+            if (j >= n_tiles) return -1;
             const int r0 = r_beg + j * kRows;
-            return gt < min(kRows, r_end - r0) ? irow[r0 + gt] : -1;
+            return lane < min(kRows, r_end - r0) ? irow[r0 + lane] : -1;
         };
         int nxt = fetch_row(g);
-        for (int j = g; j < n_tiles; j += 2) {
+        for (int j = g; j < n_tiles; j += kStagesA) {
             const int cur = nxt;
-            nxt = fetch_row(j + 2);                                // prefetch the group's next tile
-            if (!tc::mbar_wait(&sm.kv_empty[g], ((j >> 1) + 1) & 1, abort_flag)) break;
-            const int r0 = r_beg + j * kRows;
-            const int nr = min(kRows, r_end - r0);
-            if (gt < kRows) {
+            nxt = fetch_row(j + kStagesA);                         // prefetch this warp's next tile
+            if (!tc::mbar_wait(&sm.kv_empty[g], ((j / kStagesA) + 1) & 1, abort_flag)) break;
+            const int nr = min(kRows, r_end - (r_beg + j * kRows));
+            {
                 const bool v = cur >= 0 && cur < len;
-                if (gt < nr && !v) report(a.status, LSA_ERR_DEVICE_DATA);
-                sm.rows[g][gt] = v ? cur : -1;
-                sm.valid[g][gt] = v;
-                sm.kscale[g][gt] = KV_FP8 ? (v ? kvs[cur] : 0.f) : 1.f;
+                if (lane < nr && !v) report(a.status, LSA_ERR_DEVICE_DATA);
+                const float vs = KV_FP8 ? (v ? kvs[cur] : 0.f) : 1.f;
+                sm.rows[g][lane] = v ? cur : -1;
+                sm.vscale[g][lane] = vs;
+                sm.kscale[g][lane] = v ? vs * a.sm_scale_log2 : 0.f;
             }
-            asm volatile("bar.sync %0, %1;" :: "r"(1 + g), "r"(kGroupThreads) : "memory");
+            __syncwarp();
             uint8_t* tile = sm.kv[g];
             if (!KV_FP8) {
-                for (int i = gt; i < kRows * (kD / 8); i += kGroupThreads) {
+#pragma unroll 4
+                for (int i = lane; i < kRows * (kD / 8); i += 32) {
                     const int r = i / (kD / 8), c = i % (kD / 8);
                     const int row = sm.rows[g][r];
                     uint8_t* dst = tile + (c >> 3) * (kRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
@@ -137,12 +166,12 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                 cp_async_wait<0>();
             } else {
                 constexpr int kChunks = kRows * (kD / 16);             // 16 codes per chunk
-                constexpr int kBatch = 6;
-                for (int i0 = gt; i0 < kChunks; i0 += kGroupThreads * kBatch) {
+                constexpr int kBatch = 12;
+                for (int i0 = lane; i0 < kChunks; i0 += 32 * kBatch) {
                     uint4 raw[kBatch];
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
-                        const int i = i0 + u * kGroupThreads;
+                        const int i = i0 + u * 32;
                         raw[u] = make_uint4(0, 0, 0, 0);
                         if (i < kChunks) {
                             const int row = sm.rows[g][i / (kD / 16)];
@@ -151,7 +180,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                     }
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
-                        const int i = i0 + u * kGroupThreads;
+                        const int i = i0 + u * 32;
                         if (i >= kChunks) break;
                         const int r = i / (kD / 16), c = i % (kD / 16);
                         const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw[u]);
@@ -175,46 +204,59 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
             tc::mbar_arrive(&sm.kv_full[g]);
         }
     } else if (warp == 8) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: S_j and P_j V_j, each in order, whichever is ready
         const uint32_t idesc_s = tc::idesc_f16(128, kRows, 1);
         const uint32_t idesc_o = tc::idesc_f16_bmn(128, kHalf, 1);
         const uint32_t qaddr = tc::smem_u32(sm.q);
         if (tc::elect_one() && n_tiles > 0) {
-            auto issue_s = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!tc::mbar_wait(&sm.kv_full[s], (j >> 1) & 1, abort_flag)) return false;
-                tc::fence_proxy_async_smem();
-                tc::tc_fence_after();
-                const uint32_t kaddr = tc::smem_u32(sm.kv[s]);
-#pragma unroll 4
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint64_t ad = tc::sdesc_sw128(qaddr + (kk >> 2) * (128 * 128) + (kk & 3) * 32);
-                    const uint64_t bd = tc::sdesc_sw128(kaddr + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-                    tc::mma_f16_ss(s_col + s * 32, ad, bd, idesc_s, kk > 0);
-                }
-                tc::mma_commit(&sm.s_full[s]);
-                return true;
-            };
-            int last_pv = -1;
-            bool alive = issue_s(0);
-            for (int j = 0; j < n_tiles && alive; ++j) {
-                const int s = j & 1;
-                if (j + 1 < n_tiles && !issue_s(j + 1)) break;
-                if (!tc::mbar_wait(&sm.p_full[s], (j >> 1) & 1, abort_flag)) break;
-                tc::tc_fence_after();
-                const uint32_t vaddr = tc::smem_u32(sm.kv[s]) + (4 * half) * (kRows * 128);
+            int ns = 0, npv = 0;                 // next S tile, next PV tile
+            const uint64_t t0 = tc::global_ns();
+            uint32_t polls = 0;
+            while (npv < n_tiles) {
+                bool progressed = false;
+                // S_ns needs its KV tile and its S/P buffer free (P V_{ns-2} issued).
+                if (ns < n_tiles && ns <= npv + 1 && tc::mbar_try_wait(&sm.kv_full[ns % kStagesA], (ns / kStagesA) & 1)) {
+                    tc::fence_proxy_async_smem();
+                    tc::tc_fence_after();
+                    const int sb = ns & 1;
+                    const uint32_t kaddr = tc::smem_u32(sm.kv[ns % kStagesA]);
 #pragma unroll
-                for (int kk = 0; kk < kRows / 16; ++kk) {
-                    const uint64_t bd = tc::sdesc_sw128_lbo(vaddr + kk * 16 * 128, kRows * 128, 1024);
-                    tc::mma_f16_ts(o_col, p_col + s * 16 + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kQSmemAtoms * 4; ++kk) {
+                        const uint64_t ad = tc::sdesc_sw128(qaddr + (kk >> 2) * (128 * 128) + (kk & 3) * 32);
+                        const uint64_t bd = tc::sdesc_sw128(kaddr + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+                        tc::mma_f16_ss(s_col + sb * 32, ad, bd, idesc_s, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = kQSmemAtoms * 4; kk < kD / 16; ++kk) {
+                        const uint64_t bd = tc::sdesc_sw128(kaddr + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+                        tc::mma_f16_ts(s_col + sb * 32, qt_col + (kk - kQSmemAtoms * 4) * 8, bd, idesc_s, 1u);
+                    }
+                    tc::mma_commit(&sm.s_full[sb]);
+                    ++ns;
+                    progressed = true;
                 }
-                tc::mma_commit(&sm.kv_empty[s]);
-                tc::mma_commit(&sm.o_done);
-                last_pv = j;
+                // P V_npv needs the softmax of tile npv.
+                if (npv < ns && tc::mbar_try_wait(&sm.p_full[npv & 1], (npv >> 1) & 1)) {
+                    tc::tc_fence_after();
+                    const uint32_t vaddr = tc::smem_u32(sm.kv[npv % kStagesA]) + (4 * half) * (kRows * 128);
+#pragma unroll
+                    for (int kk = 0; kk < kRows / 16; ++kk) {
+                        const uint64_t bd = tc::sdesc_sw128_lbo(vaddr + kk * 16 * 128, kRows * 128, 1024);
+                        tc::mma_f16_ts(o_col, p_col + (npv & 1) * 16 + kk * 8, bd, idesc_o,
+                                       (npv > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(&sm.kv_empty[npv % kStagesA]);
+                    tc::mma_commit(&sm.o_done[npv & 1]);
+                    ++npv;
+                    progressed = true;
+                }
+                if (!progressed && (++polls & 255) == 0) {
+                    if (*abort_flag || tc::global_ns() - t0 > tc::kWaitNs * 4) { *abort_flag = 1; break; }
+                }
             }
-            if (last_pv >= 0) {                          // drain before TMEM is freed
+            if (npv > 0) {                          // drain before TMEM is freed
                 volatile int drain_abort = 0;
-                tc::mbar_wait(&sm.o_done, last_pv & 1, &drain_abort);
+                tc::mbar_wait(&sm.o_done[(npv - 1) & 1], ((npv - 1) >> 1) & 1, &drain_abort);
             }
         }
     } else {
@@ -225,42 +267,69 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
         float m_run = kNegInf, l_run = 0.f;
         bool alive = true;
         for (int j = 0; j < n_tiles; ++j) {
-            const int s = j & 1;
-            if (!tc::mbar_wait(&sm.s_full[s], (j >> 1) & 1, abort_flag)) { alive = false; break; }
-            // The tile's row scales / validity were written by the gather warps before kv_full.
-            if (!tc::mbar_wait(&sm.kv_full[s], (j >> 1) & 1, abort_flag)) { alive = false; break; }
+            const int sb = j & 1, st = j % kStagesA;
+            if (!tc::mbar_wait(&sm.s_full[sb], (j >> 1) & 1, abort_flag)) { alive = false; break; }
+            // The tile's row scales were written by the gather warp before kv_full.
+            if (!tc::mbar_wait(&sm.kv_full[st], (j / kStagesA) & 1, abort_flag)) { alive = false; break; }
+            // P buffer sb was last read by P V_{j-2}.
+            if (j >= 2 && !tc::mbar_wait(&sm.o_done[sb], ((j - 2) >> 1) & 1, abort_flag)) { alive = false; break; }
             tc::tc_fence_after();
             uint32_t sv[32];
-            tc::tmem_ld32(s_col + s * 32 + lane_off, sv);
+            tc::tmem_ld32(s_col + sb * 32 + lane_off, sv);
             tc::tmem_wait_ld();
-            if (j > 0 && !tc::mbar_wait(&sm.o_done, (j - 1) & 1, abort_flag)) { alive = false; break; }
             float x[32];
-            float mt = kNegInf;
+            const float4* ks4 = reinterpret_cast<const float4*>(sm.kscale[st]);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                x[i] = sm.valid[s][i] ? __uint_as_float(sv[i]) * sm.kscale[s][i] * a.sm_scale_log2 : kNegInf;
-                mt = fmaxf(mt, x[i]);
+            for (int i = 0; i < 8; ++i) {
+                const float4 k4 = ks4[i];
+                x[4 * i + 0] = k4.x != 0.f ? __uint_as_float(sv[4 * i + 0]) * k4.x : kNegInf;
+                x[4 * i + 1] = k4.y != 0.f ? __uint_as_float(sv[4 * i + 1]) * k4.y : kNegInf;
+                x[4 * i + 2] = k4.z != 0.f ? __uint_as_float(sv[4 * i + 2]) * k4.z : kNegInf;
+                x[4 * i + 3] = k4.w != 0.f ? __uint_as_float(sv[4 * i + 3]) * k4.w : kNegInf;
             }
+            float mx[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mx[i] = fmaxf(x[2 * i], x[2 * i + 1]);
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+            const float mt = mx[0];
             float alpha = 1.f;
             bool rescale = false;
             if (mt > m_run + 8.f) {
-                if (m_run != kNegInf) { alpha = exp2f(m_run - mt); rescale = true; }
+                if (m_run != kNegInf) { alpha = ex2(m_run - mt); rescale = true; }
                 l_run *= alpha;
                 m_run = mt;
             }
-            uint32_t pw[16];
-            float ls = 0.f;
+            const float mref = m_run == kNegInf ? 0.f : m_run;            // all rows masked so far: p = 0
+            float p[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float p0 = m_run == kNegInf ? 0.f : exp2f(x[2 * i] - m_run);
-                const float p1 = m_run == kNegInf ? 0.f : exp2f(x[2 * i + 1] - m_run);
-                ls += p0;
-                ls += p1;
-                pw[i] = pack_bf16x2(p0 * sm.kscale[s][2 * i], p1 * sm.kscale[s][2 * i + 1]);
+            for (int i = 0; i < 32; ++i) p[i] = ex2(x[i] - mref);         // ex2(-inf) = 0
+            float ps[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ps[i] = p[2 * i] + p[2 * i + 1];
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int i = 0; i < w; ++i) ps[i] += ps[i + w];
+            l_run += ps[0];
+            uint32_t pw[16];
+            const float4* vs4 = reinterpret_cast<const float4*>(sm.vscale[st]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 v4 = vs4[i];
+                pw[2 * i] = pack_bf16x2(p[4 * i] * v4.x, p[4 * i + 1] * v4.y);
+                pw[2 * i + 1] = pack_bf16x2(p[4 * i + 2] * v4.z, p[4 * i + 3] * v4.w);
             }
-            l_run += ls;
-            tc::tmem_st16(p_col + s * 16 + lane_off, pw);
+            tc::tmem_st16(p_col + sb * 16 + lane_off, pw);
             if (__any_sync(0xffffffffu, rescale)) {
+                // O must hold P V_{j-1} before it is rescaled.
+                if (j >= 1 && !tc::mbar_wait(&sm.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
+                    alive = false;
+                    break;
+                }
+                tc::tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < kHalf / 32; ++c) {
                     uint32_t ov[32];
@@ -273,10 +342,12 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
             }
             tc::tmem_wait_st();
             tc::tc_fence_before();
-            tc::mbar_arrive(&sm.p_full[s]);
+            tc::mbar_arrive(&sm.p_full[sb]);
         }
         // Epilogue: O / l, lse.
-        if (alive && n_tiles > 0 && !tc::mbar_wait(&sm.o_done, (n_tiles - 1) & 1, abort_flag)) alive = false;
+        if (alive && n_tiles > 0 &&
+            !tc::mbar_wait(&sm.o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag))
+            alive = false;
         tc::tc_fence_after();
         const float kLn2 = 0.69314718055994530942f;
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;

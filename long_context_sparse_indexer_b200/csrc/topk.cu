@@ -64,18 +64,26 @@ __device__ __forceinline__ void hist_add(int* hist, int bin, bool on) {
     if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
 }
 
-// Sums the histograms of all CTAs of the cluster (read through DSMEM) into `sum`, then finds
-// the bin where the count from the top first reaches `need`.  Identical in every CTA.
-__device__ void cluster_threshold(cg::cluster_group& cl, int* hist, int* sum, int nb, int need, int* s_warp,
-                                  int* s_bin, int* s_above) {
+// Sums the histograms of all CTAs of the cluster into `sum` in every CTA, then finds the bin
+// where the count from the top first reaches `need` (identical in every CTA).  CTA r adds up
+// the r-th eighth of the bins over the cluster (distributed shared memory loads) and writes
+// the sums into every CTA's `sum` (distributed shared memory stores).
+__device__ void cluster_threshold(cg::cluster_group& cl, int rank, int* hist, int* sum, int nb, int need,
+                                  int* s_warp, int* s_bin, int* s_above) {
     cl.sync();                                           // all local histograms complete
-    for (int i = threadIdx.x; i < nb; i += kTopkThreads) {
+    const int share = nb / kTopkCluster;
+    for (int i = threadIdx.x; i < share; i += kTopkThreads) {
+        const int bin = rank * share + i;
+        int v[kTopkCluster];
+#pragma unroll
+        for (int r = 0; r < kTopkCluster; ++r) v[r] = cl.map_shared_rank(hist, r)[bin];
         int s = 0;
 #pragma unroll
-        for (int r = 0; r < kTopkCluster; ++r) s += cl.map_shared_rank(hist, r)[i];
-        sum[i] = s;
+        for (int r = 0; r < kTopkCluster; ++r) s += v[r];
+#pragma unroll
+        for (int r = 0; r < kTopkCluster; ++r) cl.map_shared_rank(sum, r)[bin] = s;
     }
-    __syncthreads();
+    cl.sync();                                           // sums everywhere; peers done reading `hist`
     const int per = (nb + kTopkThreads - 1) / kTopkThreads;     // bins per thread, from the top
     int local = 0;
     for (int i = 0; i < per; ++i) {
@@ -93,7 +101,6 @@ __device__ void cluster_threshold(cg::cluster_group& cl, int* hist, int* sum, in
         run += h;
     }
     __syncthreads();
-    cl.sync();                                           // peers done reading `hist` before it is reused
 }
 
 // Cluster-wide exclusive prefix of one int per CTA (the value in `slot` of each CTA).
@@ -162,20 +169,32 @@ topk_kernel(TopkArgs a) {
     for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
     if (threadIdx.x == 0) s_nvalid = 0;
     if (CACHED) {
-        for (int cc = c0 + threadIdx.x * 4; cc < c1; cc += kTopkThreads * 4) {
-            float f[4];
-            if (cc + 3 < c1 && (((uintptr_t)(row + cc)) & 15) == 0) {
-                const float4 v4 = *reinterpret_cast<const float4*>(row + cc);
-                f[0] = v4.x; f[1] = v4.y; f[2] = v4.z; f[3] = v4.w;
-            } else {
+        // Batches of 8 independent 16-byte loads per thread, then conversion to keys.
+        constexpr int kB = 8;
+        const bool vec = (((uintptr_t)(row + c0)) & 15) == 0;
+        for (int base = c0 + threadIdx.x * 4; base < c1; base += kTopkThreads * 4 * kB) {
+            float f[kB][4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) f[u] = cc + u < c1 ? row[cc + u] : kNegInf;
+            for (int u = 0; u < kB; ++u) {
+                const int cc = base + u * kTopkThreads * 4;
+                if (vec && cc + 3 < c1) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(row + cc);
+                    f[u][0] = v4.x; f[u][1] = v4.y; f[u][2] = v4.z; f[u][3] = v4.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) f[u][e] = cc + e < c1 ? row[cc + e] : kNegInf;
+                }
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (cc + u >= c1) break;
-                if (f[u] != f[u]) report(a.status, LSA_ERR_DEVICE_DATA);
-                s_keys[cc + u - c0] = (f[u] != f[u] || f[u] == kNegInf) ? 0u : order_key(f[u]);
+            for (int u = 0; u < kB; ++u) {
+                const int cc = base + u * kTopkThreads * 4;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (cc + e >= c1) break;
+                    const float x = f[u][e];
+                    if (x != x) report(a.status, LSA_ERR_DEVICE_DATA);
+                    s_keys[cc + e - c0] = (x != x || x == kNegInf) ? 0u : order_key(x);
+                }
             }
         }
     }
@@ -201,7 +220,7 @@ topk_kernel(TopkArgs a) {
     uint32_t vstar = 0;
     int above = 0;
     if (!take_all && a.k > 0) {
-        cluster_threshold(cl, hist, hsum, 4096, a.k, s_warp, &s_bin, &s_above);
+        cluster_threshold(cl, rank, hist, hsum, 4096, a.k, s_warp, &s_bin, &s_above);
         const uint32_t b1 = (uint32_t)s_bin;
         above = s_above;
         // ---- pass 2: next 12 bits among keys with prefix b1
@@ -211,7 +230,7 @@ topk_kernel(TopkArgs a) {
             const uint32_t key = key_at(c + lane);
             hist_add(hist, (int)((key >> 8) & 0xfff), key != 0u && (key >> 20) == b1);
         }
-        cluster_threshold(cl, hist, hsum, 4096, a.k - above, s_warp, &s_bin, &s_above);
+        cluster_threshold(cl, rank, hist, hsum, 4096, a.k - above, s_warp, &s_bin, &s_above);
         const uint32_t b2 = (uint32_t)s_bin;
         above += s_above;
         // ---- pass 3: last 8 bits among keys with prefix (b1, b2)
@@ -222,7 +241,7 @@ topk_kernel(TopkArgs a) {
             const uint32_t key = key_at(c + lane);
             hist_add(hist, (int)(key & 0xff), key != 0u && (key >> 8) == pre);
         }
-        cluster_threshold(cl, hist, hsum, 256, a.k - above, s_warp, &s_bin, &s_above);
+        cluster_threshold(cl, rank, hist, hsum, 256, a.k - above, s_warp, &s_bin, &s_above);
         above += s_above;
         vstar = (pre << 8) | (uint32_t)s_bin;
     }
