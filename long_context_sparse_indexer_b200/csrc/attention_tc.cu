@@ -50,7 +50,7 @@ struct AttnSmem {
     alignas(16) float kscale[kStagesA][kRows];   // per-row FP8 scale x softmax scale (0 for masked rows)
     alignas(16) float vscale[kStagesA][kRows];   // per-row FP8 scale (1 for BF16)
     int rows[kStagesA][kRows];
-    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[2], p_full[2], o_done[2];
+    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[2], p_full[2], o_done[2], q_ready;
     uint32_t tmem_base;
     int abort;
 };
@@ -91,26 +91,26 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
             tc::mbar_init(&sm.p_full[i], 128);
             tc::mbar_init(&sm.o_done[i], 1);
         }
+        tc::mbar_init(&sm.q_ready, 128);
         sm.abort = 0;
         tc::fence_barrier_init();
     }
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
-    // Q dims 0..255 -> shared memory (K-major, 128-byte swizzle).
-    for (int i = threadIdx.x; i < 128 * (kQSmemAtoms * 8); i += kAThreads) {
-        const int h = i / (kQSmemAtoms * 8), c = i % (kQSmemAtoms * 8);
-        uint8_t* dst = sm.q + (c >> 3) * (128 * 128) + h * 128 + (((c & 7) ^ (h & 7)) << 4);
-        cp_async16(dst, qt + (size_t)h * kD + c * 8, true);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t o_col = tmem, s_col = tmem + 256, p_col = tmem + 320, qt_col = tmem + 352;
-    // Q dims 256..575 -> TMEM (softmax warps: thread = head = lane).
+    // The softmax warps load Q while the gather warps already fetch KV tiles: dims 0..255 into
+    // shared memory (K-major, 128-byte swizzle), dims 256..575 into TMEM (thread = head = lane).
     if (warp >= 4 && warp < 8) {
+        const int tq = threadIdx.x - 128;
+        for (int i = tq; i < 128 * (kQSmemAtoms * 8); i += 128) {
+            const int h = i / (kQSmemAtoms * 8), c = i % (kQSmemAtoms * 8);
+            uint8_t* dst = sm.q + (c >> 3) * (128 * 128) + h * 128 + (((c & 7) ^ (h & 7)) << 4);
+            cp_async16(dst, qt + (size_t)h * kD + c * 8, true);
+        }
+        cp_async_commit();
         const int h = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint4* src = reinterpret_cast<const uint4*>(qt + (size_t)h * kD + kQSmemAtoms * 64);
@@ -125,10 +125,11 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
             tc::tmem_st32(qt_col + c * 32 + lane_off, v);
         }
         tc::tmem_wait_st();
+        cp_async_wait<0>();
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&sm.q_ready);
     }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
 
     if (warp < 4) {
         // ---------------- gather producers: warp g owns stage g and the tiles j = g, g + 4, ...
@@ -208,7 +209,9 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
         const uint32_t idesc_s = tc::idesc_f16(128, kRows, 1);
         const uint32_t idesc_o = tc::idesc_f16_bmn(128, kHalf, 1);
         const uint32_t qaddr = tc::smem_u32(sm.q);
-        if (tc::elect_one() && n_tiles > 0) {
+        if (tc::elect_one() && n_tiles > 0 && tc::mbar_wait(&sm.q_ready, 0, abort_flag)) {
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_after();
             int ns = 0, npv = 0;                 // next S tile, next PV tile
             const uint64_t t0 = tc::global_ns();
             uint32_t polls = 0;

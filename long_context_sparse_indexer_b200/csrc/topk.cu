@@ -56,20 +56,17 @@ __device__ __forceinline__ int cta_inclusive_scan(int v, int* s_warp, int& total
     return res;
 }
 
-// Adds 1 to hist[bin] for every lane with `on`, one atomic per distinct bin in the warp.
+// Adds 1 to hist[bin] for every lane with `on` (shared-memory integer atomics).
 __device__ __forceinline__ void hist_add(int* hist, int bin, bool on) {
-    const unsigned act = __ballot_sync(0xffffffffu, on);
-    if (!on) return;
-    const unsigned peers = __match_any_sync(act, bin);
-    if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+    if (on) atomicAdd(&hist[bin], 1);
 }
 
 // Sums the histograms of all CTAs of the cluster into `sum` in every CTA, then finds the bin
 // where the count from the top first reaches `need` (identical in every CTA).  CTA r adds up
 // the r-th eighth of the bins over the cluster (distributed shared memory loads) and writes
 // the sums into every CTA's `sum` (distributed shared memory stores).
-__device__ void cluster_threshold(cg::cluster_group& cl, int rank, int* hist, int* sum, int nb, int need,
-                                  int* s_warp, int* s_bin, int* s_above) {
+__device__ int cluster_threshold(cg::cluster_group& cl, int rank, int* hist, int* sum, int nb, int need,
+                                 int* s_warp, int* s_bin, int* s_above) {
     cl.sync();                                           // all local histograms complete
     const int share = nb / kTopkCluster;
     for (int i = threadIdx.x; i < share; i += kTopkThreads) {
@@ -101,9 +98,11 @@ __device__ void cluster_threshold(cg::cluster_group& cl, int rank, int* hist, in
         run += h;
     }
     __syncthreads();
+    return total;
 }
 
-// Cluster-wide exclusive prefix of one int per CTA (the value in `slot` of each CTA).
+// Cluster-wide exclusive prefix of one int per CTA (the value in `slot` of each CTA).  Every
+// exchange uses its own slot, so the slot is never rewritten while a peer may still read it.
 __device__ int cluster_exclusive(cg::cluster_group& cl, int* slot, int rank, int& total) {
     cl.sync();
     int before = 0;
@@ -113,7 +112,6 @@ __device__ int cluster_exclusive(cg::cluster_group& cl, int* slot, int rank, int
         if (r < rank) before += v;
         total += v;
     }
-    cl.sync();
     return before;
 }
 
@@ -126,7 +124,7 @@ topk_kernel(TopkArgs a) {
     __shared__ int hist[4096];
     __shared__ int hsum[4096];
     __shared__ int s_warp[kTopkWarps];
-    __shared__ int s_bin, s_above, s_slot, s_nvalid;
+    __shared__ int s_bin, s_above, s_slot[2];
     extern __shared__ uint32_t s_keys[];          // CACHED: order key of each column of the segment, 0 = invalid
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
@@ -167,7 +165,6 @@ topk_kernel(TopkArgs a) {
 
     // ---- pass 1: top 12 bits (and, when cached, the segment's keys into shared memory)
     for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
-    if (threadIdx.x == 0) s_nvalid = 0;
     if (CACHED) {
         // Batches of 8 independent 16-byte loads per thread, then conversion to keys.
         constexpr int kB = 8;
@@ -199,7 +196,6 @@ topk_kernel(TopkArgs a) {
         }
     }
     __syncthreads();
-    int nvalid = 0;
     for (int c = w0; c < w1; c += 32) {
         const int cc = c + lane;
         if (!CACHED && cc < w1) {
@@ -207,20 +203,14 @@ topk_kernel(TopkArgs a) {
             if (f != f) report(a.status, LSA_ERR_DEVICE_DATA);
         }
         const uint32_t key = key_at(cc);
-        const bool v = key != 0u;
-        nvalid += v;
-        hist_add(hist, v ? (int)(key >> 20) : 0, v);
+        hist_add(hist, (int)(key >> 20), key != 0u);
     }
-    atomicAdd(&s_nvalid, nvalid);
-    __syncthreads();
-    if (threadIdx.x == 0) s_slot = s_nvalid;
-    int n_valid;
-    cluster_exclusive(cl, &s_slot, rank, n_valid);
+    // Cluster histogram of the top 12 bits; its total is the number of candidates.
+    const int n_valid = cluster_threshold(cl, rank, hist, hsum, 4096, a.k, s_warp, &s_bin, &s_above);
     const bool take_all = n_valid <= a.k;
     uint32_t vstar = 0;
     int above = 0;
     if (!take_all && a.k > 0) {
-        cluster_threshold(cl, rank, hist, hsum, 4096, a.k, s_warp, &s_bin, &s_above);
         const uint32_t b1 = (uint32_t)s_bin;
         above = s_above;
         // ---- pass 2: next 12 bits among keys with prefix b1
@@ -272,9 +262,9 @@ topk_kernel(TopkArgs a) {
     }
     int eq_cta;
     const int eq_wbase = cta_inclusive_scan(lane == 0 ? eq_w : 0, s_warp, eq_cta) - (lane == 0 ? eq_w : 0);
-    if (threadIdx.x == 0) s_slot = eq_cta;
+    if (threadIdx.x == 0) s_slot[0] = eq_cta;
     int eq_all;
-    const int eq_cbase = cluster_exclusive(cl, &s_slot, rank, eq_all);
+    const int eq_cbase = cluster_exclusive(cl, &s_slot[0], rank, eq_all);
     const int eq_base = eq_cbase + __shfl_sync(0xffffffffu, eq_wbase, 0);
     // B: kept entries per warp -> CTA prefix -> cluster prefix.
     int keep_w = 0;
@@ -294,9 +284,9 @@ topk_kernel(TopkArgs a) {
     }
     int keep_cta;
     const int keep_wbase = cta_inclusive_scan(lane == 0 ? keep_w : 0, s_warp, keep_cta) - (lane == 0 ? keep_w : 0);
-    if (threadIdx.x == 0) s_slot = keep_cta;
+    if (threadIdx.x == 0) s_slot[1] = keep_cta;
     int written;
-    const int keep_cbase = cluster_exclusive(cl, &s_slot, rank, written);
+    const int keep_cbase = cluster_exclusive(cl, &s_slot[1], rank, written);
     // C: write.
     {
         int eq_run = eq_base;
@@ -315,6 +305,7 @@ topk_kernel(TopkArgs a) {
             eq_run += __popc(eqm);
         }
     }
+    cl.sync();                    // no CTA leaves while a peer may still read its shared memory
     if (rank != kTopkCluster - 1) return;
     int n_out = a_lo + written;
     if (!a.raw) {
