@@ -313,7 +313,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, AttnArgs a, int
                 tc::mbar_wait(&sm.o_done[(npv - 1) & 1], ((npv - 1) >> 1) & 1, &drain_abort);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else {
         // ---------------- softmax / epilogue: thread = head = TMEM lane
         const int quarter = warp & 3;
         const int h = quarter * 32 + lane;
