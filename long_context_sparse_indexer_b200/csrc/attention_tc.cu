@@ -15,12 +15,10 @@
 // 16 K-steps, and a 4-stage ring of 32-row KV tiles (36 KB each) in the 128-byte-swizzled
 // K-major layout, read as the B operand of S (K-major) and of P V (MN-major).
 //
-//   warps 0..3 : gather.  BF16 rows with a row-uniform cache layout: warp 0 alone gathers every
-//                tile with TMA tile::gather4 (4 rows x 128 bytes per instruction, one-row
-//                boxes, 128-byte swizzle), up to 4 tiles ahead.  Otherwise warp g fills stage g
-//                with the tiles j = g, g+4, ... by 16-byte cp.async (FP8 rows are widened to
-//                BF16 exactly on the way).  Row indices are prefetched one tile ahead; per-row
-//                scale and validity go to shared memory.
+//   warps 0..3 : gather -- warp g fills stage g with the tiles j = g, g+4, ...: the tile's 32
+//                row indices (prefetched one tile ahead) go to shared memory, then the rows
+//                are copied with 16-byte cp.async (FP8 rows are widened to BF16 exactly on the
+//                way); per-row scale and validity.
 //   warp 8     : MMA issuer -- issues whatever is ready, in order per kind: S_j (16 SS + 20 TS
 //                MMAs, N = 32) once tile j has landed and P V_{j-2} has been issued, and
 //                O += P_j V_j (2 TS MMAs, N = 256) once the softmax of tile j is done.
@@ -29,8 +27,6 @@
 //                deterministic), P to TMEM as BF16; finally O / l and lse.
 //
 // All waits are bounded (2 s); a CTA that gives up reports LSA_ERR_TIMEOUT.
-#include <cstring>
-
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -65,19 +61,8 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* m, uint64_t* bar, int x, int y0,
-                                            int y1, int y2, int y3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-        :: "r"(tc::smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(tc::smem_u32(bar)), "r"(x),
-           "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-        : "memory");
-}
-
-template <bool KV_FP8, bool GTMA>
-__global__ void __launch_bounds__(kAThreads, 1)
-sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, AttnArgs a, int rows_per_seq) {
+template <bool KV_FP8>
+__global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int split = blockIdx.x, half = blockIdx.y, t = blockIdx.z;
@@ -100,8 +85,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, AttnArgs a, int
     const uint16_t* qt = a.q + (size_t)t * 128 * kD;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStagesA; ++i) { tc::mbar_init(&sm.kv_full[i], GTMA ? 1 : 32); tc::mbar_init(&sm.kv_empty[i], 1); }
-        if (GTMA) tc::prefetch_tmap(&kvmap);
+        for (int i = 0; i < kStagesA; ++i) { tc::mbar_init(&sm.kv_full[i], 32); tc::mbar_init(&sm.kv_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.s_full[i], 1);
             tc::mbar_init(&sm.p_full[i], 128);
@@ -147,42 +131,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, AttnArgs a, int
         tc::mbar_arrive(&sm.q_ready);
     }
 
-    if (GTMA && warp == 0) {
-        // ---------------- TMA gather: warp 0 issues every tile, lanes 0..7 one 4-row group each
-        auto fetch_row = [&](int j) -> int {
-            if (j >= n_tiles) return -1;
-            const int r0 = r_beg + j * kRows;
-            return lane < min(kRows, r_end - r0) ? irow[r0 + lane] : -1;
-        };
-        const int seq_row0 = max(b, 0) * rows_per_seq;
-        int nxt = fetch_row(0);
-        for (int j = 0; j < n_tiles; ++j) {
-            const int st = j % kStagesA;
-            const int cur = nxt;
-            nxt = fetch_row(j + 1);
-            if (!tc::mbar_wait(&sm.kv_empty[st], ((j / kStagesA) + 1) & 1, abort_flag)) break;
-            const int nr = min(kRows, r_end - (r_beg + j * kRows));
-            const bool v = cur >= 0 && cur < len;
-            if (lane < nr && !v) report(a.status, LSA_ERR_DEVICE_DATA);
-            sm.rows[st][lane] = v ? cur : -1;
-            sm.vscale[st][lane] = 1.f;
-            sm.kscale[st][lane] = v ? a.sm_scale_log2 : 0.f;
-            const int fr = seq_row0 + (v ? cur : 0);            // masked rows read row 0 of the sequence
-            const int y0 = __shfl_sync(0xffffffffu, fr, (lane & 7) * 4 + 0);
-            const int y1 = __shfl_sync(0xffffffffu, fr, (lane & 7) * 4 + 1);
-            const int y2 = __shfl_sync(0xffffffffu, fr, (lane & 7) * 4 + 2);
-            const int y3 = __shfl_sync(0xffffffffu, fr, (lane & 7) * 4 + 3);
-            __syncwarp();
-            if (lane == 0) tc::mbar_expect_tx(&sm.kv_full[st], kTileBytes);
-            __syncwarp();
-            if (lane < 8) {
-                uint8_t* tile = sm.kv[st];
-#pragma unroll
-                for (int atom = 0; atom < kAtoms; ++atom)
-                    tma_gather4(tile + atom * (kRows * 128) + lane * 512, &kvmap, &sm.kv_full[st], atom * 64, y0, y1, y2, y3);
-            }
-        }
-    } else if (!GTMA && warp < 4) {
+    if (warp < 4) {
         // ---------------- gather producers: warp g owns stage g and the tiles j = g, g + 4, ...
         const int g = warp;
         auto fetch_row = [&](int j) -> int {
@@ -451,14 +400,14 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, AttnArgs a, int
     }
 }
 
-template <bool KV_FP8, bool GTMA>
-cudaError_t launch_t(const CUtensorMap& m, const AttnArgs& a, int rows_per_seq, cudaStream_t st) {
+template <bool KV_FP8>
+cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
     const size_t smem = sizeof(AttnSmem) + 1024;
-    auto kern = sparse_attn_tc_kernel<KV_FP8, GTMA>;
+    auto kern = sparse_attn_tc_kernel<KV_FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_split, 2, a.T);
-    kern<<<grid, kAThreads, smem, st>>>(m, a, rows_per_seq);
+    kern<<<grid, kAThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -470,26 +419,7 @@ bool sparse_attn_tc_supported(const AttnArgs& a, int DQK, int DV, bool sep_v) {
 }
 
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, bool kv_fp8, cudaStream_t st) {
-    CUtensorMap m;
-    memset(&m, 0, sizeof(m));
-    if (kv_fp8) return launch_t<true, false>(m, a, 0, st);
-    // TMA gathers need every sequence's rows on one row grid: seq_stride a multiple of tok_stride,
-    // and row indices that fit in 32 bits.
-    const int64_t tok = a.kv_tok_b, seq = a.kv_seq_b;
-    const int64_t rps = tok > 0 && seq % tok == 0 ? seq / tok : -1;
-    const int64_t total_rows = rps > 0 ? (int64_t)(a.B - 1) * rps + a.L_alloc : -1;
-    if (rps > 0 && total_rows < ((int64_t)1 << 31) && encode_fn()) {
-        const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)total_rows};
-        const cuuint64_t strides[1] = {(cuuint64_t)tok};
-        const cuuint32_t box[2] = {64, 1};
-        const cuuint32_t estr[2] = {1, 1};
-        if (encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint8_t*>(a.kv), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
-            return launch_t<false, true>(m, a, (int)rps, st);
-        memset(&m, 0, sizeof(m));
-    }
-    return launch_t<false, false>(m, a, 0, st);
+    return kv_fp8 ? launch_t<true>(a, st) : launch_t<false>(a, st);
 }
 
 }  // namespace lsa

@@ -104,46 +104,28 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         sm.pos[gi] = ok ? pos : -1;
         sm.ok[gi] = ok;
     }
-    // Queries -> f16, scaled per head, into the 128-byte-swizzled K-major B layout.  Each warp
-    // takes rows warp, warp + 10, ...; the rows' loads are issued in batches before use.
-    {
-        constexpr int kWarps = kTcThreads / 32;
-        constexpr int kQB = 4;
-        for (int r0 = warp; r0 < G * H_I; r0 += kWarps * kQB) {
-            uint2 raw[kQB];
-#pragma unroll
-            for (int u = 0; u < kQB; ++u) {
-                const int rowi = r0 + u * kWarps;
-                raw[u] = make_uint2(0, 0);
-                if (rowi < G * H_I) {
-                    const int gi = rowi / H_I, h = rowi % H_I;
-                    raw[u] = *reinterpret_cast<const uint2*>(a.q + ((size_t)(t0 + gi) * H_I + h) * 128 + 4 * lane);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kQB; ++u) {
-                const int rowi = r0 + u * kWarps;
-                if (rowi >= G * H_I) break;
-                const int gi = rowi / H_I, h = rowi % H_I;
-                float v[4];
-                v[0] = bf16_bits_to_float((uint16_t)(raw[u].x & 0xffff)); v[1] = bf16_bits_to_float((uint16_t)(raw[u].x >> 16));
-                v[2] = bf16_bits_to_float((uint16_t)(raw[u].y & 0xffff)); v[3] = bf16_bits_to_float((uint16_t)(raw[u].y >> 16));
-                float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-                m = warp_max(m);
-                const int e = (int)((__float_as_uint(m) >> 23) & 0xff) - 127;
-                int k = m > 0.f ? 14 - e : 0;
-                k = max(-126, min(126, k));
-                const float sc = exp2i(k);
-                const uint32_t h01 = (uint32_t)__half_as_ushort(__float2half_rn(v[0] * sc)) |
-                                     ((uint32_t)__half_as_ushort(__float2half_rn(v[1] * sc)) << 16);
-                const uint32_t h23 = (uint32_t)__half_as_ushort(__float2half_rn(v[2] * sc)) |
-                                     ((uint32_t)__half_as_ushort(__float2half_rn(v[3] * sc)) << 16);
-                const int d = 4 * lane, atom = d >> 6, c16 = (d & 63) >> 3, inb = (d & 7) * 2;
-                uint8_t* dst = sm.q[atom] + (rowi >> 3) * 1024 + (rowi & 7) * 128 + ((c16 ^ (rowi & 7)) << 4) + inb;
-                *reinterpret_cast<uint2*>(dst) = make_uint2(h01, h23);
-                if (lane == 0) sm.w[rowi] = a.w[(size_t)(t0 + gi) * H_I + h] * exp2i(-k);
-            }
-        }
+    // Queries -> f16, scaled per head, into the 128-byte-swizzled K-major B layout.
+    for (int rowi = warp; rowi < G * H_I; rowi += kTcThreads / 32) {
+        const int gi = rowi / H_I, h = rowi % H_I;
+        const uint16_t* src = a.q + ((size_t)(t0 + gi) * H_I + h) * 128;
+        const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);      // elements 4l .. 4l+3
+        float v[4];
+        v[0] = bf16_bits_to_float((uint16_t)(raw.x & 0xffff)); v[1] = bf16_bits_to_float((uint16_t)(raw.x >> 16));
+        v[2] = bf16_bits_to_float((uint16_t)(raw.y & 0xffff)); v[3] = bf16_bits_to_float((uint16_t)(raw.y >> 16));
+        float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+        m = warp_max(m);
+        const int e = (int)((__float_as_uint(m) >> 23) & 0xff) - 127;
+        int k = m > 0.f ? 14 - e : 0;
+        k = max(-126, min(126, k));
+        const float sc = exp2i(k);
+        const uint32_t h01 = (uint32_t)__half_as_ushort(__float2half_rn(v[0] * sc)) |
+                             ((uint32_t)__half_as_ushort(__float2half_rn(v[1] * sc)) << 16);
+        const uint32_t h23 = (uint32_t)__half_as_ushort(__float2half_rn(v[2] * sc)) |
+                             ((uint32_t)__half_as_ushort(__float2half_rn(v[3] * sc)) << 16);
+        const int d = 4 * lane, atom = d >> 6, c16 = (d & 63) >> 3, inb = (d & 7) * 2;
+        uint8_t* dst = sm.q[atom] + (rowi >> 3) * 1024 + (rowi & 7) * 128 + ((c16 ^ (rowi & 7)) << 4) + inb;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(h01, h23);
+        if (lane == 0) sm.w[rowi] = a.w[(size_t)(t0 + gi) * H_I + h] * exp2i(-k);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -276,18 +258,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
             tc::tc_fence_after();
             for (int gi = 0; gi < G; ++gi) {
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int h0 = 0; h0 < H_I; h0 += 64) {
-                    // Two 32-column TMEM loads in flight, one wait (H_I is a multiple of 32).
-                    uint32_t v[64];
-                    tc::tmem_ld32(d_col + db * N + gi * H_I + h0 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(v));
-                    const bool two = h0 + 32 < H_I;
-                    if (two) tc::tmem_ld32(d_col + db * N + gi * H_I + h0 + 32 + lane_off,
-                                           *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                for (int h0 = 0; h0 < H_I; h0 += 32) {
+                    uint32_t v[32];
+                    tc::tmem_ld32(d_col + db * N + gi * H_I + h0 + lane_off, v);
                     tc::tmem_wait_ld();
                     const float4* wp = reinterpret_cast<const float4*>(sm.w + gi * H_I + h0);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        if (i >= 8 && !two) break;
+                    for (int i = 0; i < 8; ++i) {
                         const float4 ww = wp[i];
                         acc[0] = fmaf(ww.x, fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), acc[0]);
                         acc[1] = fmaf(ww.y, fmaxf(__uint_as_float(v[4 * i + 1]), 0.f), acc[1]);
@@ -318,7 +295,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
     }
 }
 
-}  // namespace
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiled encode_fn() {
     static EncodeTiled fn = nullptr;
@@ -332,8 +311,6 @@ EncodeTiled encode_fn() {
     });
     return fn;
 }
-
-namespace {
 
 template <int N>
 cudaError_t launch_n(const CUtensorMap& m, const CUtensorMap& sm, const TcArgs& ta, cudaStream_t st) {

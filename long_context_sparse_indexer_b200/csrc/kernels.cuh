@@ -1,8 +1,6 @@
 // Internal kernel interfaces of the LSA library (argument blocks and host launchers).
 #pragma once
 
-#include <cuda.h>
-
 #include "common.cuh"
 
 namespace lsa {
@@ -96,12 +94,6 @@ struct AttnArgs {
     float* part_lse;            // [T][n_split][H]
     int32_t* status;
 };
-
-// cuTensorMapEncodeTiled from the driver (looked up once through the runtime); NULL if unavailable.
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-EncodeTiled encode_fn();
 
 cudaError_t launch_index_score(IndexArgs a, int H_I, int D_I, bool fp8, cudaStream_t st);
 bool index_score_tc_supported(const IndexArgs& a, int H_I, int D_I, bool fp8);
