@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                 tc::mbar_wait(&sm.o_done[(npv - 1) & 1], ((npv - 1) >> 1) & 1, &drain_abort);
             }
         }
-    } else {
+    } else if (warp >= 4 && warp < 8) {
         // ---------------- softmax / epilogue: thread = head = TMEM lane
         const int quarter = warp & 3;
         const int h = quarter * 32 + lane;
