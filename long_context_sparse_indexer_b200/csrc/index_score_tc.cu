@@ -104,28 +104,55 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         sm.pos[gi] = ok ? pos : -1;
         sm.ok[gi] = ok;
     }
-    // Queries -> f16, scaled per head, into the 128-byte-swizzled K-major B layout.
-    for (int rowi = warp; rowi < G * H_I; rowi += kTcThreads / 32) {
-        const int gi = rowi / H_I, h = rowi % H_I;
-        const uint16_t* src = a.q + ((size_t)(t0 + gi) * H_I + h) * 128;
-        const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);      // elements 4l .. 4l+3
-        float v[4];
-        v[0] = bf16_bits_to_float((uint16_t)(raw.x & 0xffff)); v[1] = bf16_bits_to_float((uint16_t)(raw.x >> 16));
-        v[2] = bf16_bits_to_float((uint16_t)(raw.y & 0xffff)); v[3] = bf16_bits_to_float((uint16_t)(raw.y >> 16));
-        float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-        m = warp_max(m);
-        const int e = (int)((__float_as_uint(m) >> 23) & 0xff) - 127;
-        int k = m > 0.f ? 14 - e : 0;
-        k = max(-126, min(126, k));
-        const float sc = exp2i(k);
-        const uint32_t h01 = (uint32_t)__half_as_ushort(__float2half_rn(v[0] * sc)) |
-                             ((uint32_t)__half_as_ushort(__float2half_rn(v[1] * sc)) << 16);
-        const uint32_t h23 = (uint32_t)__half_as_ushort(__float2half_rn(v[2] * sc)) |
-                             ((uint32_t)__half_as_ushort(__float2half_rn(v[3] * sc)) << 16);
-        const int d = 4 * lane, atom = d >> 6, c16 = (d & 63) >> 3, inb = (d & 7) * 2;
-        uint8_t* dst = sm.q[atom] + (rowi >> 3) * 1024 + (rowi & 7) * 128 + ((c16 ^ (rowi & 7)) << 4) + inb;
-        *reinterpret_cast<uint2*>(dst) = make_uint2(h01, h23);
-        if (lane == 0) sm.w[rowi] = a.w[(size_t)(t0 + gi) * H_I + h] * exp2i(-k);
+    // Queries -> f16, scaled per head, into the 128-byte-swizzled K-major B layout.  Thread i
+    // handles 16-byte chunk i (8 elements) of the group's N rows; the 16 chunks of a row sit in
+    // 16 consecutive lanes, which reduce the row maximum by shuffles.  All loads of a batch are
+    // issued before use.
+    {
+        constexpr int kQB = 4;
+        const int nchunks = N * 16;                       // a multiple of 32
+        for (int base = threadIdx.x; base < nchunks; base += kTcThreads * kQB) {
+            uint4 raw[kQB];
+#pragma unroll
+            for (int u = 0; u < kQB; ++u) {
+                const int i = base + u * kTcThreads;
+                const int rowi = i >> 4;
+                raw[u] = i < nchunks ? *reinterpret_cast<const uint4*>(
+                                           a.q + ((size_t)(t0 + rowi / H_I) * H_I + rowi % H_I) * 128 + (i & 15) * 8)
+                                     : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kQB; ++u) {
+                const int i = base + u * kTcThreads;
+                if (i >= nchunks) break;                  // warp-uniform: nchunks is a multiple of 32
+                const int rowi = i >> 4, cc = i & 15;
+                const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw[u]);
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    v[2 * e] = bf16_bits_to_float((uint16_t)(wd[e] & 0xffff));
+                    v[2 * e + 1] = bf16_bits_to_float((uint16_t)(wd[e] >> 16));
+                }
+                float m = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                const int ex = (int)((__float_as_uint(m) >> 23) & 0xff) - 127;
+                int k = m > 0.f ? 14 - ex : 0;
+                k = max(-126, min(126, k));
+                const float sc = exp2i(k);
+                uint32_t hv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    hv[e] = (uint32_t)__half_as_ushort(__float2half_rn(v[2 * e] * sc)) |
+                            ((uint32_t)__half_as_ushort(__float2half_rn(v[2 * e + 1] * sc)) << 16);
+                const int atom = cc >> 3, c16 = cc & 7;
+                uint8_t* dst = sm.q[atom] + (rowi >> 3) * 1024 + (rowi & 7) * 128 + ((c16 ^ (rowi & 7)) << 4);
+                *reinterpret_cast<uint4*>(dst) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                if (cc == 0) sm.w[rowi] = a.w[(size_t)(t0 + rowi / H_I) * H_I + rowi % H_I] * exp2i(-k);
+            }
+        }
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
