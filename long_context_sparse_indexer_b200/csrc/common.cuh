@@ -47,6 +47,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // 2^k as a float for -126 <= k <= 127.
 __device__ __forceinline__ float exp2i(int k) { return __int_as_float((127 + k) << 23); }
 
+// Two independent FP32 fused multiply-adds (round to nearest) in one packed sm_100 instruction:
+// (d.x, d.y) = (a.x * b.x + c.x, a.y * b.y + c.y), each rounded exactly as fmaf would.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{ .reg .b64 ra, rb, rc, rd;\n"
+        "mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; mov.b64 rc, {%6, %7};\n"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n"
+        "mov.b64 {%0, %1}, rd; }"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
 // Monotone map of a float to uint32 (larger float -> larger key); -0 maps like +0.
 __device__ __forceinline__ uint32_t order_key(float f) {
     uint32_t b = __float_as_uint(f);
