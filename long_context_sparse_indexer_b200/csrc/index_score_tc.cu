@@ -4,6 +4,16 @@
 // the lightweight indexer scoring every cached key; DSA form sum_h w_h * ReLU(q_h . k)),
 // restated for sm_100a as a persistent kernel, one CTA per SM.
 //
+// Arithmetic.  The key tile goes to the tensor core as it sits in the cache: 128 e4m3 codes per
+// key row, MMA kind::f8f6f4 with A read from shared memory.  Each BF16 query row q_h is scaled by
+// a power of two 2^s_h (its largest magnitude into [128, 256)) and split into two e4m3 rows,
+// hi = rn(q_h 2^s_h) and lo = rn(q_h 2^s_h - hi).  The residual of a bf16 value after rounding
+// to 4 significant bits has at most 4 significant bits, so hi + lo equals q_h 2^s_h exactly for
+// every element whose magnitude is at least 2^-10 of the row maximum; smaller elements keep an
+// absolute error below 2^-17 of the row maximum.  The MMA runs over K = 256 (the key row twice,
+// against hi then lo), so the FP32 accumulator holds 2^s_h (q_h . k); products of e4m3 values are
+// exact.  2^-s_h is folded into the head weight.
+//
 // Scheduling.  Query tokens come in groups of G <= 4 tokens of one sequence (N = G*H_I <= 256
 // query rows share every key row).  A group's key range is cut into 128-key tiles; only tiles
 // holding a visible key are active.  Every CTA counts the active tiles of all groups, takes an
@@ -11,27 +21,20 @@
 // one group reuse its prepared queries; a CTA prepares a group's queries once ("epoch"), into
 // one of two buffers, so the next group's preparation overlaps the current group's tiles.
 //
-//   warp 0      : TMA producer -- key tiles (two 64-row boxes, 128-byte swizzle) and their
-//                 per-token scales into a KS-stage shared-memory ring; allocates / frees TMEM.
-//   warp 1      : MMA issuer -- per tile and accumulator slot, 8 x tcgen05.mma kind::f16
-//                 (M = 128 keys, N = min(N, 128), K = 16), A from TMEM, B (queries) from smem.
-//   warps 2..5  : converters -- thread = key row (= TMEM lane): widen the row's 128 FP8 codes to
-//                 f16 (exact) into one of 4 TMEM A stages; at each epoch, prepare the group's
-//                 queries: f16 scaled per head by a power of two, 128-byte-swizzled K-major.
-//   warps 6..13 : epilogue, two warpgroups -- thread = key row: load the accumulator row, apply
-//                 ReLU, the weighted head sum (four partial sums combined in a fixed order) and
-//                 the token's FP8 scale, store.
+//   warp 0      : TMA producer -- key tiles (two 64-row boxes, 128-byte swizzle, which is the
+//                 K-major operand layout) and their per-token scales into a KS-stage ring;
+//                 allocates / frees TMEM.
+//   warp 1      : MMA issuer -- per tile, 8 x tcgen05.mma kind::f8f6f4 (M = 128 keys, N, K = 32)
+//                 into one of 512 / N accumulator slots; its commit frees the key stage.
+//   warps 2..5  : query preparation, once per epoch (hi / lo split, 128-byte-swizzled K-major).
+//   warps 6..13 : epilogue, two warpgroups taking alternate tiles -- thread = key row (= TMEM
+//                 lane): load the accumulator row, apply ReLU, the weighted head sum (eight
+//                 partial sums combined in a fixed order) and the token's FP8 scale, store.
 //
-// TMEM: 4 A stages x 64 columns, then 256 / min(N, 128) accumulator slots of min(N, 128)
-// columns.  N <= 128: tile j uses slot j % slots and the epilogue warpgroups take alternate
-// tiles.  N = 256: a tile's two halves go to slots 0 and 1 and warpgroup h always takes half h,
-// so the epilogue of one half overlaps the MMA of the other.  Either way every slot has a
-// single consumer warpgroup, which keeps the mbarrier phase parities unambiguous.
-//
-// The power-of-two query scaling is exact for all values within 2^28 of the head's maximum;
-// its inverse is folded into the head weight.  Products of f16 values are exact in the FP32
-// accumulator.  All waits are bounded (2 s); a CTA that gives up reports LSA_ERR_TIMEOUT and
-// returns after its copies and MMAs in flight have landed and its TMEM is freed.
+// Every accumulator slot has a single consumer warpgroup (slot j % slots, an even count), which
+// keeps the mbarrier phase parities unambiguous.  All waits are bounded (2 s); a CTA that gives
+// up reports LSA_ERR_TIMEOUT and returns after its copies and MMAs in flight have landed and its
+// TMEM is freed.
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -45,11 +48,10 @@ namespace {
 
 constexpr int kPThreads = 448;         // 14 warps
 constexpr int kPWarps = kPThreads / 32;
-constexpr int kTile = 128;             // keys per MMA tile
-constexpr int kKeyTileBytes = kTile * 128;
+constexpr int kBlock = 128;            // keys per MMA (M); a tile is NB such blocks
+constexpr int kBlockBytes = kBlock * 128;
 constexpr int kMaxG = 4;
 constexpr int kMaxGroups = 2048;       // query-token groups one launch schedules
-constexpr int kAStages = 4;            // A-operand (widened keys) stages in TMEM
 
 struct PArgs {
     IndexArgs a;
@@ -57,44 +59,42 @@ struct PArgs {
     int scale_tma;                     // per-token scales arrive by TMA with the keys
 };
 
-template <int N, int KS>
+template <int N, int NB, int KS>
 struct PSmem {
-    static constexpr int NS = N < 128 ? N : 128;          // accumulator slot width
-    static constexpr int kSub = N / NS;                    // slots per tile
-    static constexpr int kSlots = 256 / NS;
-    alignas(1024) uint8_t keys[KS][kKeyTileBytes];
-    alignas(1024) uint8_t q[2][2][N * 128];              // [buffer][K atom]: B operand, SW128
-    alignas(16) float scl[KS][kTile];                    // per-token FP8 scales of each key tile
-    alignas(16) float w[2][N];                           // head weights (inverse query scale folded in)
+    static constexpr int kSlots = (512 / (NB * N)) < 8 ? (512 / (NB * N)) : 8;
+    alignas(1024) uint8_t keys[KS][NB * kBlockBytes];
+    alignas(1024) uint8_t q[2][2][N * 128];              // [buffer][hi, lo]: B operand, e4m3, SW128
+    alignas(16) float scl[KS][NB * kBlock];              // per-token FP8 scales of each key tile
+    alignas(16) float w[2][N];                           // head weights times 2^-s
     int pos[2][kMaxG], ok[2][kMaxG];
     int tstart[kMaxGroups + 1];                          // exclusive prefix sums of active tiles
-    uint64_t full_k[KS], empty_k[KS], a_full[kAStages], a_empty[kAStages];
+    uint64_t full_k[KS], empty_k[KS];
     uint64_t d_full[kSlots], d_empty[kSlots];
     uint64_t q_full[2], q_free[2][2];                    // q_free[buffer][epilogue warpgroup]
     uint32_t tmem_base;
     int abort;
 };
 
-// Walks a CTA's tiles in order: group, tile within the group, and the CTA-local group epoch.
-struct TileCursor {
+// Walks a CTA's tiles k_lo, k_lo + 1, ...: the group g of the current tile and the CTA-local
+// group epoch (0 for the group of tile k_lo, +1 at every change of group).
+struct Walk {
     const int* tstart;
-    int n_groups;
-    int g = 0, epoch = -1, lt = 0;
-    __device__ void seek(int k) {
-        int ng = g;
-        if (epoch < 0) {                                  // first tile: binary search
-            int lo = 0, hi = n_groups - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (tstart[mid + 1] > k) hi = mid; else lo = mid + 1;
-            }
-            ng = lo;
-        } else {
-            while (tstart[ng + 1] <= k) ++ng;
+    int g, next_b, epoch;
+    __device__ Walk(const int* ts, int n_groups, int k) : tstart(ts), epoch(0) {
+        int lo = 0, hi = n_groups - 1;                    // the group holding tile k
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (ts[mid + 1] > k) hi = mid; else lo = mid + 1;
         }
-        if (ng != g || epoch < 0) ++epoch;
-        g = ng;
-        lt = k - tstart[g];
+        g = lo;
+        next_b = ts[g + 1];
+    }
+    // Moves to tile k (never backwards); true when the group changed.
+    __device__ bool to(int k) {
+        if (k < next_b) return false;
+        do { ++g; next_b = tstart[g + 1]; } while (k >= next_b);
+        ++epoch;
+        return true;
     }
 };
 
@@ -134,12 +134,131 @@ __device__ void cta_exclusive_scan(int* tstart, int n, int* s_tmp) {
     __syncthreads();
 }
 
-template <int N, int KS>
+// Two floats to two e4m3 codes (round to nearest even, saturating): x0 in the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float x0, float x1) {
+    uint16_t r;
+    asm("{ .reg .b16 t; cvt.rn.satfinite.e4m3x2.f32 t, %1, %2; mov.b16 %0, t; }" : "=h"(r) : "f"(x1), "f"(x0));
+    return r;
+}
+
+// Decodes two e4m3 codes (low byte first) to floats, exactly.
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t v) {
+    const uint32_t h = e4m3x2_to_f16x2(v);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// One epoch's query preparation by 128 threads (thread ct).  Work item i: row n = i / 8 (token
+// n / H_I, head n % H_I), 16-element chunk c = i % 8; the 8 chunks of a row sit in 8 consecutive
+// lanes, which reduce the row maximum by shuffles.  Loads are issued four items at a time.
+template <int N>
+__device__ void prepare_queries(const IndexArgs& a, int t0, int H_I, int ct, uint8_t* q_hi, uint8_t* q_lo,
+                                float* w_out) {
+    constexpr int kB = 4;
+    for (int i0 = ct; i0 < N * 8; i0 += 128 * kB) {
+        uint4 raw[kB][2];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int i = i0 + u * 128;
+            if (i < N * 8) {                                  // warp-uniform: N * 8 is a multiple of 128
+                const int n = i >> 3, c = i & 7;
+                const uint16_t* src = a.q + ((size_t)(t0 + n / H_I) * H_I + n % H_I) * 128 + c * 16;
+                raw[u][0] = *reinterpret_cast<const uint4*>(src);
+                raw[u][1] = *reinterpret_cast<const uint4*>(src + 8);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int i = i0 + u * 128;
+            if (i >= N * 8) break;
+            const int n = i >> 3, c = i & 7;
+            const uint32_t wd[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                                    raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                v[2 * e] = bf16_bits_to_float((uint16_t)(wd[e] & 0xffff));
+                v[2 * e + 1] = bf16_bits_to_float((uint16_t)(wd[e] >> 16));
+            }
+            float m = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[e]));
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            // 2^s brings the maximum into [128, 256): s = 7 - floor(log2 m).
+            const int ex = (int)((__float_as_uint(m) >> 23) & 0xff) - 127;
+            int s = m > 0.f ? 7 - ex : 0;
+            s = max(-126, min(126, s));
+            const float sc = exp2i(s);
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float x0 = v[4 * e] * sc, x1 = v[4 * e + 1] * sc, x2 = v[4 * e + 2] * sc, x3 = v[4 * e + 3] * sc;
+                const uint16_t h01 = f32x2_to_e4m3x2(x0, x1), h23 = f32x2_to_e4m3x2(x2, x3);
+                const float2 d01 = e4m3x2_to_f32x2(h01), d23 = e4m3x2_to_f32x2(h23);
+                const uint16_t l01 = f32x2_to_e4m3x2(x0 - d01.x, x1 - d01.y);
+                const uint16_t l23 = f32x2_to_e4m3x2(x2 - d23.x, x3 - d23.y);
+                hw[e] = (uint32_t)h01 | ((uint32_t)h23 << 16);
+                lw[e] = (uint32_t)l01 | ((uint32_t)l23 << 16);
+            }
+            const int off = (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4);
+            *reinterpret_cast<uint4*>(q_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(q_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            if (c == 0) w_out[n] = a.w[(size_t)(t0 + n / H_I) * H_I + n % H_I] * exp2i(-s);
+        }
+    }
+}
+
+// Weighted ReLU head sums of two accumulator rows held by this thread: item a (columns
+// ca .. ca + H_I - 1 of the TMEM row, weights wa) and item b (cb, wb; skipped unless `two`).
+// Head h goes to partial sum h % 8, two per packed FMA; the eight sums are combined pairwise in a
+// fixed order.  The two items are interleaved 32 heads at a time for instruction-level
+// parallelism; when both use the same weights (same token) they share the weight loads.
+__device__ __forceinline__ void head_sums2(uint32_t ca, uint32_t cb, const float* wa, const float* wb, int H_I,
+                                           bool two, float& out_a, float& out_b) {
+    float2 aa[4], ab[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { aa[i] = make_float2(0.f, 0.f); ab[i] = make_float2(0.f, 0.f); }
+    const bool same = wa == wb;
+    for (int h0 = 0; h0 < H_I; h0 += 32) {
+        uint32_t va[32], vb[32];
+        tc::tmem_ld32(ca + h0, va);
+        if (two) tc::tmem_ld32(cb + h0, vb);
+        tc::tmem_wait_ld();
+        const float4* pa = reinterpret_cast<const float4*>(wa + h0);
+        const float4* pb = reinterpret_cast<const float4*>(wb + h0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 w4 = pa[i];
+            aa[(i & 1) * 2] = ffma2(make_float2(w4.x, w4.y),
+                                    make_float2(fmaxf(__uint_as_float(va[4 * i]), 0.f), fmaxf(__uint_as_float(va[4 * i + 1]), 0.f)),
+                                    aa[(i & 1) * 2]);
+            aa[(i & 1) * 2 + 1] = ffma2(make_float2(w4.z, w4.w),
+                                        make_float2(fmaxf(__uint_as_float(va[4 * i + 2]), 0.f), fmaxf(__uint_as_float(va[4 * i + 3]), 0.f)),
+                                        aa[(i & 1) * 2 + 1]);
+            if (two) {
+                float4 u4 = w4;
+                if (!same) u4 = pb[i];
+                ab[(i & 1) * 2] = ffma2(make_float2(u4.x, u4.y),
+                                        make_float2(fmaxf(__uint_as_float(vb[4 * i]), 0.f), fmaxf(__uint_as_float(vb[4 * i + 1]), 0.f)),
+                                        ab[(i & 1) * 2]);
+                ab[(i & 1) * 2 + 1] = ffma2(make_float2(u4.z, u4.w),
+                                            make_float2(fmaxf(__uint_as_float(vb[4 * i + 2]), 0.f), fmaxf(__uint_as_float(vb[4 * i + 3]), 0.f)),
+                                            ab[(i & 1) * 2 + 1]);
+            }
+        }
+    }
+    out_a = ((aa[0].x + aa[0].y) + (aa[1].x + aa[1].y)) + ((aa[2].x + aa[2].y) + (aa[3].x + aa[3].y));
+    out_b = ((ab[0].x + ab[0].y) + (ab[1].x + ab[1].y)) + ((ab[2].x + ab[2].y) + (ab[3].x + ab[3].y));
+}
+
+template <int N, int NB, int KS>
 __global__ void __launch_bounds__(kPThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap smap,
                       PArgs pa) {
-    using Smem = PSmem<N, KS>;
-    constexpr int NS = Smem::NS, kSub = Smem::kSub, kSlots = Smem::kSlots;
+    using Smem = PSmem<N, NB, KS>;
+    constexpr int kSlots = Smem::kSlots;
+    constexpr int TK = NB * kBlock;                      // keys per tile
+    constexpr int SW = NB * N;                           // TMEM columns per accumulator slot
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ int s_tmp[32];
@@ -151,9 +270,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
 
     // ---- set-up: barriers, TMEM, active tiles per group and this CTA's share
     if (threadIdx.x == 0) {
-        // A key stage is free once the converters have read its keys and the epilogue its scales.
-        for (int s = 0; s < KS; ++s) { tc::mbar_init(&sm.full_k[s], 1); tc::mbar_init(&sm.empty_k[s], 128 + 128 * kSub); }
-        for (int s = 0; s < kAStages; ++s) { tc::mbar_init(&sm.a_full[s], 128); tc::mbar_init(&sm.a_empty[s], 1); }
+        // A key stage is free once the MMAs reading it have completed (one commit) and the
+        // epilogue has read its scales (128 arrivals).
+        for (int s = 0; s < KS; ++s) { tc::mbar_init(&sm.full_k[s], 1); tc::mbar_init(&sm.empty_k[s], 129); }
         for (int s = 0; s < kSlots; ++s) { tc::mbar_init(&sm.d_full[s], 1); tc::mbar_init(&sm.d_empty[s], 128); }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&sm.q_full[b], 128);
@@ -181,7 +300,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
             else if (blockIdx.x == 0) report(a.status, LSA_ERR_DEVICE_DATA);
         }
         const int cols = hi ? a.n_cols : min(a.n_cols, max_pos + 1);
-        sm.tstart[gl] = (max_pos < 0 || cols <= 0) ? 0 : (cols + kTile - 1) / kTile;
+        sm.tstart[gl] = (max_pos < 0 || cols <= 0) ? 0 : (cols + TK - 1) / TK;
     }
     __syncthreads();
     cta_exclusive_scan(sm.tstart, NG, s_tmp);
@@ -192,37 +311,32 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    const uint32_t tmem = sm.tmem_base;
-    const uint32_t a_col = tmem, d_col = tmem + kAStages * 64;
+    const uint32_t d_col = sm.tmem_base;
 
     if (warp == 0) {
         // ---------------- TMA producer
         if (tc::elect_one()) {
-            TileCursor cur{sm.tstart, NG};
-            int issued = 0;
-            for (int j = 0; j < n_mine; ++j) {
-                cur.seek(k_lo + j);
-                const int s = j % KS;
-                if (!tc::mbar_wait(&sm.empty_k[s], ((j / KS) + 1) & 1, abort_flag)) break;
+            Walk wk(sm.tstart, NG, k_lo);
+            int t0 = (pa.group0 + wk.g) * G, bseq = max(a.q_seq[t0], 0);
+            int s = 0, ph = 0, issued = 0;
+            for (int k = k_lo; k < k_hi; ++k) {
+                if (wk.to(k)) { t0 = (pa.group0 + wk.g) * G; bseq = max(a.q_seq[t0], 0); }
+                if (!tc::mbar_wait(&sm.empty_k[s], ph ^ 1, abort_flag)) break;
                 ++issued;
-                const int t0 = (pa.group0 + cur.g) * G;
-                const int bseq = max(a.q_seq[t0], 0);
-                tc::mbar_expect_tx(&sm.full_k[s], kKeyTileBytes + (pa.scale_tma ? kTile * 4 : 0));
-                const int c = cur.lt * kTile;
-                int r0 = c, r1 = c + 64;
-                if (hi) {
-                    const int nb = a.n_cand;
-                    const int bk0 = (c / 64) < nb ? a.cand[(size_t)t0 * nb + c / 64] : -1;
-                    const int bk1 = (c / 64 + 1) < nb ? a.cand[(size_t)t0 * nb + c / 64 + 1] : -1;
-                    r0 = bk0 >= 0 ? bk0 * 64 : 0;
-                    r1 = bk1 >= 0 ? bk1 * 64 : 0;
+                tc::mbar_expect_tx(&sm.full_k[s], NB * kBlockBytes + (pa.scale_tma ? TK * 4 : 0));
+                const int c = (k - sm.tstart[wk.g]) * TK;
+#pragma unroll
+                for (int i = 0; i < 2 * NB; ++i) {               // 64-row boxes
+                    int r0 = c + 64 * i;
+                    if (hi) {
+                        const int bi = c / 64 + i;
+                        const int bk = bi < a.n_cand ? a.cand[(size_t)t0 * a.n_cand + bi] : -1;
+                        r0 = bk >= 0 ? bk * 64 : 0;
+                    }
+                    tc::tma_load_3d(sm.keys[s] + i * (kBlockBytes / 2), &tmap, &sm.full_k[s], 0, r0, bseq);
+                    if (pa.scale_tma) tc::tma_load_2d(sm.scl[s] + 64 * i, &smap, &sm.full_k[s], r0, bseq);
                 }
-                tc::tma_load_3d(sm.keys[s], &tmap, &sm.full_k[s], 0, r0, bseq);
-                tc::tma_load_3d(sm.keys[s] + kKeyTileBytes / 2, &tmap, &sm.full_k[s], 0, r1, bseq);
-                if (pa.scale_tma) {
-                    tc::tma_load_2d(sm.scl[s], &smap, &sm.full_k[s], r0, bseq);
-                    tc::tma_load_2d(sm.scl[s] + 64, &smap, &sm.full_k[s], r1, bseq);
-                }
+                if (++s == KS) { s = 0; ph ^= 1; }
             }
             // Drain: every issued tile has landed before the CTA can exit (bounded; already true
             // unless the consumers gave up early).
@@ -231,239 +345,163 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                 tc::mbar_wait(&sm.full_k[j % KS], (j / KS) & 1, &drain_abort);
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
-        const uint32_t idesc = tc::idesc_f16(128, NS, 0);
+        // ---------------- MMA issuer: a lean loop (descriptors precomputed; K chunk kk of a
+        // 128-byte swizzled row starts kk * 32 bytes in, i.e. 2 * kk in the descriptor's address
+        // field, which cannot carry since shared addresses are below 256 KB)
+        const uint32_t idesc = tc::idesc_f16(128, N, 0);      // e4m3 x e4m3 -> f32, both K-major
         if (tc::elect_one()) {
-            TileCursor cur{sm.tstart, NG};
-            int last_slot = -1, last_ph = 0;
-            for (int j = 0; j < n_mine; ++j) {
-                const int prev_epoch = cur.epoch;
-                cur.seek(k_lo + j);
-                const int qb = cur.epoch & 1;
-                if (cur.epoch != prev_epoch &&
-                    !tc::mbar_wait(&sm.q_full[qb], (cur.epoch >> 1) & 1, abort_flag)) break;
-                const int ab = j % kAStages;
-                if (!tc::mbar_wait(&sm.a_full[ab], (j / kAStages) & 1, abort_flag)) break;
-                const uint32_t q0 = tc::smem_u32(sm.q[qb][0]), q1 = tc::smem_u32(sm.q[qb][1]);
-                bool ok = true;
+            const uint64_t da0 = tc::sdesc_sw128(tc::smem_u32(sm.keys[0]));
+            const uint64_t dh0 = tc::sdesc_sw128(tc::smem_u32(sm.q[0][0])), dl0 = tc::sdesc_sw128(tc::smem_u32(sm.q[0][1]));
+            const uint64_t dh1 = tc::sdesc_sw128(tc::smem_u32(sm.q[1][0])), dl1 = tc::sdesc_sw128(tc::smem_u32(sm.q[1][1]));
+            Walk wk(sm.tstart, NG, k_lo);
+            int s = 0, kph = 0, slot = 0, dph = 0, last_slot = -1, last_ph = 0;
+            bool alive = n_mine == 0 || tc::mbar_wait(&sm.q_full[0], 0, abort_flag);
+            for (int k = k_lo; alive && k < k_hi; ++k) {
+                if (wk.to(k) && !tc::mbar_wait(&sm.q_full[wk.epoch & 1], (wk.epoch >> 1) & 1, abort_flag)) break;
+                if (!tc::mbar_wait(&sm.full_k[s], kph, abort_flag)) break;
+                if (!tc::mbar_wait(&sm.d_empty[slot], dph ^ 1, abort_flag)) break;
+                tc::tc_fence_after();
+                const uint64_t dh = (wk.epoch & 1) ? dh1 : dh0, dl = (wk.epoch & 1) ? dl1 : dl0;
 #pragma unroll
-                for (int h = 0; h < kSub; ++h) {
-                    const int slot = kSub == 2 ? h : j % kSlots, ph = kSub == 2 ? j : j / kSlots;
-                    if (!tc::mbar_wait(&sm.d_empty[slot], (ph + 1) & 1, abort_flag)) { ok = false; break; }
-                    tc::tc_fence_after();
+                for (int b = 0; b < NB; ++b) {                   // block b: keys b*128 .. b*128+127
+                    const uint64_t da = da0 + (uint64_t)((s * NB + b) * (kBlockBytes >> 4));
+                    const uint32_t dc = d_col + slot * SW + b * N;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t qa = (k < 4 ? q0 : q1) + (k & 3) * 32 + h * NS * 128;
-                        tc::mma_f16_ts(d_col + slot * NS, a_col + ab * 64 + k * 8, tc::sdesc_sw128(qa), idesc, k > 0);
-                    }
-                    tc::mma_commit(&sm.d_full[slot]);
-                    last_slot = slot;
-                    last_ph = ph;
+                    for (int k8 = 0; k8 < 8; ++k8)
+                        tc::mma_f8_ss(dc, da + 2 * (k8 & 3), (k8 < 4 ? dh : dl) + 2 * (k8 & 3), idesc, k8 > 0);
                 }
-                if (!ok) break;
-                tc::mma_commit(&sm.a_empty[ab]);
+                tc::mma_commit(&sm.empty_k[s]);
+                tc::mma_commit(&sm.d_full[slot]);
+                last_slot = slot;
+                last_ph = dph;
+                if (++s == KS) { s = 0; kph ^= 1; }
+                if (++slot == kSlots) { slot = 0; dph ^= 1; }
             }
             if (last_slot >= 0) {                     // drain: issued MMAs complete before TMEM is freed
                 volatile int drain_abort = 0;
-                tc::mbar_wait(&sm.d_full[last_slot], last_ph & 1, &drain_abort);
+                tc::mbar_wait(&sm.d_full[last_slot], last_ph, &drain_abort);
             }
         }
     } else if (warp < 6) {
-        // ---------------- converters (thread = TMEM lane = key row) and query preparation
-        const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;
+        // ---------------- query preparation, once per group epoch
         const int ct = threadIdx.x - 64;                                // 0..127
-        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        TileCursor cur{sm.tstart, NG};
-        for (int j = 0; j < n_mine; ++j) {
-            const int prev_epoch = cur.epoch;
-            cur.seek(k_lo + j);
-            if (cur.epoch != prev_epoch) {
-                // New group: its queries go to buffer e & 1 once both epilogue warpgroups have
-                // released the group that used the buffer before (epoch e - 2).
-                const int e = cur.epoch, qb = e & 1;
-                if (e >= 2 && (!tc::mbar_wait(&sm.q_free[qb][0], ((e - 2) >> 1) & 1, abort_flag) ||
-                               !tc::mbar_wait(&sm.q_free[qb][1], ((e - 2) >> 1) & 1, abort_flag)))
-                    break;
-                const int t0 = (pa.group0 + cur.g) * G;
-                if (ct < kMaxG) {
-                    int okv = 0, p = -1;
-                    if (ct < G) {
-                        const int b0 = a.q_seq[t0], s = a.q_seq[t0 + ct];
-                        p = a.q_pos[t0 + ct];
-                        okv = s == b0 && s >= 0 && s < a.B;
-                        if (okv) {
-                            const int len = a.seq_len[s];
-                            okv = len >= 1 && len <= a.L_alloc && p >= 0 && p < len;
-                        }
-                    }
-                    sm.pos[qb][ct] = okv ? p : -1;
-                    sm.ok[qb][ct] = okv;
-                }
-                // Thread ct handles 16-byte chunks ct, ct + 128, ... of the N rows (16 chunks per
-                // row, in 16 consecutive lanes that reduce the row maximum by shuffles).
-                constexpr int kQB = 4;
-                for (int base = ct; base < N * 16; base += 128 * kQB) {
-                    uint4 raw[kQB];
-#pragma unroll
-                    for (int u = 0; u < kQB; ++u) {
-                        const int i = base + u * 128;
-                        const int rowi = i >> 4;
-                        raw[u] = i < N * 16 ? *reinterpret_cast<const uint4*>(
-                                                  a.q + ((size_t)(t0 + rowi / H_I) * H_I + rowi % H_I) * 128 + (i & 15) * 8)
-                                            : make_uint4(0, 0, 0, 0);
-                    }
-#pragma unroll
-                    for (int u = 0; u < kQB; ++u) {
-                        const int i = base + u * 128;
-                        if (i >= N * 16) break;                  // warp-uniform: N * 16 is a multiple of 128
-                        const int rowi = i >> 4, cc = i & 15;
-                        const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw[u]);
-                        float v[8];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            v[2 * e2] = bf16_bits_to_float((uint16_t)(wd[e2] & 0xffff));
-                            v[2 * e2 + 1] = bf16_bits_to_float((uint16_t)(wd[e2] >> 16));
-                        }
-                        float m = 0.f;
-#pragma unroll
-                        for (int e2 = 0; e2 < 8; ++e2) m = fmaxf(m, fabsf(v[e2]));
-#pragma unroll
-                        for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                        const int ex = (int)((__float_as_uint(m) >> 23) & 0xff) - 127;
-                        int k = m > 0.f ? 14 - ex : 0;
-                        k = max(-126, min(126, k));
-                        const float sc = exp2i(k);
-                        uint32_t hv[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2)
-                            hv[e2] = (uint32_t)__half_as_ushort(__float2half_rn(v[2 * e2] * sc)) |
-                                     ((uint32_t)__half_as_ushort(__float2half_rn(v[2 * e2 + 1] * sc)) << 16);
-                        const int atom = cc >> 3, c16 = cc & 7;
-                        uint8_t* dst = sm.q[qb][atom] + (rowi >> 3) * 1024 + (rowi & 7) * 128 + ((c16 ^ (rowi & 7)) << 4);
-                        *reinterpret_cast<uint4*>(dst) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                        if (cc == 0) sm.w[qb][rowi] = a.w[(size_t)(t0 + rowi / H_I) * H_I + rowi % H_I] * exp2i(-k);
+        Walk wk(sm.tstart, NG, k_lo);
+        for (int k = k_lo; k < k_hi; k = sm.tstart[wk.g + 1]) {
+            wk.to(k);
+            // Group epoch e: its queries go to buffer e & 1 once both epilogue warpgroups have
+            // released the group that used the buffer before (epoch e - 2).
+            const int e = wk.epoch, qb = e & 1;
+            if (e >= 2 && (!tc::mbar_wait(&sm.q_free[qb][0], ((e - 2) >> 1) & 1, abort_flag) ||
+                           !tc::mbar_wait(&sm.q_free[qb][1], ((e - 2) >> 1) & 1, abort_flag)))
+                break;
+            const int t0 = (pa.group0 + wk.g) * G;
+            if (ct < kMaxG) {
+                int okv = 0, p = -1;
+                if (ct < G) {
+                    const int b0 = a.q_seq[t0], sq = a.q_seq[t0 + ct];
+                    p = a.q_pos[t0 + ct];
+                    okv = sq == b0 && sq >= 0 && sq < a.B;
+                    if (okv) {
+                        const int len = a.seq_len[sq];
+                        okv = len >= 1 && len <= a.L_alloc && p >= 0 && p < len;
                     }
                 }
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(&sm.q_full[qb]);
+                sm.pos[qb][ct] = okv ? p : -1;
+                sm.ok[qb][ct] = okv;
             }
-            const int s = j % KS, ab = j % kAStages;
-            if (!tc::mbar_wait(&sm.full_k[s], (j / KS) & 1, abort_flag)) break;
-            const uint8_t* rowp = sm.keys[s] + r * 128;          // 128-byte rows, 16-byte chunks XOR-swizzled
-            uint4 ch[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) ch[c] = *reinterpret_cast<const uint4*>(rowp + ((c ^ (r & 7)) << 4));
-            tc::mbar_arrive(&sm.empty_k[s]);
-            if (!tc::mbar_wait(&sm.a_empty[ab], ((j / kAStages) + 1) & 1, abort_flag)) break;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t wv[32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t* wd = reinterpret_cast<const uint32_t*>(&ch[half * 4 + c]);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        wv[c * 8 + 2 * u] = e4m3x2_to_f16x2((uint16_t)(wd[u] & 0xffff));
-                        wv[c * 8 + 2 * u + 1] = e4m3x2_to_f16x2((uint16_t)(wd[u] >> 16));
-                    }
-                }
-                tc::tmem_st32(a_col + ab * 64 + half * 32 + lane_off, wv);
-            }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
-            tc::mbar_arrive(&sm.a_full[ab]);
+            prepare_queries<N>(a, t0, H_I, ct, sm.q[qb][0], sm.q[qb][1], sm.w[qb]);
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&sm.q_full[qb]);
         }
     } else {
-        // ---------------- epilogue warpgroups: N <= 128, warpgroup wg takes the tiles j with
-        // j % 2 == wg; N = 256, it takes half wg of every tile
+        // ---------------- epilogue warpgroups: warpgroup wg takes the tiles j with j % 2 == wg
         const int wg = (warp - 6) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const bool fp8 = a.kscale != nullptr;
-        const int tps = NS / H_I;                            // query tokens per accumulator slot
-        TileCursor cur{sm.tstart, NG};
+        Walk wk(sm.tstart, NG, k_lo);
+        int t0 = (pa.group0 + wk.g) * G;
         int released = -1, waited = -1;                      // last epoch released / whose queries are known ready
-        for (int j = 0; j < n_mine; ++j) {
-            cur.seek(k_lo + j);
-            const int e = cur.epoch, qb = e & 1;
+        int s = 0, kph = 0, slot = 0, dph = 0;
+        for (int k = k_lo, j = 0; k < k_hi; ++k, ++j) {
+            if (wk.to(k)) t0 = (pa.group0 + wk.g) * G;
+            const int e = wk.epoch, qb = e & 1;
             // Every tile of this warpgroup before j is done: release the earlier groups' buffers.
             for (; released < e - 1; ++released) tc::mbar_arrive(&sm.q_free[(released + 1) & 1][wg]);
-            if (kSub == 1 && (j & 1) != wg) continue;
-            if (e != waited) {
-                if (!tc::mbar_wait(&sm.q_full[qb], (e >> 1) & 1, abort_flag)) break;
-                waited = e;
-            }
-            const int s = j % KS;
-            const int t0 = (pa.group0 + cur.g) * G;
-            const int col = cur.lt * kTile + r;
-            int row = col;
-            if (hi) {
-                const int bi = col / 64;
-                const int blk = (col < a.n_cols && bi < a.n_cand) ? a.cand[(size_t)t0 * a.n_cand + bi] : -1;
-                row = blk >= 0 ? blk * 64 + (col & 63) : -1;
-            }
-            if (!tc::mbar_wait(&sm.full_k[s], (j / KS) & 1, abort_flag)) break;
-            float ks = 1.f;
-            if (fp8) {
-                if (pa.scale_tma) ks = sm.scl[s][r];
-                else if (row >= 0 && row < a.L_alloc) ks = a.kscale[(size_t)max(a.q_seq[t0], 0) * a.scale_seq_stride + row];
-            }
-            tc::mbar_arrive(&sm.empty_k[s]);
-            {
-                const int h = kSub == 2 ? wg : 0;
-                const int slot = kSub == 2 ? wg : j % kSlots, ph = kSub == 2 ? j : j / kSlots;
-                if (!tc::mbar_wait(&sm.d_full[slot], ph & 1, abort_flag)) break;
-                tc::tc_fence_after();
-                for (int ti = 0; ti < tps; ++ti) {
-                    const int gi = h * tps + ti;
-                    // Four partial sums (head h goes to sum h % 4), two per packed FMA.
-                    float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
-                    for (int h0 = 0; h0 < H_I; h0 += 32) {
-                        uint32_t v[32];
-                        tc::tmem_ld32(d_col + slot * NS + ti * H_I + h0 + lane_off, v);
-                        tc::tmem_wait_ld();
-                        const float4* wp = reinterpret_cast<const float4*>(sm.w[qb] + gi * H_I + h0);
+            if ((j & 1) == wg) {
+                if (e != waited) {
+                    if (!tc::mbar_wait(&sm.q_full[qb], (e >> 1) & 1, abort_flag)) break;
+                    waited = e;
+                }
+                int col[NB], row[NB];
+                float ks[NB];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 ww = wp[i];
-                            acc01 = ffma2(make_float2(ww.x, ww.y),
-                                          make_float2(fmaxf(__uint_as_float(v[4 * i + 0]), 0.f),
-                                                      fmaxf(__uint_as_float(v[4 * i + 1]), 0.f)), acc01);
-                            acc23 = ffma2(make_float2(ww.z, ww.w),
-                                          make_float2(fmaxf(__uint_as_float(v[4 * i + 2]), 0.f),
-                                                      fmaxf(__uint_as_float(v[4 * i + 3]), 0.f)), acc23);
-                        }
+                for (int b = 0; b < NB; ++b) {
+                    col[b] = (k - sm.tstart[wk.g]) * TK + b * kBlock + r;
+                    row[b] = col[b];
+                    if (hi) {
+                        const int bi = col[b] / 64;
+                        const int blk = (col[b] < a.n_cols && bi < a.n_cand) ? a.cand[(size_t)t0 * a.n_cand + bi] : -1;
+                        row[b] = blk >= 0 ? blk * 64 + (col[b] & 63) : -1;
                     }
-                    const float tot = (acc01.x + acc01.y) + (acc23.x + acc23.y);
-                    if (col < a.n_cols) {
-                        const bool vis = sm.ok[qb][gi] && row >= 0 && row <= sm.pos[qb][gi];
-                        a.scores[(size_t)(t0 + gi) * a.ld + col] = vis ? tot * ks : kNegInf;
+                }
+                if (!tc::mbar_wait(&sm.full_k[s], kph, abort_flag)) break;
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    ks[b] = 1.f;
+                    if (fp8) {
+                        if (pa.scale_tma) ks[b] = sm.scl[s][b * kBlock + r];
+                        else if (row[b] >= 0 && row[b] < a.L_alloc)
+                            ks[b] = a.kscale[(size_t)max(a.q_seq[t0], 0) * a.scale_seq_stride + row[b]];
                     }
+                }
+                tc::mbar_arrive(&sm.empty_k[s]);
+                if (!tc::mbar_wait(&sm.d_full[slot], dph, abort_flag)) break;
+                tc::tc_fence_after();
+                const uint32_t tb = d_col + slot * SW + lane_off;
+                const auto store = [&](int gi, int b, float tot) {
+                    if (col[b] < a.n_cols) {
+                        const bool vis = sm.ok[qb][gi] && row[b] >= 0 && row[b] <= sm.pos[qb][gi];
+                        a.scores[(size_t)(t0 + gi) * a.ld + col[b]] = vis ? tot * ks[b] : kNegInf;
+                    }
+                };
+                // Items (block, token), two at a time: both blocks of one token when NB = 2 (same
+                // weights), else two tokens of the one block.
+                const int n_items = NB * G;
+                for (int it = 0; it < n_items; it += 2) {
+                    constexpr int ba = 0, bb = NB == 2 ? 1 : 0;
+                    const int ga = NB == 2 ? it / 2 : it, gb = NB == 2 ? it / 2 : it + 1;
+                    const bool two = it + 1 < n_items;
+                    float ta, tv;
+                    head_sums2(tb + ba * N + ga * H_I, tb + bb * N + gb * H_I, sm.w[qb] + ga * H_I, sm.w[qb] + gb * H_I,
+                               H_I, two, ta, tv);
+                    store(ga, ba, ta);
+                    if (two) store(gb, bb, tv);
                 }
                 tc::tc_fence_before();
                 tc::mbar_arrive(&sm.d_empty[slot]);
             }
+            if (++s == KS) { s = 0; kph ^= 1; }
+            if (++slot == kSlots) { slot = 0; dph ^= 1; }
         }
         // Columns past a group's active tiles (all columns of a group with no visible key) are
         // -inf; CTA b fills the groups g with g % grid == b.
         const int et = threadIdx.x - 192;                           // 0..255
         for (int gl = blockIdx.x; gl < NG; gl += gridDim.x) {
-            const int t0 = (pa.group0 + gl) * G;
-            const int from = (sm.tstart[gl + 1] - sm.tstart[gl]) * kTile;
+            const int tg = (pa.group0 + gl) * G;
+            const int from = (sm.tstart[gl + 1] - sm.tstart[gl]) * TK;
             for (int gi = 0; gi < G; ++gi)
                 for (int col = from + et; col < a.n_cols; col += 256)
-                    a.scores[(size_t)(t0 + gi) * a.ld + col] = kNegInf;
+                    a.scores[(size_t)(tg + gi) * a.ld + col] = kNegInf;
         }
     }
-
     tc::tc_fence_before();
     __syncthreads();
     if (sm.abort && threadIdx.x == 0) report(a.status, LSA_ERR_TIMEOUT);
     if (warp == 0) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, 512);
+        tc::tmem_dealloc(sm.tmem_base, 512);
     }
 }
 
@@ -491,10 +529,10 @@ int num_sms() {
     return n;
 }
 
-template <int N, int KS>
+template <int N, int NB, int KS>
 cudaError_t launch_n(const CUtensorMap& m, const CUtensorMap& sm, const PArgs& pa, cudaStream_t st) {
-    const size_t smem = sizeof(PSmem<N, KS>) + 1024;
-    auto kern = index_score_tc_kernel<N, KS>;
+    const size_t smem = sizeof(PSmem<N, NB, KS>) + 1024;
+    auto kern = index_score_tc_kernel<N, NB, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<num_sms(), kPThreads, smem, st>>>(m, sm, pa);
@@ -558,10 +596,10 @@ cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st) {
         pa.n_groups = std::min(kMaxGroups, total_groups - g0);
         cudaError_t e;
         switch (N) {
-            case 32: e = launch_n<32, 8>(m, sc, pa, st); break;
-            case 64: e = launch_n<64, 8>(m, sc, pa, st); break;
-            case 128: e = launch_n<128, 8>(m, sc, pa, st); break;
-            case 256: e = launch_n<256, 4>(m, sc, pa, st); break;
+            case 32: e = launch_n<32, 2, 5>(m, sc, pa, st); break;
+            case 64: e = launch_n<64, 2, 5>(m, sc, pa, st); break;
+            case 128: e = launch_n<128, 2, 4>(m, sc, pa, st); break;
+            case 256: e = launch_n<256, 1, 4>(m, sc, pa, st); break;
             default: return cudaErrorInvalidValue;
         }
         if (e != cudaSuccess) return e;
