@@ -15,14 +15,15 @@
 // 16 K-steps, and a 4-stage ring of 32-row KV tiles (36 KB each) in the 128-byte-swizzled
 // K-major layout, read as the B operand of S (K-major) and of P V (MN-major).
 //
-//   warps 0..3 : gather -- warp g fills stage g with the tiles j = g, g+4, ...: the tile's 32
-//                row indices (prefetched one tile ahead) go to shared memory, then the rows
-//                are copied with 16-byte cp.async (FP8 rows are widened to BF16 exactly on the
-//                way); per-row scale and validity.
-//   warp 8     : MMA issuer -- issues whatever is ready, in order per kind: S_j (16 SS + 20 TS
+//   warps 0..7 : gather -- warps 2s and 2s+1 fill stage s with the tiles j = s, s+4, ..., 16
+//                rows each: the rows' indices (prefetched one tile ahead) go to shared memory,
+//                then the rows are copied with 16-byte cp.async (FP8 rows are widened to BF16
+//                exactly on the way); per-row scale and validity.  Two warps per tile keep
+//                twice the copies in flight that one warp would.
+//   warp 12    : MMA issuer -- issues whatever is ready, in order per kind: S_j (16 SS + 20 TS
 //                MMAs, N = 32) once tile j has landed and P V_{j-2} has been issued, and
 //                O += P_j V_j (2 TS MMAs, N = 256) once the softmax of tile j is done.
-//   warps 4..7 : softmax -- thread = head (TMEM lane): online max / sum with lazy rescaling
+//   warps 8..11: softmax -- thread = head (TMEM lane): online max / sum with lazy rescaling
 //                of O (only when the running max grows by more than 2^8; warp-uniform, so
 //                deterministic), P to TMEM as BF16; finally O / l and lse.
 //
@@ -34,7 +35,7 @@ namespace lsa {
 
 namespace {
 
-constexpr int kAThreads = 288;
+constexpr int kAThreads = 416;
 constexpr int kRows = 32;                    // KV rows per tile
 constexpr int kStagesA = 4;                  // KV tile ring
 constexpr int kD = 576, kDv = 512, kHalf = 256;
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
     const uint16_t* qt = a.q + (size_t)t * 128 * kD;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStagesA; ++i) { tc::mbar_init(&sm.kv_full[i], 32); tc::mbar_init(&sm.kv_empty[i], 1); }
+        for (int i = 0; i < kStagesA; ++i) { tc::mbar_init(&sm.kv_full[i], 64); tc::mbar_init(&sm.kv_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.s_full[i], 1);
             tc::mbar_init(&sm.p_full[i], 128);
@@ -103,8 +104,8 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
     const uint32_t o_col = tmem, s_col = tmem + 256, p_col = tmem + 320, qt_col = tmem + 352;
     // The softmax warps load Q while the gather warps already fetch KV tiles: dims 0..255 into
     // shared memory (K-major, 128-byte swizzle), dims 256..575 into TMEM (thread = head = lane).
-    if (warp >= 4 && warp < 8) {
-        const int tq = threadIdx.x - 128;
+    if (warp >= 8 && warp < 12) {
+        const int tq = threadIdx.x - 256;
         for (int i = tq; i < 128 * (kQSmemAtoms * 8); i += 128) {
             const int h = i / (kQSmemAtoms * 8), c = i % (kQSmemAtoms * 8);
             uint8_t* dst = sm.q + (c >> 3) * (128 * 128) + h * 128 + (((c & 7) ^ (h & 7)) << 4);
@@ -131,34 +132,35 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
         tc::mbar_arrive(&sm.q_ready);
     }
 
-    if (warp < 4) {
-        // ---------------- gather producers: warp g owns stage g and the tiles j = g, g + 4, ...
-        const int g = warp;
+    if (warp < 8) {
+        // ---------------- gather producers: warps 2s, 2s + 1 own stage s (rows 0..15 / 16..31
+        // of the tiles j = s, s + 4, ...)
+        const int g = warp >> 1, rh = (warp & 1) * (kRows / 2);
         auto fetch_row = [&](int j) -> int {
             if (j >= n_tiles) return -1;
-            const int r0 = r_beg + j * kRows;
-            return lane < min(kRows, r_end - r0) ? irow[r0 + lane] : -1;
+            const int r0 = r_beg + j * kRows + rh;
+            return lane < min(kRows / 2, r_end - r0) ? irow[r0 + lane] : -1;
         };
         int nxt = fetch_row(g);
         for (int j = g; j < n_tiles; j += kStagesA) {
             const int cur = nxt;
             nxt = fetch_row(j + kStagesA);                         // prefetch this warp's next tile
             if (!tc::mbar_wait(&sm.kv_empty[g], ((j / kStagesA) + 1) & 1, abort_flag)) break;
-            const int nr = min(kRows, r_end - (r_beg + j * kRows));
-            {
+            const int nr = min(kRows / 2, r_end - (r_beg + j * kRows + rh));
+            if (lane < kRows / 2) {
                 const bool v = cur >= 0 && cur < len;
                 if (lane < nr && !v) report(a.status, LSA_ERR_DEVICE_DATA);
                 const float vs = KV_FP8 ? (v ? kvs[cur] : 0.f) : 1.f;
-                sm.rows[g][lane] = v ? cur : -1;
-                sm.vscale[g][lane] = vs;
-                sm.kscale[g][lane] = v ? vs * a.sm_scale_log2 : 0.f;
+                sm.rows[g][rh + lane] = v ? cur : -1;
+                sm.vscale[g][rh + lane] = vs;
+                sm.kscale[g][rh + lane] = v ? vs * a.sm_scale_log2 : 0.f;
             }
             __syncwarp();
             uint8_t* tile = sm.kv[g];
             if (!KV_FP8) {
 #pragma unroll 4
-                for (int i = lane; i < kRows * (kD / 8); i += 32) {
-                    const int r = i / (kD / 8), c = i % (kD / 8);
+                for (int i = lane; i < (kRows / 2) * (kD / 8); i += 32) {
+                    const int r = rh + i / (kD / 8), c = i % (kD / 8);
                     const int row = sm.rows[g][r];
                     uint8_t* dst = tile + (c >> 3) * (kRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
                     cp_async16(dst, kvb + (size_t)(row >= 0 ? row : 0) * a.kv_tok_b + c * 16, row >= 0);
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                 cp_async_commit();
                 cp_async_wait<0>();
             } else {
-                constexpr int kChunks = kRows * (kD / 16);             // 16 codes per chunk
+                constexpr int kChunks = (kRows / 2) * (kD / 16);       // 16 codes per chunk
                 constexpr int kBatch = 12;
                 for (int i0 = lane; i0 < kChunks; i0 += 32 * kBatch) {
                     uint4 raw[kBatch];
@@ -175,7 +177,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                         const int i = i0 + u * 32;
                         raw[u] = make_uint4(0, 0, 0, 0);
                         if (i < kChunks) {
-                            const int row = sm.rows[g][i / (kD / 16)];
+                            const int row = sm.rows[g][rh + i / (kD / 16)];
                             if (row >= 0) raw[u] = ldg_nc16(kvb + (size_t)row * a.kv_tok_b + (i % (kD / 16)) * 16);
                         }
                     }
@@ -183,7 +185,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                     for (int u = 0; u < kBatch; ++u) {
                         const int i = i0 + u * 32;
                         if (i >= kChunks) break;
-                        const int r = i / (kD / 16), c = i % (kD / 16);
+                        const int r = rh + i / (kD / 16), c = i % (kD / 16);
                         const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw[u]);
                         uint32_t ow[8];
 #pragma unroll
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(&sm.kv_full[g]);
         }
-    } else if (warp == 8) {
+    } else if (warp == 12) {
         // ---------------- MMA issuer: S_j and P_j V_j, each in order, whichever is ready
         const uint32_t idesc_s = tc::idesc_f16(128, kRows, 1);
         const uint32_t idesc_o = tc::idesc_f16_bmn(128, kHalf, 1);
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                 tc::mbar_wait(&sm.o_done[(npv - 1) & 1], ((npv - 1) >> 1) & 1, &drain_abort);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 8 && warp < 12) {
         // ---------------- softmax / epilogue: thread = head = TMEM lane
         const int quarter = warp & 3;
         const int h = quarter * 32 + lane;
