@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
     // shared memory (K-major, 128-byte swizzle), dims 256..575 into TMEM (thread = head = lane).
     if (warp >= 8 && warp < 12) {
         const int tq = threadIdx.x - 256;
+        prefetch_l2_bulk(qt + (size_t)tq * kD, kD * 2);              // head tq's row into L2
         for (int i = tq; i < 128 * (kQSmemAtoms * 8); i += 128) {
             const int h = i / (kQSmemAtoms * 8), c = i % (kQSmemAtoms * 8);
             uint8_t* dst = sm.q + (c >> 3) * (128 * 128) + h * 128 + (((c & 7) ^ (h & 7)) << 4);
@@ -115,15 +116,25 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
         const int h = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint4* src = reinterpret_cast<const uint4*>(qt + (size_t)h * kD + kQSmemAtoms * 64);
+        // Software-pipelined: the loads of 32-column group c + 1 are in flight while group c is
+        // stored to TMEM.
+        uint4 cur[8], nxt[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cur[u] = src[u];
 #pragma unroll 1
         for (int c = 0; c < kQTmemCols / 32; ++c) {
+            if (c + 1 < kQTmemCols / 32) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) nxt[u] = src[(c + 1) * 8 + u];
+            }
             uint32_t v[32];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const uint4 x = src[c * 8 + u];
-                v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+                v[4 * u] = cur[u].x; v[4 * u + 1] = cur[u].y; v[4 * u + 2] = cur[u].z; v[4 * u + 3] = cur[u].w;
             }
             tc::tmem_st32(qt_col + c * 32 + lane_off, v);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) cur[u] = nxt[u];
         }
         tc::tmem_wait_st();
         cp_async_wait<0>();
