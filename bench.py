@@ -316,7 +316,8 @@ def run_gpu(args, rank, world, local_rank):
         "algorithmic_gb_per_step": total_bytes / 1e9,
         "step_hbm_gbs": total_bytes / (ms / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "peak_source": f"{src} hbm_gbs",
+                     "frac": achieved / hbm, "traffic": indexer_traffic(kern, idx_bytes),
+                     "peak_source": f"{src} hbm_gbs",
                      "launch_ms": kms, "algorithmic_bytes_per_launch": idx_bytes},
         "e2e": {"value": q_per_step * world / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -324,6 +325,28 @@ def run_gpu(args, rank, world, local_rank):
         "clocks": clk.summary(),
     }
     return res, w, wt
+
+
+def indexer_traffic(kern: str, idx_bytes: float):
+    """DRAM bytes per launch of the flat tensor-core indexer, from the committed ncu capture.
+
+    The capture's summary (profiles/kernels_decode_cli_128k_batch8.md) records the ratio of
+    measured DRAM traffic to algorithmic bytes on a small case and the SHA-256 of the kernel
+    source it was taken on; the ratio is applied only while the source still has that hash
+    (otherwise the counters describe another kernel and the field is null)."""
+    import hashlib
+    import re
+    if not kern.startswith("index_score"):
+        return None
+    try:
+        txt = open(os.path.join(ROOT, "profiles", "kernels_decode_cli_128k_batch8.md")).read()
+        m = re.search(r"indexer_traffic_ratio=([0-9.]+) source_sha256=([0-9a-f]{64})", txt)
+        src = open(os.path.join(ROOT, "long_context_sparse_indexer_b200", "csrc", "index_score_tc.cu"), "rb").read()
+    except OSError:
+        return None
+    if not m or hashlib.sha256(src).hexdigest() != m.group(2):
+        return None
+    return float(m.group(1)) * idx_bytes
 
 
 # ------------------------------------------------------------------ the CPU oracle (baseline / reference arm)
