@@ -44,6 +44,25 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def bf16_peak():
+    """Dense BF16 tensor throughput for a kernel timed alone (the burst figure)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def indexer_flops(w, p):
+    """Algorithmic flops of one flat indexer pass: 2 * H_I * d_I per (query, visible key)."""
+    _, q_pos = W.query_rows(w, p)
+    return float(2 * w.H_I * w.d_I) * float(np.sum(q_pos.astype(np.int64) + 1))
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -271,6 +290,20 @@ def run_gpu(args, rank, world, local_rank):
     kms = time_region(idx_fn, max(10, args.steps), stream)
     hbm, src = peaks()
     achieved = idx_bytes / (kms / 1e3) / 1e9
+    roof = {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": indexer_traffic(kern, idx_bytes), "peak_source": f"{src} hbm_gbs",
+            "launch_ms": kms, "algorithmic_bytes_per_launch": idx_bytes}
+    if not w.hi:
+        # The flat indexer issues FP8 MMAs (e4m3 x e4m3, two query terms): peak = measured BF16
+        # burst x 2 (the nominal FP8 / BF16 ratio).  Tensor-bound when its flops at that peak take
+        # longer than its bytes at the HBM peak (prefill; not decode).
+        flops = indexer_flops(w, w.passes[0])
+        bf16, bsrc = bf16_peak()
+        fp8 = 2.0 * bf16
+        if flops / (fp8 * 1e12) > idx_bytes / (hbm * 1e9):
+            tf = flops / (kms / 1e3) / 1e12
+            roof.update({"bound": "tensor", "achieved": tf, "peak": fp8, "unit": "TFLOP/s", "frac": tf / fp8,
+                         "peak_source": f"{bsrc} bf16_tflops x 2 (FP8 MMA)", "algorithmic_flops_per_launch": flops})
 
     # End to end through the public API: H2D of the step's queries from pinned host memory, the
     # fused calls, D2H of every layer's output.
@@ -315,10 +348,7 @@ def run_gpu(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (indexer keys + selected KV rows per step >> 126 MB)"},
         "algorithmic_gb_per_step": total_bytes / 1e9,
         "step_hbm_gbs": total_bytes / (ms / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": indexer_traffic(kern, idx_bytes),
-                     "peak_source": f"{src} hbm_gbs",
-                     "launch_ms": kms, "algorithmic_bytes_per_launch": idx_bytes},
+        "roofline": roof,
         "e2e": {"value": q_per_step * world / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step(w, [sd["n_split"] for sd in sds]) * args.steps,

@@ -26,8 +26,8 @@
 //                 allocates / frees TMEM.
 //   warp 1      : MMA issuer -- per tile, 8 x tcgen05.mma kind::f8f6f4 (M = 128 keys, N, K = 32)
 //                 into one of 512 / N accumulator slots; its commit frees the key stage.
-//   warps 2..5  : query preparation, once per epoch (hi / lo split, 128-byte-swizzled K-major).
-//   warps 6..13 : epilogue, two warpgroups taking alternate tiles -- thread = key row (= TMEM
+//   warps 2..3  : query preparation, once per epoch (hi / lo split, 128-byte-swizzled K-major).
+//   warps 4..11 : epilogue, two warpgroups taking alternate tiles -- thread = key row (= TMEM
 //                 lane): load the accumulator row, apply ReLU, the weighted head sum (eight
 //                 partial sums combined in a fixed order) and the token's FP8 scale, store.
 //
@@ -46,7 +46,8 @@ namespace lsa {
 
 namespace {
 
-constexpr int kPThreads = 448;         // 14 warps
+constexpr int kPThreads = 384;         // 12 warps
+constexpr int kPrepThreads = 64;       // warps 2..3
 constexpr int kPWarps = kPThreads / 32;
 constexpr int kBlock = 128;            // keys per MMA (M); a tile is NB such blocks
 constexpr int kBlockBytes = kBlock * 128;
@@ -147,19 +148,20 @@ __device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t v) {
     return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-// One epoch's query preparation by 128 threads (thread ct).  Work item i: row n = i / 8 (token
+// One epoch's query preparation by nthr threads (thread ct; nthr a multiple of 32).  Work item
+// i: row n = i / 8 (token
 // n / H_I, head n % H_I), 16-element chunk c = i % 8; the 8 chunks of a row sit in 8 consecutive
 // lanes, which reduce the row maximum by shuffles.  Loads are issued four items at a time.
 template <int N>
-__device__ void prepare_queries(const IndexArgs& a, int t0, int H_I, int ct, uint8_t* q_hi, uint8_t* q_lo,
-                                float* w_out) {
+__device__ void prepare_queries(const IndexArgs& a, int t0, int H_I, int ct, int nthr, uint8_t* q_hi,
+                                uint8_t* q_lo, float* w_out) {
     constexpr int kB = 4;
-    for (int i0 = ct; i0 < N * 8; i0 += 128 * kB) {
+    for (int i0 = ct; i0 < N * 8; i0 += nthr * kB) {
         uint4 raw[kB][2];
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
-            const int i = i0 + u * 128;
-            if (i < N * 8) {                                  // warp-uniform: N * 8 is a multiple of 128
+            const int i = i0 + u * nthr;
+            if (i < N * 8) {                                  // warp-uniform: N * 8 is a multiple of 32
                 const int n = i >> 3, c = i & 7;
                 const uint16_t* src = a.q + ((size_t)(t0 + n / H_I) * H_I + n % H_I) * 128 + c * 16;
                 raw[u][0] = *reinterpret_cast<const uint4*>(src);
@@ -168,7 +170,7 @@ __device__ void prepare_queries(const IndexArgs& a, int t0, int H_I, int ct, uin
         }
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
-            const int i = i0 + u * 128;
+            const int i = i0 + u * nthr;
             if (i >= N * 8) break;
             const int n = i >> 3, c = i & 7;
             const uint32_t wd[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
@@ -206,6 +208,23 @@ __device__ void prepare_queries(const IndexArgs& a, int t0, int H_I, int ct, uin
             if (c == 0) w_out[n] = a.w[(size_t)(t0 + n / H_I) * H_I + n % H_I] * exp2i(-s);
         }
     }
+}
+
+// Token gi (< kMaxG) of the group starting at t0: its position, and whether it is a valid query of
+// the group's sequence (a token of another sequence, or out of range, sees no key).
+__device__ __forceinline__ void set_group_validity(const IndexArgs& a, int t0, int G, int gi, int* pos, int* ok) {
+    int okv = 0, p = -1;
+    if (gi < G) {
+        const int b0 = a.q_seq[t0], sq = a.q_seq[t0 + gi];
+        p = a.q_pos[t0 + gi];
+        okv = sq == b0 && sq >= 0 && sq < a.B;
+        if (okv) {
+            const int len = a.seq_len[sq];
+            okv = len >= 1 && len <= a.L_alloc && p >= 0 && p < len;
+        }
+    }
+    pos[gi] = okv ? p : -1;
+    ok[gi] = okv;
 }
 
 // Weighted ReLU head sums of two accumulator rows held by this thread: item a (columns
@@ -275,7 +294,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         for (int s = 0; s < KS; ++s) { tc::mbar_init(&sm.full_k[s], 1); tc::mbar_init(&sm.empty_k[s], 129); }
         for (int s = 0; s < kSlots; ++s) { tc::mbar_init(&sm.d_full[s], 1); tc::mbar_init(&sm.d_empty[s], 128); }
         for (int b = 0; b < 2; ++b) {
-            tc::mbar_init(&sm.q_full[b], 128);
+            tc::mbar_init(&sm.q_full[b], kPrepThreads);
             tc::mbar_init(&sm.q_free[b][0], 128);
             tc::mbar_init(&sm.q_free[b][1], 128);
         }
@@ -312,6 +331,19 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t d_col = sm.tmem_base;
+
+    // The first group's queries: prepared by the query-preparation and epilogue warps together
+    // (the epilogue has nothing to do before the first accumulator is ready).
+    if (warp >= 2 && n_mine > 0) {
+        const int ct = threadIdx.x - 64;                                // 0..319
+        const Walk w0(sm.tstart, NG, k_lo);
+        const int t0 = (pa.group0 + w0.g) * G;
+        if (ct < kMaxG) set_group_validity(a, t0, G, ct, sm.pos[0], sm.ok[0]);
+        prepare_queries<N>(a, t0, H_I, ct, kPThreads - 64, sm.q[0][0], sm.q[0][1], sm.w[0]);
+        tc::fence_proxy_async_smem();
+        asm volatile("bar.sync 2, %0;" :: "n"(kPThreads - 64) : "memory");
+        if (warp < 4) tc::mbar_arrive(&sm.q_full[0]);
+    }
 
     if (warp == 0) {
         // ---------------- TMA producer
@@ -382,11 +414,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                 tc::mbar_wait(&sm.d_full[last_slot], last_ph, &drain_abort);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < 4) {
         // ---------------- query preparation, once per group epoch
-        const int ct = threadIdx.x - 64;                                // 0..127
-        Walk wk(sm.tstart, NG, k_lo);
-        for (int k = k_lo; k < k_hi; k = sm.tstart[wk.g + 1]) {
+        const int ct = threadIdx.x - 64;                                // 0..63
+        Walk wk(sm.tstart, NG, k_lo);                                   // epoch 0 is prepared above
+        for (int k = sm.tstart[wk.g + 1]; k < k_hi; k = sm.tstart[wk.g + 1]) {
             wk.to(k);
             // Group epoch e: its queries go to buffer e & 1 once both epilogue warpgroups have
             // released the group that used the buffer before (epoch e - 2).
@@ -395,27 +427,14 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                            !tc::mbar_wait(&sm.q_free[qb][1], ((e - 2) >> 1) & 1, abort_flag)))
                 break;
             const int t0 = (pa.group0 + wk.g) * G;
-            if (ct < kMaxG) {
-                int okv = 0, p = -1;
-                if (ct < G) {
-                    const int b0 = a.q_seq[t0], sq = a.q_seq[t0 + ct];
-                    p = a.q_pos[t0 + ct];
-                    okv = sq == b0 && sq >= 0 && sq < a.B;
-                    if (okv) {
-                        const int len = a.seq_len[sq];
-                        okv = len >= 1 && len <= a.L_alloc && p >= 0 && p < len;
-                    }
-                }
-                sm.pos[qb][ct] = okv ? p : -1;
-                sm.ok[qb][ct] = okv;
-            }
-            prepare_queries<N>(a, t0, H_I, ct, sm.q[qb][0], sm.q[qb][1], sm.w[qb]);
+            if (ct < kMaxG) set_group_validity(a, t0, G, ct, sm.pos[qb], sm.ok[qb]);
+            prepare_queries<N>(a, t0, H_I, ct, kPrepThreads, sm.q[qb][0], sm.q[qb][1], sm.w[qb]);
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(&sm.q_full[qb]);
         }
     } else {
         // ---------------- epilogue warpgroups: warpgroup wg takes the tiles j with j % 2 == wg
-        const int wg = (warp - 6) >> 2;
+        const int wg = (warp - 4) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -487,7 +506,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         }
         // Columns past a group's active tiles (all columns of a group with no visible key) are
         // -inf; CTA b fills the groups g with g % grid == b.
-        const int et = threadIdx.x - 192;                           // 0..255
+        const int et = threadIdx.x - 128;                           // 0..255
         for (int gl = blockIdx.x; gl < NG; gl += gridDim.x) {
             const int tg = (pa.group0 + gl) * G;
             const int from = (sm.tstart[gl + 1] - sm.tstart[gl]) * TK;
