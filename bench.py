@@ -196,6 +196,21 @@ def algorithmic_bytes(w, wt, steps_data):
     return total, idx_first
 
 
+def rank_workload(w, rank: int, world: int):
+    """The workload rank `rank` runs: same shapes on every rank (weak scaling), its own seed."""
+    return W.scaled(w.name, B=w.B, seed=w.seed + 1000 * rank) if world > 1 else w
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's value (all ranks take part; a plain return at world == 1)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def time_region(fn, steps, stream):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -217,8 +232,7 @@ def run_gpu(args, rank, world, local_rank):
     w = W.WORKLOADS[args.workload]
     if args.batch:
         w = W.scaled(args.workload, B=args.batch)
-    if world > 1:
-        w = W.scaled(args.workload, B=w.B, seed=w.seed + 1000 * rank)
+    w = rank_workload(w, rank, world)
     wt = D.build_workload(w, dev)
     stream = torch.cuda.current_stream()
     sds = [build_step(w, wt, pi, launch.split_for(w.T(p), w.H, w.cap)) for pi, p in enumerate(w.passes)]
@@ -259,9 +273,7 @@ def run_gpu(args, rank, world, local_rank):
         ms = time_region(fn, args.steps, stream)
     if world > 1:
         dist.barrier()
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
 
     q_per_step = w.queries_per_step()
     value = q_per_step * world / (ms / 1e3)
@@ -327,11 +339,7 @@ def run_gpu(args, rank, world, local_rank):
 
     for _ in range(2):
         e2e()
-    e2e_ms = time_region(e2e, args.steps, stream)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(time_region(e2e, args.steps, stream), world, dev)
     h2d = sum(h.numel() * h.element_size() for h in h_in)
     d2h = sum(h.numel() * h.element_size() for h in h_out)
 
@@ -381,8 +389,11 @@ def indexer_traffic(kern: str, idx_bytes: float):
 
 # ------------------------------------------------------------------ the CPU oracle (baseline / reference arm)
 
-def oracle_sample(w, n_tokens=1, layers_all=True):
-    """Times the float64 oracle's compute (selection + attention) on pre-decoded inputs of sampled tokens."""
+def oracle_sample(w, n_tokens=1, min_seconds=0.0):
+    """Times the float64 oracle's compute (selection + attention) on pre-decoded inputs of sampled tokens.
+
+    The compute over the sampled tokens repeats until at least `min_seconds` have been spent;
+    returns (tokens processed, seconds)."""
     from oracle import formats, lsa as olsa, run
     p = w.passes[0]
     T = w.T(p)
@@ -393,16 +404,19 @@ def oracle_sample(w, n_tokens=1, layers_all=True):
         b, pos, L, qi, wi = run.query_context(w, p, t)
         K = run.index_keys(w, p, b, np.arange(L if w.hi else pos + 1), plan)
         prepared.append((t, b, pos, L, qi, wi, K))
-    t0 = time.perf_counter()
-    for (t, b, pos, L, qi, wi, K) in prepared:
-        idx, _ = olsa.select(qi, wi, K, pos, w.k, w.n_sink, w.window, hi=w.hi, length=L, block_size=w.block_size,
-                             n_recall=w.n_recall)
-        for layer in p.layers:
-            q = formats.bf16_to_f64(W.attn_q_bits(w, layer, [t])[0])
-            Kr, Vr = run.kv_decoded(w, layer, b, idx)
-            olsa.attention(q, Kr, Vr, w.sm_scale)
-    dt = time.perf_counter() - t0
-    return len(toks), dt
+    done, dt = 0, 0.0
+    while done == 0 or dt < min_seconds:
+        t0 = time.perf_counter()
+        for (t, b, pos, L, qi, wi, K) in prepared:
+            idx, _ = olsa.select(qi, wi, K, pos, w.k, w.n_sink, w.window, hi=w.hi, length=L,
+                                 block_size=w.block_size, n_recall=w.n_recall)
+            for layer in p.layers:
+                q = formats.bf16_to_f64(W.attn_q_bits(w, layer, [t])[0])
+                Kr, Vr = run.kv_decoded(w, layer, b, idx)
+                olsa.attention(q, Kr, Vr, w.sm_scale)
+        dt += time.perf_counter() - t0
+        done += len(prepared)
+    return done, dt
 
 
 def cpu_cores():
@@ -467,10 +481,11 @@ def main():
     res, w, wt = run_gpu(args, rank, world, local_rank)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            n, dt = oracle_sample(W.WORKLOADS[args.workload], 2)
+            n, dt = oracle_sample(W.WORKLOADS[args.workload], 2, min_seconds=10.0)
             res["cpu_baseline"] = {"value": n / dt, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
-                                   "sample": f"{n} query tokens of {w.name} (all layers), float64 numpy/BLAS, "
-                                             f"inputs decoded beforehand; {dt:.2f} s"}
+                                   "sample": f"2 query tokens of {w.name} (all layers), computed {n // 2} times "
+                                             f"({n} tokens), float64 numpy/BLAS, inputs decoded beforehand; "
+                                             f"{dt:.1f} s"}
         print(json.dumps(res), flush=True)
     if world > 1:
         import torch.distributed as dist
