@@ -153,7 +153,7 @@ lsa_status lsa_topk(const lsa_batch* batch, const float* scores, int64_t ld_scor
  * K_j is row j of `kv` (dim = Dqk).  V_j is row j of `v` (dim = Dv) or, when v == NULL,
  * the first Dv elements of K_j (MLA absorbed layout).  FP8 rows are scale * code.
  * The list is cut into n_split contiguous chunks processed in parallel; the partial
- * results are merged with the log-sum-exp rule in a fixed binary tree ([explainer]
+ * results are merged with the log-sum-exp rule in chunk order ([explainer]
  * "③ KVP 解码切分示意": partial attention per KV shard, then merged -- here the shards are
  * chunks of one GPU's work).
  *   q [T][H][Dqk] BF16, o [T][H][Dv] BF16, lse [T][H] float (may be NULL).

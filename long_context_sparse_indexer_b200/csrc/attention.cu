@@ -279,52 +279,81 @@ sparse_attn_kernel(AttnArgs a) {
     }
 }
 
-// Merge of split partials: a fixed pairwise tree in binary-counter order (the balanced tree
-// when n_split is a power of two).  Thread = 4 consecutive V dims of one (token, head).
-__device__ __forceinline__ void lse_combine(float4& o1, float& l1, const float4& o2, float l2) {
-    const float m = fmaxf(l1, l2);
-    if (m == kNegInf) { o1 = make_float4(0.f, 0.f, 0.f, 0.f); l1 = kNegInf; return; }
-    const float w1 = expf(l1 - m), w2 = expf(l2 - m);
-    const float s = w1 + w2, r = 1.f / s;
-    o1.x = (w1 * o1.x + w2 * o2.x) * r;
-    o1.y = (w1 * o1.y + w2 * o2.y) * r;
-    o1.z = (w1 * o1.z + w2 * o2.z) * r;
-    o1.w = (w1 * o1.w + w2 * o2.w) * r;
-    l1 = m + logf(s);
+// Split merge: thread = 8 consecutive V dims of one (token, head).  With m = max_s lse_s and
+// w_s = exp(lse_s - m): o = sum_s (w_s / sum w) o_s and lse = m + log(sum w), sums in split
+// order.  Up to kMergeRegs splits are loaded before any arithmetic (one memory round trip).
+constexpr int kMergeThreads = 256;
+constexpr int kMergeRegs = 8;
+
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* part_o, const float* part_lse,
+                                                              int n_split, int H, int DV, uint16_t* o, float* lse) {
+    const int per_row = DV / 8;
+    const int i = blockIdx.x * kMergeThreads + threadIdx.x;       // (head, 8-dim chunk) of token t
+    const int t = blockIdx.y;
+    if (i >= H * per_row) return;
+    const int h = i / per_row, d = (i % per_row) * 8;
+    const size_t row0 = (size_t)t * n_split * H + h;               // (split 0, head h)
+    float m = kNegInf, wsum = 0.f;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (n_split <= kMergeRegs) {
+        float l[kMergeRegs];
+        float4 x0[kMergeRegs], x1[kMergeRegs];
+#pragma unroll
+        for (int s = 0; s < kMergeRegs; ++s) {
+            if (s < n_split) {
+                const size_t r = row0 + (size_t)s * H;
+                l[s] = __ldcg(part_lse + r);
+                const float4* src = reinterpret_cast<const float4*>(part_o + r * DV + d);
+                x0[s] = __ldcg(src);
+                x1[s] = __ldcg(src + 1);
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < kMergeRegs; ++s) if (s < n_split) m = fmaxf(m, l[s]);
+#pragma unroll
+        for (int s = 0; s < kMergeRegs; ++s) {
+            if (s < n_split) { l[s] = m == kNegInf ? 0.f : expf(l[s] - m); wsum += l[s]; }
+        }
+        const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+        for (int s = 0; s < kMergeRegs; ++s) {
+            if (s < n_split) {
+                const float ws = l[s] * rs;
+                acc[0] = fmaf(ws, x0[s].x, acc[0]); acc[1] = fmaf(ws, x0[s].y, acc[1]);
+                acc[2] = fmaf(ws, x0[s].z, acc[2]); acc[3] = fmaf(ws, x0[s].w, acc[3]);
+                acc[4] = fmaf(ws, x1[s].x, acc[4]); acc[5] = fmaf(ws, x1[s].y, acc[5]);
+                acc[6] = fmaf(ws, x1[s].z, acc[6]); acc[7] = fmaf(ws, x1[s].w, acc[7]);
+            }
+        }
+    } else {
+        for (int s = 0; s < n_split; ++s) m = fmaxf(m, __ldcg(part_lse + row0 + (size_t)s * H));
+        for (int s = 0; s < n_split; ++s) {
+            const float ls = __ldcg(part_lse + row0 + (size_t)s * H);
+            wsum += m == kNegInf ? 0.f : expf(ls - m);
+        }
+        const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
+        for (int s = 0; s < n_split; ++s) {
+            const size_t r = row0 + (size_t)s * H;
+            const float ws = (m == kNegInf ? 0.f : expf(__ldcg(part_lse + r) - m)) * rs;
+            const float4* src = reinterpret_cast<const float4*>(part_o + r * DV + d);
+            const float4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
+            acc[0] = fmaf(ws, a0.x, acc[0]); acc[1] = fmaf(ws, a0.y, acc[1]);
+            acc[2] = fmaf(ws, a0.z, acc[2]); acc[3] = fmaf(ws, a0.w, acc[3]);
+            acc[4] = fmaf(ws, a1.x, acc[4]); acc[5] = fmaf(ws, a1.y, acc[5]);
+            acc[6] = fmaf(ws, a1.z, acc[6]); acc[7] = fmaf(ws, a1.w, acc[7]);
+        }
+    }
+    uint4 pk;
+    pk.x = pack_bf16x2(acc[0], acc[1]); pk.y = pack_bf16x2(acc[2], acc[3]);
+    pk.z = pack_bf16x2(acc[4], acc[5]); pk.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(o + ((size_t)t * H + h) * DV + d) = pk;
+    if (lse && d == 0) lse[(size_t)t * H + h] = wsum > 0.f ? m + logf(wsum) : kNegInf;
 }
 
-__global__ void merge_kernel(const float* part_o, const float* part_lse, int n_split, int H, int DV,
-                             uint16_t* o, float* lse) {
-    const int t = blockIdx.y, h = blockIdx.x, d = threadIdx.x * 4;
-    if (d >= DV) return;
-    float4 st_o[7];
-    float st_l[7];
-    for (int s = 0; s < n_split; ++s) {
-        const size_t base = ((size_t)t * n_split + s) * H + h;
-        float4 v = *reinterpret_cast<const float4*>(part_o + base * DV + d);
-        float l = part_lse[base];
-        int lvl = 0;
-        for (int m = s; m & 1; m >>= 1, ++lvl) {
-            float4 acc = st_o[lvl];
-            float la = st_l[lvl];
-            lse_combine(acc, la, v, l);
-            v = acc;
-            l = la;
-        }
-        st_o[lvl] = v;
-        st_l[lvl] = l;
-    }
-    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
-    float tl = kNegInf;
-    bool have = false;
-    for (int lvl = 0; lvl < 7; ++lvl)
-        if ((n_split >> lvl) & 1) {
-            if (!have) { tot = st_o[lvl]; tl = st_l[lvl]; have = true; }
-            else { float4 acc = st_o[lvl]; float la = st_l[lvl]; lse_combine(acc, la, tot, tl); tot = acc; tl = la; }
-        }
-    uint16_t* orow = o + ((size_t)t * H + h) * DV + d;
-    *reinterpret_cast<uint2*>(orow) = make_uint2(pack_bf16x2(tot.x, tot.y), pack_bf16x2(tot.z, tot.w));
-    if (lse && d == 0) lse[(size_t)t * H + h] = tl;
+static cudaError_t launch_merge(const AttnArgs& a, int DV, cudaStream_t st) {
+    dim3 mg((a.H * (DV / 8) + kMergeThreads - 1) / kMergeThreads, a.T);
+    merge_kernel<<<mg, kMergeThreads, 0, st>>>(a.part_o, a.part_lse, a.n_split, a.H, DV, a.o, a.lse);
+    return cudaGetLastError();
 }
 
 template <int DQK, int DV, int MT, bool KV_FP8, bool SEP_V>
@@ -337,9 +366,7 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
     kern<<<grid, C::THREADS, C::SMEM, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess || a.n_split == 1) return e;
-    dim3 mg(a.H, a.T);
-    merge_kernel<<<mg, DV / 4, 0, st>>>(a.part_o, a.part_lse, a.n_split, a.H, DV, a.o, a.lse);
-    return cudaGetLastError();
+    return launch_merge(a, DV, st);
 }
 
 // Supported: (576, 512) MLA layout, BF16 or FP8 rows, H % 32 == 0; (128, 128) with a
@@ -349,9 +376,7 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, int DQK, int DV, bool kv_fp8, 
     if (sparse_attn_tc_supported(a, DQK, DV, sep_v)) {
         cudaError_t e = launch_sparse_attn_tc(a, kv_fp8, st);
         if (e != cudaSuccess || a.n_split == 1) return e;
-        dim3 mg(a.H, a.T);
-        merge_kernel<<<mg, DV / 4, 0, st>>>(a.part_o, a.part_lse, a.n_split, a.H, DV, a.o, a.lse);
-        return cudaGetLastError();
+        return launch_merge(a, DV, st);
     }
     if (DQK == 576 && DV == 512 && !sep_v)
         return kv_fp8 ? launch_attn_t<576, 512, 2, true, false>(a, st) : launch_attn_t<576, 512, 2, false, false>(a, st);
