@@ -18,6 +18,7 @@
 // with the sinks [0, a) and the window [b, pos], so the list comes out sorted and
 // de-duplicated.  Segments of up to 40960 columns are first cached in shared memory as
 // order keys (one coalesced read of the row); longer ones are re-read from global memory.
+#include <algorithm>
 #include <cooperative_groups.h>
 
 #include "kernels.cuh"
@@ -115,8 +116,33 @@ __device__ int cluster_exclusive(cg::cluster_group& cl, int* slot, int rank, int
     return before;
 }
 
+// Within one CTA: finds the bin of `hist` where the count from the top first reaches `need`
+// (same rule as cluster_threshold, CTA barriers only).
+__device__ void local_threshold(const int* hist, int nb, int need, int* s_warp, int* s_bin, int* s_above) {
+    const int per = (nb + kTopkThreads - 1) / kTopkThreads;
+    int local = 0;
+    for (int i = 0; i < per; ++i) {
+        const int bin = nb - 1 - ((int)threadIdx.x * per + i);
+        if (bin >= 0) local += hist[bin];
+    }
+    int total;
+    const int incl = cta_inclusive_scan(local, s_warp, total);
+    int run = incl - local;
+    for (int i = 0; i < per; ++i) {
+        const int bin = nb - 1 - ((int)threadIdx.x * per + i);
+        if (bin < 0) break;
+        const int h = hist[bin];
+        if (run < need && run + h >= need) { *s_bin = bin; *s_above = run; }
+        run += h;
+    }
+    __syncthreads();
+}
+
 // Segment length (columns) a CTA caches in shared memory as order keys.
 constexpr int kTopkCacheCols = 40960;
+// Candidate lists of the compacted finish: per CTA (in its `hsum` array) and merged in CTA 0.
+constexpr int kTopkLocalCap = 2048;
+constexpr int kTopkCap = 8192;
 
 template <bool CACHED>
 __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
@@ -124,7 +150,7 @@ topk_kernel(TopkArgs a) {
     __shared__ int hist[4096];
     __shared__ int hsum[4096];
     __shared__ int s_warp[kTopkWarps];
-    __shared__ int s_bin, s_above, s_slot[2];
+    __shared__ int s_bin, s_above, s_slot[3];
     extern __shared__ uint32_t s_keys[];          // CACHED: order key of each column of the segment, 0 = invalid
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
@@ -208,6 +234,137 @@ topk_kernel(TopkArgs a) {
     // Cluster histogram of the top 12 bits; its total is the number of candidates.
     const int n_valid = cluster_threshold(cl, rank, hist, hsum, 4096, a.k, s_warp, &s_bin, &s_above);
     const bool take_all = n_valid <= a.k;
+    const int a_lo = a.raw ? 0 : min(a.n_sink, pos + 1);
+    const int b_hi = a.raw ? 0x7fffffff : (a.window > 0 ? max(a_lo, pos - a.window + 1) : pos + 1);
+    auto position = [&](int cc) -> int {
+        if (a.raw || !a.cand) return cc;
+        return a.cand[(size_t)t * a.n_cand + cc / a.block_size] * a.block_size + cc % a.block_size;
+    };
+
+    // ---- compacted finish.  The top-k lies in the threshold bin b1 of pass 1 or above it, a few
+    // thousand columns of the row: every CTA lists its candidates (column order) in `hsum`, and
+    // when they fit, CTA 0 gathers them and completes the selection and the emission alone.
+    {
+        const uint32_t tb = a.k <= 0 ? 0xffffffffu : (take_all ? 1u : ((uint32_t)s_bin << 20));
+        uint32_t* lkey = reinterpret_cast<uint32_t*>(hsum);
+        int* lcol = hsum + kTopkLocalCap;
+        int cnt_w = 0;
+        for (int c = w0; c < w1; c += 32) {
+            const uint32_t key = key_at(c + lane);
+            cnt_w += __popc(__ballot_sync(0xffffffffu, key != 0u && key >= tb));
+        }
+        int cta_cnt;
+        const int wbase = cta_inclusive_scan(lane == 0 ? cnt_w : 0, s_warp, cta_cnt) - (lane == 0 ? cnt_w : 0);
+        int run = __shfl_sync(0xffffffffu, wbase, 0);
+        for (int c = w0; c < w1; c += 32) {
+            const uint32_t key = key_at(c + lane);
+            const bool sel = key != 0u && key >= tb;
+            const uint32_t m = __ballot_sync(0xffffffffu, sel);
+            const int at = run + __popc(m & ((1u << lane) - 1));
+            if (sel && at < kTopkLocalCap) { lkey[at] = key; lcol[at] = c + lane; }
+            run += __popc(m);
+        }
+        if (threadIdx.x == 0) s_slot[2] = cta_cnt;
+        cl.sync();                                       // counts and lists complete everywhere
+        int total = 0, biggest = 0;
+        for (int r = 0; r < kTopkCluster; ++r) {
+            const int v = *cl.map_shared_rank(&s_slot[2], r);
+            total += v;
+            biggest = max(biggest, v);
+        }
+        if (biggest <= kTopkLocalCap && total <= kTopkCap) {
+            uint32_t* ckey = s_keys;                     // CTA 0: merged candidates (its cache is done)
+            int* ccol = reinterpret_cast<int*>(s_keys) + kTopkCap;
+            if (rank == 0) {
+                int base = 0;
+                for (int r = 0; r < kTopkCluster; ++r) {
+                    const int n_r = *cl.map_shared_rank(&s_slot[2], r);
+                    const uint32_t* pk = cl.map_shared_rank(lkey, r);
+                    const int* pc = cl.map_shared_rank(lcol, r);
+                    for (int i = threadIdx.x; i < n_r; i += kTopkThreads) {
+                        ckey[base + i] = pk[i];
+                        ccol[base + i] = pc[i];
+                    }
+                    base += n_r;
+                }
+            }
+            cl.sync();                                   // CTA 0 has read every list
+            if (rank != 0) return;
+            __syncthreads();
+            const int n = total;
+            uint32_t vs = 0;
+            int m_keep = 0;
+            if (!take_all && a.k > 0) {
+                const uint32_t b1 = (uint32_t)s_bin;
+                int above = s_above;
+                for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
+                __syncthreads();
+                for (int i = threadIdx.x; i < n; i += kTopkThreads) {
+                    const uint32_t key = ckey[i];
+                    if ((key >> 20) == b1) atomicAdd(&hist[(key >> 8) & 0xfff], 1);
+                }
+                __syncthreads();
+                local_threshold(hist, 4096, a.k - above, s_warp, &s_bin, &s_above);
+                const uint32_t pre = (b1 << 12) | (uint32_t)s_bin;
+                above += s_above;
+                for (int i = threadIdx.x; i < 256; i += kTopkThreads) hist[i] = 0;
+                __syncthreads();
+                for (int i = threadIdx.x; i < n; i += kTopkThreads) {
+                    const uint32_t key = ckey[i];
+                    if ((key >> 8) == pre) atomicAdd(&hist[key & 0xff], 1);
+                }
+                __syncthreads();
+                local_threshold(hist, 256, a.k - above, s_warp, &s_bin, &s_above);
+                above += s_above;
+                vs = (pre << 8) | (uint32_t)s_bin;
+                m_keep = a.k - above;                    // keys == vs to keep, lowest columns first
+            }
+            const bool every = take_all || a.k <= 0;     // every candidate is selected (none when k = 0)
+            // Emission in column order: thread = contiguous chunk of the candidates.
+            const int chunk = (n + kTopkThreads - 1) / kTopkThreads;
+            const int i0 = min(n, (int)threadIdx.x * chunk), i1 = min(n, i0 + chunk);
+            int eq_t = 0;
+            if (!every)
+                for (int i = i0; i < i1; ++i) eq_t += ckey[i] == vs;
+            int eq_tot;
+            const int eq_base = cta_inclusive_scan(eq_t, s_warp, eq_tot) - eq_t;
+            auto kept = [&](int i, int& eq_seen) -> bool {
+                const uint32_t key = ckey[i];
+                bool sel;
+                if (every) sel = a.k > 0;
+                else if (key > vs) sel = true;
+                else if (key == vs) sel = eq_base + eq_seen++ < m_keep;
+                else sel = false;
+                if (!sel) return false;
+                if (a.raw) return true;
+                const int p = position(ccol[i]);
+                return p >= a_lo && p < b_hi;
+            };
+            int keep_t = 0;
+            {
+                int eq_seen = 0;
+                for (int i = i0; i < i1; ++i) keep_t += kept(i, eq_seen);
+            }
+            int written;
+            const int keep_base = cta_inclusive_scan(keep_t, s_warp, written) - keep_t;
+            {
+                int eq_seen = 0, o = a_lo + keep_base;
+                for (int i = i0; i < i1; ++i)
+                    if (kept(i, eq_seen)) out[o++] = a.raw ? ccol[i] : position(ccol[i]);
+            }
+            int n_out = a_lo + written;
+            if (!a.raw) {
+                for (int i = threadIdx.x; i < a_lo; i += kTopkThreads) out[i] = i;
+                const int tail = pos + 1 - b_hi;
+                for (int i = threadIdx.x; i < tail; i += kTopkThreads) out[n_out + i] = b_hi + i;
+                n_out += max(tail, 0);
+            }
+            for (int i = n_out + threadIdx.x; i < a.ld_idx; i += kTopkThreads) out[i] = -1;
+            if (threadIdx.x == 0) a.count[t] = n_out;
+            return;
+        }
+        // Too many candidates: the cluster continues with the full passes below.
+    }
     uint32_t vstar = 0;
     int above = 0;
     if (!take_all && a.k > 0) {
@@ -238,8 +395,6 @@ topk_kernel(TopkArgs a) {
     const int m_ties = a.k - above;           // keys == v* to keep (lowest columns first)
 
     // ---- emission: ascending columns
-    const int a_lo = a.raw ? 0 : min(a.n_sink, pos + 1);
-    const int b_hi = a.raw ? 0x7fffffff : (a.window > 0 ? max(a_lo, pos - a.window + 1) : pos + 1);
     auto classify = [&](int cc, bool& eq, bool& gt, int& p) {
         eq = gt = false;
         p = -1;
@@ -321,14 +476,18 @@ topk_kernel(TopkArgs a) {
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
     const int per_cta = ((a.n_cols + kTopkCluster - 1) / kTopkCluster + 31) / 32 * 32;
+    const size_t cand_smem = (size_t)kTopkCap * 8;             // merged candidates (keys, columns) in CTA 0
     if (per_cta <= kTopkCacheCols) {
-        const size_t smem = (size_t)per_cta * 4;
+        const size_t smem = std::max((size_t)per_cta * 4, cand_smem);
         cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kTopkCacheCols * 4);
+                                             (int)std::max((size_t)kTopkCacheCols * 4, cand_smem));
         if (e != cudaSuccess) return e;
         topk_kernel<true><<<a.T * kTopkCluster, kTopkThreads, smem, st>>>(a);
     } else {
-        topk_kernel<false><<<a.T * kTopkCluster, kTopkThreads, 0, st>>>(a);
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)cand_smem);
+        if (e != cudaSuccess) return e;
+        topk_kernel<false><<<a.T * kTopkCluster, kTopkThreads, cand_smem, st>>>(a);
     }
     return cudaGetLastError();
 }
