@@ -15,11 +15,12 @@
 // 16 K-steps, and a 4-stage ring of 32-row KV tiles (36 KB each) in the 128-byte-swizzled
 // K-major layout, read as the B operand of S (K-major) and of P V (MN-major).
 //
-//   warps 0..7 : gather -- warps 2s and 2s+1 fill stage s with the tiles j = s, s+4, ..., 16
-//                rows each: the rows' indices (prefetched one tile ahead) go to shared memory,
-//                then the rows are copied with 16-byte cp.async (FP8 rows are widened to BF16
-//                exactly on the way); per-row scale and validity.  Two warps per tile keep
-//                twice the copies in flight that one warp would.
+//   warps 0..7 : gather -- warps 2s and 2s+1 fill stage s with the tiles j = s, s+4, ...: the
+//                rows' indices (prefetched one tile ahead) and per-row scale and validity go
+//                to shared memory; the two CTAs of a (split, token) form a cluster and each
+//                copies only its half of the rows (16-byte cp.async; FP8 rows widened to BF16
+//                exactly on the way), pushing them into the peer's stage with bulk
+//                shared-to-shared copies, so each row crosses into the SMs once.
 //   warp 12    : MMA issuer -- issues whatever is ready, in order per kind: S_j (16 SS + 20 TS
 //                MMAs, N = 32) once tile j has landed and P V_{j-2} has been issued, and
 //                O += P_j V_j (2 TS MMAs, N = 256) once the softmax of tile j is done.
@@ -63,7 +64,7 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 template <bool KV_FP8>
-__global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a) {
+__global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int split = blockIdx.x, half = blockIdx.y, t = blockIdx.z;
@@ -86,7 +87,9 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
     const uint16_t* qt = a.q + (size_t)t * 128 * kD;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStagesA; ++i) { tc::mbar_init(&sm.kv_full[i], 64); tc::mbar_init(&sm.kv_empty[i], 1); }
+        // kv_full: this CTA's two gather warps (one of them also expecting the peer's rows);
+        // kv_empty: the P V commits of both CTAs of the pair.
+        for (int i = 0; i < kStagesA; ++i) { tc::mbar_init(&sm.kv_full[i], 64); tc::mbar_init(&sm.kv_empty[i], 2); }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.s_full[i], 1);
             tc::mbar_init(&sm.p_full[i], 128);
@@ -99,6 +102,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
     tc::tc_fence_before();
     __syncthreads();
+    tc::cluster_sync_all();                      // the peer's barriers exist before any cross-CTA traffic
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t o_col = tmem, s_col = tmem + 256, p_col = tmem + 320, qt_col = tmem + 352;
@@ -144,34 +148,40 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
     }
 
     if (warp < 8) {
-        // ---------------- gather producers: warps 2s, 2s + 1 own stage s (rows 0..15 / 16..31
-        // of the tiles j = s, s + 4, ...)
-        const int g = warp >> 1, rh = (warp & 1) * (kRows / 2);
-        auto fetch_row = [&](int j) -> int {
+        // ---------------- gather producers: warps 2s, 2s + 1 own stage s (tiles j = s, s + 4, ...).
+        // The two CTAs of the pair (V halves) gather the same rows: this CTA copies the 16 rows of
+        // its own half of each tile (8 per warp) and pushes them into the peer's stage with
+        // unicast bulk shared-to-shared copies, completing on the peer's kv_full; the peer does
+        // the same for the other 16.  A stage is reused only once both CTAs' P V have read it.
+        const int g = warp >> 1, wsub = warp & 1;
+        const uint32_t peer = (uint32_t)(half ^ 1);
+        const int rcopy = half * (kRows / 2) + wsub * (kRows / 4);  // first row this warp copies
+        auto fetch_row = [&](int j) -> int {                       // lane l: index of row l of tile j
             if (j >= n_tiles) return -1;
-            const int r0 = r_beg + j * kRows + rh;
-            return lane < min(kRows / 2, r_end - r0) ? irow[r0 + lane] : -1;
+            const int r0 = r_beg + j * kRows;
+            return lane < min(kRows, r_end - r0) ? irow[r0 + lane] : -1;
         };
         int nxt = fetch_row(g);
         for (int j = g; j < n_tiles; j += kStagesA) {
             const int cur = nxt;
             nxt = fetch_row(j + kStagesA);                         // prefetch this warp's next tile
             if (!tc::mbar_wait(&sm.kv_empty[g], ((j / kStagesA) + 1) & 1, abort_flag)) break;
-            const int nr = min(kRows / 2, r_end - (r_beg + j * kRows + rh));
-            if (lane < kRows / 2) {
+            const int nr = min(kRows, r_end - (r_beg + j * kRows));
+            {
+                // Both warps of the pair write the same metadata of all 32 rows (identical values).
                 const bool v = cur >= 0 && cur < len;
-                if (lane < nr && !v) report(a.status, LSA_ERR_DEVICE_DATA);
+                if (wsub == 0 && half == 0 && lane < nr && !v) report(a.status, LSA_ERR_DEVICE_DATA);
                 const float vs = KV_FP8 ? (v ? kvs[cur] : 0.f) : 1.f;
-                sm.rows[g][rh + lane] = v ? cur : -1;
-                sm.vscale[g][rh + lane] = vs;
-                sm.kscale[g][rh + lane] = v ? vs * a.sm_scale_log2 : 0.f;
+                sm.rows[g][lane] = v ? cur : -1;
+                sm.vscale[g][lane] = vs;
+                sm.kscale[g][lane] = v ? vs * a.sm_scale_log2 : 0.f;
             }
             __syncwarp();
             uint8_t* tile = sm.kv[g];
             if (!KV_FP8) {
-#pragma unroll 4
-                for (int i = lane; i < (kRows / 2) * (kD / 8); i += 32) {
-                    const int r = rh + i / (kD / 8), c = i % (kD / 8);
+#pragma unroll 3
+                for (int i = lane; i < (kRows / 4) * (kD / 8); i += 32) {
+                    const int r = rcopy + i / (kD / 8), c = i % (kD / 8);
                     const int row = sm.rows[g][r];
                     uint8_t* dst = tile + (c >> 3) * (kRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
                     cp_async16(dst, kvb + (size_t)(row >= 0 ? row : 0) * a.kv_tok_b + c * 16, row >= 0);
@@ -179,43 +189,49 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                 cp_async_commit();
                 cp_async_wait<0>();
             } else {
-                constexpr int kChunks = (kRows / 2) * (kD / 16);       // 16 codes per chunk
-                constexpr int kBatch = 12;
+                constexpr int kChunks = (kRows / 4) * (kD / 16);       // 16 codes per chunk
+                constexpr int kBatch = 5;
                 for (int i0 = lane; i0 < kChunks; i0 += 32 * kBatch) {
-                    uint4 raw[kBatch];
+                uint4 raw[kBatch];
 #pragma unroll
-                    for (int u = 0; u < kBatch; ++u) {
-                        const int i = i0 + u * 32;
-                        raw[u] = make_uint4(0, 0, 0, 0);
-                        if (i < kChunks) {
-                            const int row = sm.rows[g][rh + i / (kD / 16)];
-                            if (row >= 0) raw[u] = ldg_nc16(kvb + (size_t)row * a.kv_tok_b + (i % (kD / 16)) * 16);
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < kBatch; ++u) {
-                        const int i = i0 + u * 32;
-                        if (i >= kChunks) break;
-                        const int r = rh + i / (kD / 16), c = i % (kD / 16);
-                        const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw[u]);
-                        uint32_t ow[8];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            ow[2 * q] = e4m3x2_to_bf16x2((uint16_t)(wd[q] & 0xffff));
-                            ow[2 * q + 1] = e4m3x2_to_bf16x2((uint16_t)(wd[q] >> 16));
-                        }
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int cb = 2 * c + hh;                  // bf16 chunk index (8 dims)
-                            uint8_t* dst = tile + (cb >> 3) * (kRows * 128) + r * 128 + (((cb & 7) ^ (r & 7)) << 4);
-                            *reinterpret_cast<uint4*>(dst) =
-                                make_uint4(ow[4 * hh], ow[4 * hh + 1], ow[4 * hh + 2], ow[4 * hh + 3]);
-                        }
+                for (int u = 0; u < kBatch; ++u) {
+                    const int i = i0 + u * 32;
+                    raw[u] = make_uint4(0, 0, 0, 0);
+                    if (i < kChunks) {
+                        const int row = sm.rows[g][rcopy + i / (kD / 16)];
+                        if (row >= 0) raw[u] = ldg_nc16(kvb + (size_t)row * a.kv_tok_b + (i % (kD / 16)) * 16);
                     }
                 }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int i = i0 + u * 32;
+                    if (i >= kChunks) break;
+                    const int r = rcopy + i / (kD / 16), c = i % (kD / 16);
+                    const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw[u]);
+                    uint32_t ow[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        ow[2 * q] = e4m3x2_to_bf16x2((uint16_t)(wd[q] & 0xffff));
+                        ow[2 * q + 1] = e4m3x2_to_bf16x2((uint16_t)(wd[q] >> 16));
+                    }
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int cb = 2 * c + hh;                  // bf16 chunk index (8 dims)
+                        uint8_t* dst = tile + (cb >> 3) * (kRows * 128) + r * 128 + (((cb & 7) ^ (r & 7)) << 4);
+                        *reinterpret_cast<uint4*>(dst) =
+                            make_uint4(ow[4 * hh], ow[4 * hh + 1], ow[4 * hh + 2], ow[4 * hh + 3]);
+                    }
+                }
+                }
             }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&sm.kv_full[g]);
+            tc::fence_proxy_async_smem();                          // this warp's rows, for the bulk copies
+            __syncwarp();
+            if (lane < kAtoms) {                                   // its 8 rows of atom `lane` to the peer
+                const uint8_t* src = tile + lane * (kRows * 128) + rcopy * 128;
+                tc::bulk_copy_to_peer(tc::peer_smem(src, peer), src, (kRows / 4) * 128, tc::peer_smem(&sm.kv_full[g], peer));
+            }
+            if (wsub == 0 && lane == 0) tc::mbar_expect_tx(&sm.kv_full[g], (kRows / 2) * 128 * kAtoms);   // the peer's rows
+            else tc::mbar_arrive(&sm.kv_full[g]);
         }
     } else if (warp == 12) {
         // ---------------- MMA issuer: S_j and P_j V_j, each in order, whichever is ready
@@ -261,7 +277,7 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
                         tc::mma_f16_ts(o_col, p_col + (npv & 1) * 16 + kk * 8, bd, idesc_o,
                                        (npv > 0 || kk > 0) ? 1u : 0u);
                     }
-                    tc::mma_commit(&sm.kv_empty[npv % kStagesA]);
+                    tc::mma_commit_cluster(&sm.kv_empty[npv % kStagesA], 0x3);   // both CTAs of the pair
                     tc::mma_commit(&sm.o_done[npv & 1]);
                     ++npv;
                     progressed = true;
@@ -406,6 +422,15 @@ __global__ void __launch_bounds__(kAThreads, 1) sparse_attn_tc_kernel(AttnArgs a
 
     tc::tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) {
+        // The peer's copies into this CTA's last stages have landed (already true unless a wait gave
+        // up; bounded) before either CTA can leave.
+        volatile int drain_abort = 0;
+        for (int j = max(0, n_tiles - kStagesA); j < n_tiles; ++j)
+            tc::mbar_wait(&sm.kv_full[j % kStagesA], (j / kStagesA) & 1, &drain_abort);
+    }
+    __syncthreads();
+    tc::cluster_sync_all();                      // every copy into either CTA has landed and been read
     if (sm.abort && threadIdx.x == 0) report(a.status, LSA_ERR_TIMEOUT);
     if (warp == 0) {
         tc::tc_fence_after();
