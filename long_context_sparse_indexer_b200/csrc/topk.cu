@@ -142,6 +142,7 @@ __device__ void local_threshold(const int* hist, int nb, int need, int* s_warp, 
 constexpr int kTopkCacheCols = 40960;
 // Candidate lists of the compacted finish: per CTA (in its `hsum` array) and merged in CTA 0.
 constexpr int kTopkLocalCap = 2048;
+constexpr int kTopkWarpCap = kTopkLocalCap / kTopkWarps;   // per warp
 constexpr int kTopkCap = 8192;
 
 template <bool CACHED>
@@ -150,7 +151,8 @@ topk_kernel(TopkArgs a) {
     __shared__ int hist[4096];
     __shared__ int hsum[4096];
     __shared__ int s_warp[kTopkWarps];
-    __shared__ int s_bin, s_above, s_slot[3];
+    __shared__ int s_bin, s_above, s_slot[3], s_wmax;
+    __shared__ int s_wcnt[kTopkWarps];
     extern __shared__ uint32_t s_keys[];          // CACHED: order key of each column of the segment, 0 = invalid
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
@@ -242,53 +244,55 @@ topk_kernel(TopkArgs a) {
     };
 
     // ---- compacted finish.  The top-k lies in the threshold bin b1 of pass 1 or above it, a few
-    // thousand columns of the row: every CTA lists its candidates (column order) in `hsum`, and
-    // when they fit, CTA 0 gathers them and completes the selection and the emission alone.
+    // thousand columns of the row: every warp lists its candidates (column order) in its region
+    // of `hsum`; when they fit, every warp stores them into CTA 0's merged list, and CTA 0
+    // completes the selection and the emission alone.
     {
         const uint32_t tb = a.k <= 0 ? 0xffffffffu : (take_all ? 1u : ((uint32_t)s_bin << 20));
+        // One pass: warp w appends its candidates (column order) to its own region of kTopkWarpCap
+        // slots of the CTA's list in `hsum` (keys, then columns).
         uint32_t* lkey = reinterpret_cast<uint32_t*>(hsum);
         int* lcol = hsum + kTopkLocalCap;
-        int cnt_w = 0;
-        for (int c = w0; c < w1; c += 32) {
-            const uint32_t key = key_at(c + lane);
-            cnt_w += __popc(__ballot_sync(0xffffffffu, key != 0u && key >= tb));
-        }
-        int cta_cnt;
-        const int wbase = cta_inclusive_scan(lane == 0 ? cnt_w : 0, s_warp, cta_cnt) - (lane == 0 ? cnt_w : 0);
-        int run = __shfl_sync(0xffffffffu, wbase, 0);
+        int run = 0;
         for (int c = w0; c < w1; c += 32) {
             const uint32_t key = key_at(c + lane);
             const bool sel = key != 0u && key >= tb;
             const uint32_t m = __ballot_sync(0xffffffffu, sel);
             const int at = run + __popc(m & ((1u << lane) - 1));
-            if (sel && at < kTopkLocalCap) { lkey[at] = key; lcol[at] = c + lane; }
+            if (sel && at < kTopkWarpCap) { lkey[warp * kTopkWarpCap + at] = key; lcol[warp * kTopkWarpCap + at] = c + lane; }
             run += __popc(m);
         }
-        if (threadIdx.x == 0) s_slot[2] = cta_cnt;
-        cl.sync();                                       // counts and lists complete everywhere
-        int total = 0, biggest = 0;
+        if (lane == 0) s_wcnt[warp] = run;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int tot = 0, big = 0;
+            for (int w = 0; w < kTopkWarps; ++w) { tot += s_wcnt[w]; big = max(big, s_wcnt[w]); }
+            s_slot[2] = tot;
+            s_wmax = big;
+        }
+        cl.sync();                                       // counts everywhere (CTA 0's cache is done)
+        int total = 0, biggest = 0, before = 0;
         for (int r = 0; r < kTopkCluster; ++r) {
             const int v = *cl.map_shared_rank(&s_slot[2], r);
+            if (r < rank) before += v;
             total += v;
-            biggest = max(biggest, v);
+            biggest = max(biggest, *cl.map_shared_rank(&s_wmax, r));
         }
-        if (biggest <= kTopkLocalCap && total <= kTopkCap) {
-            uint32_t* ckey = s_keys;                     // CTA 0: merged candidates (its cache is done)
+        if (biggest <= kTopkWarpCap && total <= kTopkCap) {
+            uint32_t* ckey = s_keys;                     // CTA 0: merged candidates, column order
             int* ccol = reinterpret_cast<int*>(s_keys) + kTopkCap;
-            if (rank == 0) {
-                int base = 0;
-                for (int r = 0; r < kTopkCluster; ++r) {
-                    const int n_r = *cl.map_shared_rank(&s_slot[2], r);
-                    const uint32_t* pk = cl.map_shared_rank(lkey, r);
-                    const int* pc = cl.map_shared_rank(lcol, r);
-                    for (int i = threadIdx.x; i < n_r; i += kTopkThreads) {
-                        ckey[base + i] = pk[i];
-                        ccol[base + i] = pc[i];
-                    }
-                    base += n_r;
+            {
+                // Every warp stores its candidates straight into CTA 0's merged list.
+                int wb = before;
+                for (int w = 0; w < warp; ++w) wb += s_wcnt[w];
+                uint32_t* dk = cl.map_shared_rank(ckey, 0);
+                int* dc = cl.map_shared_rank(ccol, 0);
+                for (int i = lane; i < s_wcnt[warp]; i += 32) {
+                    dk[wb + i] = lkey[warp * kTopkWarpCap + i];
+                    dc[wb + i] = lcol[warp * kTopkWarpCap + i];
                 }
             }
-            cl.sync();                                   // CTA 0 has read every list
+            cl.sync();                                   // every candidate has reached CTA 0
             if (rank != 0) return;
             __syncthreads();
             const int n = total;
