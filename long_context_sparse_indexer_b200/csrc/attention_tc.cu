@@ -9,9 +9,9 @@
 // the duplicated QK^T keeps every CTA independent (no cross-CTA exchange) at 1.53x the
 // minimum tensor work.
 //
-// Memory plan.  TMEM (512 columns): O half [0,256), S double buffer [256,320), P double
-// buffer [320,352), and Q dims 256..575 [352,512) as the A operand of the last 20 K-steps of
-// S.  Shared memory: Q dims 0..255 (4 swizzled K atoms, 64 KB) as the A operand of the first
+// Memory plan.  TMEM (512 columns): O half [0,256), three S / P buffers [256,352) -- the
+// softmax writes P (BF16, 16 columns) over the S it has just read, so S can run two tiles
+// ahead of P V -- and Q dims 256..575 [352,512) as the A operand of the last 20 K-steps of S.  Shared memory: Q dims 0..255 (4 swizzled K atoms, 64 KB) as the A operand of the first
 // 16 K-steps, and a 4-stage ring of 32-row KV tiles (36 KB each) in the 128-byte-swizzled
 // K-major layout, read as the B operand of S (K-major) and of P V (MN-major).
 //
@@ -22,7 +22,7 @@
 //                exactly on the way), pushing them into the peer's stage with bulk
 //                shared-to-shared copies, so each row crosses into the SMs once.
 //   warp 12    : MMA issuer -- issues whatever is ready, in order per kind: S_j (16 SS + 20 TS
-//                MMAs, N = 32) once tile j has landed and P V_{j-2} has been issued, and
+//                MMAs, N = 32) once tile j has landed and P V_{j-3} has been issued, and
 //                O += P_j V_j (2 TS MMAs, N = 256) once the softmax of tile j is done.
 //   warps 8..11: softmax -- thread = head (TMEM lane): online max / sum with lazy rescaling
 //                of O (only when the running max grows by more than 2^8; warp-uniform, so
@@ -39,6 +39,7 @@ namespace {
 constexpr int kAThreads = 416;
 constexpr int kRows = 32;                    // KV rows per tile
 constexpr int kStagesA = 4;                  // KV tile ring
+constexpr int kSP = 3;                       // S / P buffers in TMEM (P overwrites its own S)
 constexpr int kD = 576, kDv = 512, kHalf = 256;
 constexpr int kAtoms = kD / 64;              // 64-element (128-byte) K atoms of a KV row
 constexpr int kQSmemAtoms = 4;               // Q dims 0..255 in shared memory
@@ -50,9 +51,10 @@ struct AttnSmem {
     alignas(1024) uint8_t q[kQBytes];
     alignas(1024) uint8_t kv[kStagesA][kTileBytes];
     alignas(16) float kscale[kStagesA][kRows];   // per-row FP8 scale x softmax scale (0 for masked rows)
+    alignas(16) float kmask[kStagesA][kRows];    // 0, or -inf for masked rows (added to the scaled score)
     alignas(16) float vscale[kStagesA][kRows];   // per-row FP8 scale (1 for BF16)
     int rows[kStagesA][kRows];
-    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[2], p_full[2], o_done[2], q_ready;
+    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[kSP], p_full[kSP], o_done[2], q_ready;
     uint32_t tmem_base;
     int abort;
 };
@@ -91,10 +93,9 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1) sparse
         // kv_empty: the P V commits of both CTAs of the pair.
         for (int i = 0; i < kStagesA; ++i) { tc::mbar_init(&sm.kv_full[i], 64); tc::mbar_init(&sm.kv_empty[i], 2); }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&sm.s_full[i], 1);
-            tc::mbar_init(&sm.p_full[i], 128);
             tc::mbar_init(&sm.o_done[i], 1);
         }
+        for (int i = 0; i < kSP; ++i) { tc::mbar_init(&sm.s_full[i], 1); tc::mbar_init(&sm.p_full[i], 128); }
         tc::mbar_init(&sm.q_ready, 128);
         sm.abort = 0;
         tc::fence_barrier_init();
@@ -105,7 +106,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1) sparse
     tc::cluster_sync_all();                      // the peer's barriers exist before any cross-CTA traffic
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t o_col = tmem, s_col = tmem + 256, p_col = tmem + 320, qt_col = tmem + 352;
+    const uint32_t o_col = tmem, s_col = tmem + 256, qt_col = tmem + 256 + kSP * 32;   // O, S / P, Q tail
     // The softmax warps load Q while the gather warps already fetch KV tiles: dims 0..255 into
     // shared memory (K-major, 128-byte swizzle), dims 256..575 into TMEM (thread = head = lane).
     if (warp >= 8 && warp < 12) {
@@ -175,6 +176,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1) sparse
                 sm.rows[g][lane] = v ? cur : -1;
                 sm.vscale[g][lane] = vs;
                 sm.kscale[g][lane] = v ? vs * a.sm_scale_log2 : 0.f;
+                sm.kmask[g][lane] = v ? 0.f : kNegInf;
             }
             __syncwarp();
             uint8_t* tile = sm.kv[g];
@@ -247,10 +249,10 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1) sparse
             while (npv < n_tiles) {
                 bool progressed = false;
                 // S_ns needs its KV tile and its S/P buffer free (P V_{ns-2} issued).
-                if (ns < n_tiles && ns <= npv + 1 && tc::mbar_try_wait(&sm.kv_full[ns % kStagesA], (ns / kStagesA) & 1)) {
+                if (ns < n_tiles && ns <= npv + kSP - 1 && tc::mbar_try_wait(&sm.kv_full[ns % kStagesA], (ns / kStagesA) & 1)) {
                     tc::fence_proxy_async_smem();
                     tc::tc_fence_after();
-                    const int sb = ns & 1;
+                    const int sb = ns % kSP;
                     const uint32_t kaddr = tc::smem_u32(sm.kv[ns % kStagesA]);
 #pragma unroll
                     for (int kk = 0; kk < kQSmemAtoms * 4; ++kk) {
@@ -268,13 +270,13 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1) sparse
                     progressed = true;
                 }
                 // P V_npv needs the softmax of tile npv.
-                if (npv < ns && tc::mbar_try_wait(&sm.p_full[npv & 1], (npv >> 1) & 1)) {
+                if (npv < ns && tc::mbar_try_wait(&sm.p_full[npv % kSP], (npv / kSP) & 1)) {
                     tc::tc_fence_after();
                     const uint32_t vaddr = tc::smem_u32(sm.kv[npv % kStagesA]) + (4 * half) * (kRows * 128);
 #pragma unroll
                     for (int kk = 0; kk < kRows / 16; ++kk) {
                         const uint64_t bd = tc::sdesc_sw128_lbo(vaddr + kk * 16 * 128, kRows * 128, 1024);
-                        tc::mma_f16_ts(o_col, p_col + (npv & 1) * 16 + kk * 8, bd, idesc_o,
+                        tc::mma_f16_ts(o_col, s_col + (npv % kSP) * 32 + kk * 8, bd, idesc_o,
                                        (npv > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit_cluster(&sm.kv_empty[npv % kStagesA], 0x3);   // both CTAs of the pair
@@ -299,25 +301,24 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1) sparse
         float m_run = kNegInf, l_run = 0.f;
         bool alive = true;
         for (int j = 0; j < n_tiles; ++j) {
-            const int sb = j & 1, st = j % kStagesA;
-            if (!tc::mbar_wait(&sm.s_full[sb], (j >> 1) & 1, abort_flag)) { alive = false; break; }
+            const int sb = j % kSP, st = j % kStagesA;
+            if (!tc::mbar_wait(&sm.s_full[sb], (j / kSP) & 1, abort_flag)) { alive = false; break; }
             // The tile's row scales were written by the gather warp before kv_full.
             if (!tc::mbar_wait(&sm.kv_full[st], (j / kStagesA) & 1, abort_flag)) { alive = false; break; }
-            // P buffer sb was last read by P V_{j-2}.
-            if (j >= 2 && !tc::mbar_wait(&sm.o_done[sb], ((j - 2) >> 1) & 1, abort_flag)) { alive = false; break; }
             tc::tc_fence_after();
             uint32_t sv[32];
             tc::tmem_ld32(s_col + sb * 32 + lane_off, sv);
             tc::tmem_wait_ld();
             float x[32];
             const float4* ks4 = reinterpret_cast<const float4*>(sm.kscale[st]);
+            const float4* km4 = reinterpret_cast<const float4*>(sm.kmask[st]);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 k4 = ks4[i];
-                x[4 * i + 0] = k4.x != 0.f ? __uint_as_float(sv[4 * i + 0]) * k4.x : kNegInf;
-                x[4 * i + 1] = k4.y != 0.f ? __uint_as_float(sv[4 * i + 1]) * k4.y : kNegInf;
-                x[4 * i + 2] = k4.z != 0.f ? __uint_as_float(sv[4 * i + 2]) * k4.z : kNegInf;
-                x[4 * i + 3] = k4.w != 0.f ? __uint_as_float(sv[4 * i + 3]) * k4.w : kNegInf;
+            for (int i = 0; i < 8; ++i) {                // scaled score, or -inf for a masked row
+                const float4 k4 = ks4[i], m4 = km4[i];
+                x[4 * i + 0] = fmaf(__uint_as_float(sv[4 * i + 0]), k4.x, m4.x);
+                x[4 * i + 1] = fmaf(__uint_as_float(sv[4 * i + 1]), k4.y, m4.y);
+                x[4 * i + 2] = fmaf(__uint_as_float(sv[4 * i + 2]), k4.z, m4.z);
+                x[4 * i + 3] = fmaf(__uint_as_float(sv[4 * i + 3]), k4.w, m4.w);
             }
             float mx[16];
 #pragma unroll
@@ -347,14 +348,19 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1) sparse
                 for (int i = 0; i < w; ++i) ps[i] += ps[i + w];
             l_run += ps[0];
             uint32_t pw[16];
-            const float4* vs4 = reinterpret_cast<const float4*>(sm.vscale[st]);
+            if constexpr (KV_FP8) {                      // the row's FP8 scale goes into P
+                const float4* vs4 = reinterpret_cast<const float4*>(sm.vscale[st]);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 v4 = vs4[i];
-                pw[2 * i] = pack_bf16x2(p[4 * i] * v4.x, p[4 * i + 1] * v4.y);
-                pw[2 * i + 1] = pack_bf16x2(p[4 * i + 2] * v4.z, p[4 * i + 3] * v4.w);
+                for (int i = 0; i < 8; ++i) {
+                    const float4 v4 = vs4[i];
+                    pw[2 * i] = pack_bf16x2(p[4 * i] * v4.x, p[4 * i + 1] * v4.y);
+                    pw[2 * i + 1] = pack_bf16x2(p[4 * i + 2] * v4.z, p[4 * i + 3] * v4.w);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pw[i] = pack_bf16x2(p[2 * i], p[2 * i + 1]);
             }
-            tc::tmem_st16(p_col + sb * 16 + lane_off, pw);
+            tc::tmem_st16(s_col + sb * 32 + lane_off, pw);           // P over the S it came from
             if (__any_sync(0xffffffffu, rescale)) {
                 // O must hold P V_{j-1} before it is rescaled.
                 if (j >= 1 && !tc::mbar_wait(&sm.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
