@@ -524,23 +524,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
     }
 }
 
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-    static EncodeTiled fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(p);
-    });
-    return fn;
-}
-
 int num_sms() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -567,6 +550,23 @@ int group_size(const IndexArgs& a, int H_I) {
 
 }  // namespace
 
+namespace tc {
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+}  // namespace tc
+
 bool index_score_tc_supported(const IndexArgs& a, int H_I, int D_I, bool fp8) {
     if (!fp8 || D_I != 128 || H_I % 32 != 0 || H_I > 128) return false;
     if (a.cand && a.block_size != 64) return false;
@@ -574,7 +574,7 @@ bool index_score_tc_supported(const IndexArgs& a, int H_I, int D_I, bool fp8) {
     const int N = group_size(a, H_I) * H_I;
     if (N != 32 && N != 64 && N != 128 && N != 256) return false;
     return ((uintptr_t)a.kdata % 16 == 0) && (a.tok_stride_b % 16 == 0) && (a.seq_stride_b % 16 == 0) &&
-           a.kscale != nullptr && encode_fn() != nullptr;
+           a.kscale != nullptr && tc::encode_tiled() != nullptr;
 }
 
 cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st) {
@@ -590,7 +590,7 @@ cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st) {
     const cuuint64_t strides[2] = {(cuuint64_t)a.tok_stride_b, (cuuint64_t)a.seq_stride_b};
     const cuuint32_t box[3] = {128, 64, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(a.kdata), dims, strides, box,
+    CUresult r = tc::encode_tiled()(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(a.kdata), dims, strides, box,
                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
@@ -604,7 +604,7 @@ cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st) {
         const cuuint64_t sstr[1] = {(cuuint64_t)a.scale_seq_stride * 4};
         const cuuint32_t sbox[2] = {64, 1};
         const cuuint32_t sestr[2] = {1, 1};
-        r = encode_fn()(&sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(a.kscale), sdims, sstr, sbox, sestr,
+        r = tc::encode_tiled()(&sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(a.kscale), sdims, sstr, sbox, sestr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) { pa.scale_tma = 0; memset(&sc, 0, sizeof(sc)); }

@@ -252,6 +252,57 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src,
                  :: "r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(bar) : "memory");
 }
 
+// TMA gather of four rows (tile::gather4, 2-D tensor map whose box is one row high): rows r0..r3
+// of columns [x, x + box width) land as four consecutive box rows at dst, with the map's
+// swizzle applied by shared-memory address; the bytes complete on bar.  x times the element
+// size must be a multiple of 16 bytes; a row outside the tensor reads as zeros.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int r0, int r1,
+                                            int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+           "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Arrives (release, cluster scope) on the mbarrier at shared::cluster address bar of a peer CTA.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+
+// As mbar_arrive_remote without release semantics: orders none of this thread's earlier memory
+// accesses, so the caller must already know that the accesses it signals the end of are complete.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+
+// 16-byte store to shared::cluster address dst (a peer CTA's shared memory).
+__device__ __forceinline__ void st_cluster_v4(uint32_t dst, uint4 v) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(dst), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// mbar_wait with acquire at cluster scope, for phases completed by a peer CTA's remote arrivals
+// (the peer's stores before its release-arrive are visible afterwards).  Bounded as mbar_wait.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > kWaitNs) { *abort = 1; return false; }
+    }
+}
+
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -262,6 +313,12 @@ __device__ __forceinline__ bool elect_one() {
                  : "=r"(pred) : "r"(0xffffffffu));
     return pred != 0;
 }
+
+// Host: the driver's cuTensorMapEncodeTiled (resolved once), or nullptr when unavailable.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled();
 
 }  // namespace tc
 }  // namespace lsa
