@@ -15,26 +15,36 @@
 //
 // Memory plan.  TMEM (512 columns): O half [0,256), three S / P buffers [256,352) -- the
 // softmax writes P (BF16) over the S it has just read, so S can run two tiles ahead of P V --
-// and the query slice Q[:, D_h] [352,496) as the A operand of S.  Shared memory: a 7-stage
-// ring of 32-row KV tiles (5 swizzled 64-dim K atoms, the last half used, 20 KB), read as the
-// B operand of S (K-major) and of P V (MN-major); two 16 KB staging buffers for this CTA's
-// partial S and two that receive the peer's.
+// and the query slice Q[:, D_h] [352,496) as the A operand of S.  Shared memory: an 8-stage
+// ring of 32-row KV tiles, read as the B operand of S (K-major) and of P V (MN-major): each
+// stage has its 4 swizzled 64-dim V-half atoms (16 KB), and two stages share one 64-dim rope
+// atom, each in the half of its 128-byte rows that the other leaves (only 32 rope dims are this
+// CTA's); two 16 KB staging buffers for this CTA's partial S and two that receive the peer's.
 //
-//   warps 0..6 : gather -- warp s fills stage s with the tiles j = s, s + 7, ...: the rows'
-//                indices (prefetched one tile ahead), per-row scale and validity to shared
-//                memory, then the CTA's 288 dims of each row with 16-byte cp.async (FP8 rows
-//                are widened to BF16 exactly on the way).
-//   warp 7     : MMA issuer -- S_j (18 TS MMAs, N = 32) once tile j has landed and P V_{j-3}
-//                has been issued; O += P_j V_j (2 TS MMAs, N = 256) once the softmax of tile
-//                j is done; whichever is ready, each kind in order.
-//   warps 8..11: softmax -- thread = head (TMEM lane).  Each warp exchanges its 32 heads'
-//                rows on its own: it stages its partial S of tile j + 1 in shared memory and
-//                one lane pushes the 4 KB to the peer with a bulk shared-to-shared copy that
-//                completes on the peer's barrier (so the exchange runs under the softmax of
-//                tile j); then it adds the peer's partial of tile j to its own, runs the
-//                online max / sum with lazy rescaling of O (only when the running max grows
-//                by more than 2^8; warp-uniform, so deterministic) and writes P to TMEM as
-//                BF16; finally O / l and lse.
+// Warp roles (512 threads).  With BF16 rows:
+//   warps 0,2,3: gather -- tile j by the (j mod 3)-th: the rows' indices (prefetched three tiles
+//                of the warp ahead) and validity to shared memory, then the V-half atoms with
+//                tile::gather4 (4 rows x 64 dims per load) and the 4 rope chunks of each row with
+//                16-byte cp.async; both complete on the tile's barrier by themselves, so the warp
+//                moves on at once.  (Without a tensor map for the cache, cp.async does it all.)
+//   warp 1     : MMA issuer -- S_j (18 TS MMAs, N = 32) once tile j has landed, P V_{j-3} has
+//                been issued and S_{j-3} has been sent; O += P_j V_j (2 TS MMAs, N = 256) once
+//                the softmax of tile j is done; whichever is ready, each kind in order.
+//   warps 4..7 : send -- warp q (mod 4) stages heads [32q, 32q + 32) of each partial S in shared
+//                memory and pushes the 4 KB to the peer with one bulk shared-to-shared copy that
+//                completes on the peer's barrier, as soon as the MMA has produced it.
+//   warps 8..15: softmax -- two warpgroups taking alternate tiles; thread = head (TMEM lane).
+//                Each adds the peer's partial of its tile to its own, then runs the online
+//                softmax with lazy rescaling: the reference max is raised only when a tile's
+//                max exceeds it by more than 2^8 (warp-uniform, so deterministic).  These
+//                decisions form one chain over the tiles, handed from one warpgroup to the
+//                other through shared memory, so that only the compare runs in tile order and
+//                the exponentials of two tiles overlap; the warpgroup that raises the max
+//                rescales O.  P goes to TMEM as BF16; finally O / l and lse, half the columns
+//                each.
+// With FP8 rows warps 0..6 gather (tile j by warp j mod 7; the codes are loaded and widened to
+// BF16 exactly on the way), warp 7 issues the MMAs, warps 8..11 are a single softmax warpgroup
+// and warps 12..15 send.
 //
 // All waits are bounded (2 s); a CTA that gives up reports LSA_ERR_TIMEOUT.
 #include <cstring>
@@ -48,19 +58,20 @@ namespace {
 
 constexpr int kAThreads = 512;
 constexpr int kRows = 32;                    // KV rows per tile
-constexpr int kStagesA = 7;                  // KV tile ring (one gather warp per stage)
+constexpr int kStagesA = 8;                  // KV tile ring
 constexpr int kXB = 2;                       // partial-S exchange buffers (staging and receive)
 constexpr int kSP = 3;                       // S / P buffers in TMEM (P overwrites its own S)
 constexpr int kD = 576, kDv = 512, kHalf = 256;
-constexpr int kAtomsA = 5;                   // K atoms of a CTA's slice: 4 V atoms + half a rope atom
 constexpr int kKSteps = 4 * 4 + 2;           // 16-dim K steps of S per CTA (288 dims)
 constexpr int kQCols = kKSteps * 8;          // TMEM columns of the query slice (144)
-constexpr int kTileBytes = kAtomsA * kRows * 128;         // 20 KB
+constexpr int kVBytes = 4 * kRows * 128;                  // a tile's 4 V-half atoms, 16 KB
+constexpr int kRopeBytes = kRows * 128;                   // one rope atom, shared by two stages
 static_assert(256 + kSP * 32 + kQCols <= 512, "TMEM columns: O half, S / P buffers, query slice");
 constexpr int kXBytes = 128 * kRows * 4;                  // one partial S: 128 heads x 32 rows FP32
 
 struct AttnSmem {
-    alignas(1024) uint8_t kv[kStagesA][kTileBytes];
+    alignas(1024) uint8_t kv[kStagesA][kVBytes];       // V-half atoms of each stage
+    alignas(1024) uint8_t rope[kStagesA / 2][kRopeBytes];  // stage s: atom s / 2, chunk half (CTA half) ^ (s & 1)
     // Partial S exchange, per buffer [head][16-byte chunk ^ (head & 7)]; softmax warp q owns the
     // 4 KB of heads [32q, 32q + 32) in each.
     alignas(1024) uint8_t xs[kXB][kXBytes];      // the peer's partial S
@@ -69,8 +80,11 @@ struct AttnSmem {
     alignas(16) float kmask[kStagesA][kRows];    // 0, or -inf for masked rows (added to the scaled score)
     alignas(16) float vscale[kStagesA][kRows];   // per-row FP8 scale (1 for BF16)
     int rows[kStagesA][kRows];
-    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[kSP], p_full[kSP], o_done[2], q_ready;
+    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[kSP], p_full[kSP], o_done[2], q_ready, q_tma;
     uint64_t s_sent[kSP];                        // the send warps have read S out of this buffer
+    uint64_t hand[2][4];                         // softmax warpgroup w, quarter q: m_ref of its tile is out
+    float m_ref[128];                            // the reference max after the latest decided tile
+    float2 ml[2][128];                           // each softmax warpgroup's final (max, sum)
     uint64_t rx_full[kXB][4];                    // a quarter of the peer's partial S has arrived (4 KB tx)
     uint64_t tx_free[kXB][4];                    // the peer has read the quarter this CTA sent into buffer x
     uint32_t tmem_base;
@@ -83,19 +97,25 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Global dim offset (in elements) of 16-byte chunk c8 of local atom la in CTA `half`'s slice.
-// Atom 4 is the 64-dim rope atom at its natural position: CTA h uses chunks [4h, 4h + 4).
-__device__ __forceinline__ int slice_dim(int half, int la, int c8) {
-    return la < 4 ? half * kHalf + la * 64 + c8 * 8 : kDv + c8 * 8;
+// Named barrier `id` over `count` threads (whole warps).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(count) : "memory");
 }
 
 // KV_FP8: e4m3 rows with a per-row scale, widened to BF16 in shared memory by the gather warps.
-// TMA (BF16 rows only): the gather warps issue tile::gather4 loads through `kvmap` (a 2-D map
-// over all rows of the cache, box 64 dims x 1 row, 128-byte swizzle) instead of cp.async.
+// BF16 rows are copied as they are by three warps without waiting: the V-half atoms with TMA
+// tile::gather4 through `kvmap` (a 2-D map over all rows of the cache, box 64 dims x 1 row,
+// 128-byte swizzle) when TMA is set, else with cp.async; the rope chunks with cp.async.  Both
+// complete on the tile's barrier by themselves.
+// `qmap`: the queries as a 2-D tensor [T * 128 heads][576 dims], box 64 dims x 128 heads,
+// 128-byte swizzle.
 template <bool KV_FP8, bool TMA>
 __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
-    sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, AttnArgs a) {
+    sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
+                          AttnArgs a) {
     static_assert(!(KV_FP8 && TMA), "TMA gathers BF16 rows only");
+    constexpr bool kAsync = !KV_FP8;             // gather by 3 warps that do not wait for their copies
+    constexpr int kSmx = kAsync ? 2 : 1;         // softmax warpgroups
     extern __shared__ uint8_t smem_raw[];
     AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int split = blockIdx.x, half = blockIdx.y, t = blockIdx.z;
@@ -118,9 +138,10 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
     const float* kvs = KV_FP8 ? a.kv_scale + (size_t)max(b, 0) * a.kv_scale_seq : nullptr;
     const uint16_t* qt = a.q + (size_t)t * 128 * kD;
 
+    auto q_atom = [&](int at) -> uint8_t* { return at < 2 ? sm.xs[at] : (at < 4 ? sm.stg[at - 2] : sm.kv[7]); };
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStagesA; ++i) {
-            tc::mbar_init(&sm.kv_full[i], TMA ? 1 : 32);   // TMA: one expect_tx arrival + the bytes
+            tc::mbar_init(&sm.kv_full[i], kAsync ? 33 : 32);   // async: 32 copy completions + 1 (scales)
             tc::mbar_init(&sm.kv_empty[i], 1);
         }
         for (int i = 0; i < kSP; ++i) {
@@ -134,63 +155,82 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                 tc::mbar_init(&sm.tx_free[x][q], 1);     // one remote arrival from the peer's warp q
             }
         for (int i = 0; i < 2; ++i) tc::mbar_init(&sm.o_done[i], 1);
-        tc::mbar_init(&sm.q_ready, 128);
+        for (int w = 0; w < 2; ++w)
+            for (int q = 0; q < 4; ++q) tc::mbar_init(&sm.hand[w][q], 1);
+        tc::mbar_init(&sm.q_ready, kSmx * 128);
+        tc::mbar_init(&sm.q_tma, 1);
         sm.abort = 0;
         tc::fence_barrier_init();
+        // Q[:, V half] as 4 swizzled 64-dim atoms into the exchange buffers and its rope atom into
+        // KV stage 7, all idle until the softmax warps have moved Q to TMEM.
+        tc::prefetch_tmap(&qmap);
+        tc::mbar_expect_tx(&sm.q_tma, 5 * 128 * 128);
+        for (int at = 0; at < 5; ++at)
+            tc::tma_load_2d(q_atom(at), &qmap, &sm.q_tma, at < 4 ? half * kHalf + at * 64 : kDv, t * 128);
     }
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
     tc::tc_fence_before();
     __syncthreads();
-    tc::cluster_sync_all();                      // the peer's barriers exist before any cross-CTA traffic
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t o_col = tmem, s_col = tmem + 256, qt_col = tmem + 256 + kSP * 32;   // O, S / P, Q slice
 
-    // The softmax warps load the query slice Q[:, D_h] into TMEM (thread = head = lane) while the
-    // gather warps already fetch KV tiles.  Column c of the slice holds dims (2c, 2c + 1) of
-    // [256h, 256h + 256) for c < 128, then of the rope dims [512 + 32h, 512 + 32h + 32).
-    if (warp >= 8 && warp < 12) {
+    // Warp roles.  BF16 rows: warps 0, 2, 3 gather (tile j by the (j mod 3)-th), warp 1 issues the
+    // MMAs, warps 4..7 send the partial S, and warps 8..11 and 12..15 are two softmax warpgroups
+    // taking alternate tiles.  FP8 rows: warps 0..6 gather (warp s owns stage s), warp 7 issues
+    // the MMAs, warps 8..11 are the softmax warpgroup and warps 12..15 send.
+    constexpr int kGatherFp8 = 7;                // FP8 gather warps 0..6
+    const int mma_warp = kAsync ? 1 : kGatherFp8;
+    const bool send_warp = kAsync ? (warp >= 4 && warp < 8) : warp >= 12;
+    const int wg = warp >= 8 ? (warp - 8) >> 2 : -1;                // softmax warpgroup
+    const bool smx_warp = wg >= 0 && wg < kSmx;
+
+    // The softmax warps move the query slice Q[:, D_h] into TMEM (thread = head = lane; with two
+    // warpgroups each takes half the columns) while the gather warps already fetch KV tiles:
+    // column c holds dims (2c, 2c + 1) of [256 half, 256 half + 256) for c < 128, then of the rope
+    // dims [512 + 32 half, 512 + 32 half + 32), read from the staged atoms.
+    // Every thread arrives on the cluster barrier once its CTA's barriers exist -- the softmax
+    // warps only after their reads of the exchange buffers, so no copy from the peer lands there
+    // before.
+    if (smx_warp) {
         const int h = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint4* src = reinterpret_cast<const uint4*>(qt + (size_t)h * kD + half * kHalf);
-        const uint4* rope = reinterpret_cast<const uint4*>(qt + (size_t)h * kD + kDv + half * 32);
-        uint4 cur[8], nxt[8];
+        const bool got = tc::mbar_wait(&sm.q_tma, 0, abort_flag);
+        const int at0 = kSmx == 2 ? 2 * wg : 0, at1 = kSmx == 2 ? at0 + 2 : 4;
+        for (int at = at0; at < at1; ++at) {
+            const uint8_t* row = q_atom(at) + h * 128;
+            uint32_t w[32];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) cur[u] = src[u];
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {                // 4 groups of 64 dims = 32 columns
-            if (c + 1 < 4) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) nxt[u] = src[(c + 1) * 8 + u];
-            } else {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) nxt[u] = rope[u];
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = got ? *reinterpret_cast<const uint4*>(row + ((c ^ (h & 7)) << 4)) : make_uint4(0, 0, 0, 0);
+                w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
             }
-            uint32_t v[32];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                v[4 * u] = cur[u].x; v[4 * u + 1] = cur[u].y; v[4 * u + 2] = cur[u].z; v[4 * u + 3] = cur[u].w;
-            }
-            tc::tmem_st32(qt_col + c * 32 + lane_off, v);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) cur[u] = nxt[u];
+            tc::tmem_st32(qt_col + at * 32 + lane_off, w);
         }
-        {
-            uint32_t v[16];
+        if (kSmx == 1 || wg == 1) {                  // this CTA's rope chunks: 4 half .. 4 half + 3
+            const uint8_t* row = q_atom(4) + h * 128;
+            uint32_t w[16];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                v[4 * u] = cur[u].x; v[4 * u + 1] = cur[u].y; v[4 * u + 2] = cur[u].z; v[4 * u + 3] = cur[u].w;
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = got ? *reinterpret_cast<const uint4*>(row + (((4 * half + c) ^ (h & 7)) << 4))
+                                    : make_uint4(0, 0, 0, 0);
+                w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
             }
-            tc::tmem_st16(qt_col + 128 + lane_off, v);
+            tc::tmem_st16(qt_col + 128 + lane_off, w);
         }
         tc::tmem_wait_st();
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.q_ready);
     }
+    tc::cluster_arrive();
+    // Warps that touch the peer's shared memory wait for its barriers to exist; the others only
+    // before leaving.
+    const bool remote_warp = send_warp || smx_warp;
+    if (remote_warp) tc::cluster_wait();
 
-    if (warp < kStagesA) {
-        // ---------------- gather producers: warp s owns stage s and the tiles j = s, s + 7, ...
-        const int g = warp;
+    if (kAsync ? (warp == 0 || warp == 2 || warp == 3) : warp < kGatherFp8) {
+        // ---------------- gather producers: tiles j = first, first + step, ... into stage j % 7
+        const int first = kAsync ? (warp == 0 ? 0 : warp - 1) : warp, step = kAsync ? 3 : kGatherFp8;
         auto fetch_row = [&](int j) -> int {                       // lane l: index of row l of tile j
             if (j >= n_tiles) return -1;
             const int r0 = r_beg + j * kRows;
@@ -200,11 +240,17 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
         // Row coordinate of this sequence's row 0 in the map (TMA): the cache is B sequences of
         // kv_seq_b / kv_tok_b rows.
         const int row0 = TMA ? (int)((int64_t)max(b, 0) * (a.kv_seq_b / a.kv_tok_b)) : 0;
-        int nxt = fetch_row(g);
-        for (int j = g; j < n_tiles; j += kStagesA) {
-            const int cur = nxt;
-            nxt = fetch_row(j + kStagesA);                         // prefetch this warp's next tile
+        // The row indices run three of this warp's tiles ahead (the warp does not wait for its
+        // copies, so one tile ahead would leave the index load's latency exposed).
+        int nxt1 = fetch_row(first), nxt2 = fetch_row(first + step), nxt3 = fetch_row(first + 2 * step);
+        for (int j = first; j < n_tiles; j += step) {
+            const int cur = nxt1, g = j % kStagesA;
+            nxt1 = nxt2;
+            nxt2 = nxt3;
+            nxt3 = fetch_row(j + 3 * step);
             if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.kv_empty[g], ((j / kStagesA) + 1) & 1, abort_flag))) break;
+            // Stage 7 holds the query's rope atom until the softmax warps have read it.
+            if (j == 7 && !__all_sync(0xffffffffu, tc::mbar_wait(&sm.q_ready, 0, abort_flag))) break;
             const int nr = min(kRows, r_end - (r_beg + j * kRows));
             {
                 const bool v = cur >= 0 && cur < len;
@@ -216,36 +262,54 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                 sm.kmask[g][lane] = v ? 0.f : kNegInf;
             }
             __syncwarp();
-            uint8_t* tile = sm.kv[g];
-            if constexpr (TMA) {
-                // 8 groups of 4 rows x 5 atoms (the V half and the whole rope atom), 512 B each;
-                // a masked row reads as zeros (coordinate -1 is outside the map).
-                const int grow = (cur >= 0 && cur < len) ? row0 + cur : -1;
-                int rr[4];
+            // Destination of 16-byte chunk c8 of local atom la (4 = rope) of tile row r.
+            const int rh = half ^ (g & 1);                         // rope chunk half of this stage
+            auto dst_of = [&](int la, int r, int c8) -> uint8_t* {
+                return (la < 4 ? sm.kv[g] + la * (kRows * 128) : sm.rope[g >> 1]) + r * 128 + ((c8 ^ (r & 7)) << 4);
+            };
+            if constexpr (!KV_FP8) {
+                // A masked row reads as zeros.  Each lane's cp.async arrive on the barrier when
+                // they complete (32 of its 33 arrivals); the 33rd is lane 0's, after the scales.
+                if constexpr (TMA) {
+                    // V half: 8 groups of 4 rows x 4 atoms, 512 B per tile::gather4 (coordinate
+                    // -1 is outside the map).
+                    const int grow = (cur >= 0 && cur < len) ? row0 + cur : -1;
+                    int rr[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) rr[i] = __shfl_sync(0xffffffffu, grow, ((lane & 7) << 2) + i);
-                if (lane == 0) tc::mbar_expect_tx(&sm.kv_full[g], kTileBytes);
-                __syncwarp();
-                if (lane < 8) {
+                    for (int i = 0; i < 4; ++i) rr[i] = __shfl_sync(0xffffffffu, grow, ((lane & 7) << 2) + i);
+                    if (lane == 0) tc::mbar_expect_tx(&sm.kv_full[g], kVBytes);
+                    __syncwarp();
+                    if (lane < 8) {
 #pragma unroll
-                    for (int la = 0; la < kAtomsA; ++la)
-                        tc::tma_gather4(tile + la * (kRows * 128) + lane * 512, &kvmap, &sm.kv_full[g],
-                                        la < 4 ? half * kHalf + la * 64 : kDv, rr[0], rr[1], rr[2], rr[3]);
+                        for (int la = 0; la < 4; ++la)
+                            tc::tma_gather4(sm.kv[g] + la * (kRows * 128) + lane * 512, &kvmap, &sm.kv_full[g],
+                                            half * kHalf + la * 64, rr[0], rr[1], rr[2], rr[3]);
+                    }
+                    // Rope: 4 chunks per row.
+#pragma unroll
+                    for (int i = lane; i < kRows * 4; i += 32) {
+                        const int r = i >> 2, c = i & 3;
+                        const int row = sm.rows[g][r];
+                        cp_async16(dst_of(4, r, 4 * rh + c),
+                                   kvb + (size_t)(row >= 0 ? row : 0) * a.kv_tok_b + (kDv + 32 * half + 8 * c) * 2, row >= 0);
+                    }
+                    cp_async_mbar_arrive_noinc(&sm.kv_full[g]);
+                } else {
+                    // 36 chunks of 16 bytes per row: 32 of the V half (4 atoms x 8), 4 rope chunks.
+#pragma unroll 4
+                    for (int i = lane; i < kRows * 36; i += 32) {
+                        const int r = i / 36, q = i % 36;
+                        const int la = q < 32 ? q >> 3 : 4, c = q < 32 ? q & 7 : q - 32;
+                        const int row = sm.rows[g][r];
+                        const int dim = la < 4 ? half * kHalf + la * 64 + c * 8 : kDv + 32 * half + 8 * c;
+                        cp_async16(dst_of(la, r, la < 4 ? c : 4 * rh + c),
+                                   kvb + (size_t)(row >= 0 ? row : 0) * a.kv_tok_b + dim * 2, row >= 0);
+                    }
+                    cp_async_mbar_arrive_noinc(&sm.kv_full[g]);
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sm.kv_full[g]);
                 }
                 continue;
-            } else if (!KV_FP8) {
-                // 36 chunks of 16 bytes per row: 32 of the V half (4 atoms x 8), 4 rope chunks.
-#pragma unroll 4
-                for (int i = lane; i < kRows * 36; i += 32) {
-                    const int r = i / 36, q = i % 36;
-                    const int la = q < 32 ? q >> 3 : 4, c8 = q < 32 ? q & 7 : 4 * half + q - 32;
-                    const int row = sm.rows[g][r];
-                    uint8_t* dst = tile + la * (kRows * 128) + r * 128 + ((c8 ^ (r & 7)) << 4);
-                    cp_async16(dst, kvb + (size_t)(row >= 0 ? row : 0) * a.kv_tok_b + slice_dim(half, la, c8) * 2,
-                               row >= 0);
-                }
-                cp_async_commit();
-                cp_async_wait<0>();
             } else {
                 // 18 chunks of 16 codes per row (16 of the V half, 2 rope), each widened to two
                 // BF16 chunks.
@@ -269,7 +333,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                         const int i = i0 + u * 32;
                         if (i >= kChunks) break;
                         const int r = i / 18, q = i % 18;
-                        const int la = q < 16 ? q >> 2 : 4, cb0 = q < 16 ? (q & 3) * 2 : 4 * half + (q - 16) * 2;
+                        const int la = q < 16 ? q >> 2 : 4, cb0 = q < 16 ? (q & 3) * 2 : 4 * rh + (q - 16) * 2;
                         const uint32_t* wd = reinterpret_cast<const uint32_t*>(&raw[u]);
                         uint32_t ow[8];
 #pragma unroll
@@ -280,7 +344,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int c8 = cb0 + hh;
-                            uint8_t* dst = tile + la * (kRows * 128) + r * 128 + ((c8 ^ (r & 7)) << 4);
+                            uint8_t* dst = dst_of(la, r, c8);
                             *reinterpret_cast<uint4*>(dst) =
                                 make_uint4(ow[4 * hh], ow[4 * hh + 1], ow[4 * hh + 2], ow[4 * hh + 3]);
                         }
@@ -290,16 +354,8 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(&sm.kv_full[g]);
         }
-        if constexpr (TMA) {
-            // A CTA that gave up may still have gathers in flight into its shared memory: wait
-            // (bounded) for this warp's last tile to land before the CTA can exit.
-            const int last = g < n_tiles ? g + ((n_tiles - 1 - g) / kStagesA) * kStagesA : -1;
-            if (last >= 0 && lane == 0 && *abort_flag) {
-                volatile int drain_abort = 0;
-                tc::mbar_wait(&sm.kv_full[g], (last / kStagesA) & 1, &drain_abort);
-            }
-        }
-    } else if (warp == kStagesA) {
+        if constexpr (kAsync) cp_async_wait_all();     // no copy outlives the CTA
+    } else if (warp == mma_warp) {
         // ---------------- MMA issuer: S_j and P_j V_j, each in order, whichever is ready
         const uint32_t idesc_s = tc::idesc_f16(128, kRows, 1);
         const uint32_t idesc_o = tc::idesc_f16_bmn(128, kHalf, 1);
@@ -316,12 +372,16 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                     (ns < kSP || tc::mbar_test_wait(&sm.s_sent[ns % kSP], ((ns / kSP) - 1) & 1)) &&
                     tc::mbar_try_wait(&sm.kv_full[ns % kStagesA], (ns / kStagesA) & 1)) {
                     tc::tc_fence_after();
+                    tc::fence_proxy_async_smem();    // the tile's cp.async writes, for the tensor cores
                     const int sb = ns % kSP;
-                    const uint32_t kaddr = tc::smem_u32(sm.kv[ns % kStagesA]);
+                    const int st = ns % kStagesA;
+                    const uint32_t kaddr = tc::smem_u32(sm.kv[st]), raddr = tc::smem_u32(sm.rope[st >> 1]);
+                    const int rh = half ^ (st & 1);
 #pragma unroll
                     for (int kk = 0; kk < kKSteps; ++kk) {
-                        const int la = kk < 16 ? kk >> 2 : 4, ks = kk < 16 ? kk & 3 : 2 * half + kk - 16;
-                        const uint64_t bd = tc::sdesc_sw128(kaddr + la * (kRows * 128) + ks * 32);
+                        const uint32_t aaddr = kk < 16 ? kaddr + (kk >> 2) * (kRows * 128) + (kk & 3) * 32
+                                                       : raddr + (2 * rh + kk - 16) * 32;
+                        const uint64_t bd = tc::sdesc_sw128(aaddr);
                         tc::mma_f16_ts(s_col + sb * 32, qt_col + kk * 8, bd, idesc_s, kk > 0);
                     }
                     tc::mma_commit(&sm.s_full[sb]);
@@ -352,17 +412,18 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                 tc::mbar_wait(&sm.o_done[(npv - 1) & 1], ((npv - 1) >> 1) & 1, &drain_abort);
             }
         }
-    } else if (warp >= 8 && warp < 12) {
-        // ---------------- softmax / epilogue: thread = head = TMEM lane
+    } else if (smx_warp) {
+        // ---------------- softmax / epilogue: thread = head = TMEM lane; warpgroup wg takes the
+        // tiles j = wg, wg + kSmx, ...
         const int quarter = warp & 3;
         const int h = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int xoff = lane * 128;                 // this head's row within a quarter
-        float m_run = kNegInf, l_run = 0.f;
+        float m_w = kNegInf, l_w = 0.f;              // reference max this warpgroup last used, its sum
         bool alive = true;
-        if (lane == 0)                               // the first two tiles' partials may arrive at once
-            for (int x = 0; x < kXB && x < n_tiles; ++x) tc::mbar_expect_tx(&sm.rx_full[x][quarter], 4096);
-        for (int j = 0; j < n_tiles; ++j) {
+        if (lane == 0)                               // the first partials may arrive at once
+            for (int x = wg; x < kXB && x < n_tiles; x += kSmx) tc::mbar_expect_tx(&sm.rx_full[x][quarter], 4096);
+        for (int j = wg; j < n_tiles; j += kSmx) {
             const int sb = j % kSP, st = j % kStagesA, xb = j % kXB;
             if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.s_full[sb], (j / kSP) & 1, abort_flag))) {
                 alive = false;
@@ -412,14 +473,38 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
 #pragma unroll
                 for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
             const float mt = mx[0];
-            float alpha = 1.f;
-            bool rescale = false;
-            if (mt > m_run + 8.f) {
-                if (m_run != kNegInf) { alpha = ex2(m_run - mt); rescale = true; }
-                l_run *= alpha;
-                m_run = mt;
+            // The reference max is raised to the tile max only when that exceeds it by more than
+            // 2^8 (lazy rescaling).  With two warpgroups the decisions form one chain over the
+            // tiles: tile j's starts from tile j-1's, handed over through shared memory.
+            float m_prev = m_w;
+            if constexpr (kSmx == 2) {
+                if (j > 0) {
+                    if (!__all_sync(0xffffffffu,
+                                    tc::mbar_wait(&sm.hand[wg ^ 1][quarter], ((j - 1) >> 1) & 1, abort_flag))) {
+                        alive = false;
+                        break;
+                    }
+                    m_prev = sm.m_ref[h];
+                }
             }
-            const float mref = m_run == kNegInf ? 0.f : m_run;            // all rows masked so far: p = 0
+            float m_new = m_prev, alpha = 1.f;
+            bool rescale = false;
+            if (mt > m_prev + 8.f) {
+                if (m_prev != kNegInf) { alpha = ex2(m_prev - mt); rescale = true; }
+                m_new = mt;
+            }
+            if constexpr (kSmx == 2) {
+                if (j + 1 < n_tiles) {
+                    sm.m_ref[h] = m_new;
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sm.hand[wg][quarter]);
+                }
+            }
+            if (m_new != m_w) {                          // bring this warpgroup's sum to the new max
+                l_w = m_w == kNegInf ? 0.f : l_w * ex2(m_w - m_new);
+                m_w = m_new;
+            }
+            const float mref = m_w == kNegInf ? 0.f : m_w;                // all rows masked so far: p = 0
             float p[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) p[i] = ex2(x[i] - mref);         // ex2(-inf) = 0
@@ -430,7 +515,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             for (int w = 8; w >= 1; w >>= 1)
 #pragma unroll
                 for (int i = 0; i < w; ++i) ps[i] += ps[i + w];
-            l_run += ps[0];
+            l_w += ps[0];
             uint32_t pw[16];
             if constexpr (KV_FP8) {                      // the row's FP8 scale goes into P
                 const float4* vs4 = reinterpret_cast<const float4*>(sm.vscale[st]);
@@ -477,16 +562,33 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.p_full[sb]);
         }
-        // Epilogue: O / l, lse.
+        // Epilogue: O / l and lse.  The two warpgroups' sums are brought to the final reference max
+        // (the larger of their last ones) and added; warpgroup w writes O columns [128w, 128w + 128).
+        float m_f = m_w, l_f = l_w;
+        if constexpr (kSmx == 2) {
+            sm.ml[wg][h] = make_float2(m_w, l_w);
+            // One barrier over both warpgroups.  (Per-quarter barriers over the two warps of a
+            // lane quarter, 64 threads each, let a warp read the other's pair before it was written
+            // in a fraction of launches.)
+            named_bar_sync(6, 2 * 128);
+            const float2 o = sm.ml[wg ^ 1][h];
+            m_f = fmaxf(m_w, o.x);
+            l_f = (m_w == kNegInf ? 0.f : l_w * ex2(m_w - m_f)) + (o.x == kNegInf ? 0.f : o.y * ex2(o.x - m_f));
+        }
         if (alive && n_tiles > 0 &&
             !__all_sync(0xffffffffu, tc::mbar_wait(&sm.o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag)))
             alive = false;
         tc::tc_fence_after();
         const float kLn2 = 0.69314718055994530942f;
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        const float lse = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : kNegInf;
-        const int dv0 = half * kHalf;
-        for (int c = 0; c < kHalf / 32; ++c) {
+        const float inv = l_f > 0.f ? 1.f / l_f : 0.f;
+        const float lse = l_f > 0.f ? (m_f + log2f(l_f)) * kLn2 : kNegInf;
+        // The rows go out through shared memory (the idle KV ring; rows padded by 16 B so that
+        // consecutive heads fall in different banks), one bulk copy per head row.
+        const bool bf16_out = a.n_split == 1;
+        const int row_bytes = bf16_out ? kHalf * 2 : kHalf * 4, pitch = row_bytes + 16;
+        uint8_t* srow = sm.kv[0] + h * pitch;
+        const int c_beg = kSmx == 2 ? wg * (kHalf / 64) : 0, c_end = kSmx == 2 ? c_beg + kHalf / 64 : kHalf / 32;
+        for (int c = c_beg; c < c_end; ++c) {
             uint32_t ov[32];
             if (n_tiles > 0 && alive) {
                 tc::tmem_ld32(o_col + c * 32 + lane_off, ov);
@@ -495,8 +597,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ov[i] = 0u;
             }
-            if (a.n_split == 1) {
-                uint16_t* orow = a.o + ((size_t)t * 128 + h) * kDv + dv0 + c * 32;
+            if (bf16_out) {
 #pragma unroll
                 for (int i = 0; i < 32; i += 8) {
                     uint4 pk;
@@ -504,23 +605,32 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                     pk.y = pack_bf16x2(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv);
                     pk.z = pack_bf16x2(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv);
                     pk.w = pack_bf16x2(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv);
-                    *reinterpret_cast<uint4*>(orow + i) = pk;
+                    *reinterpret_cast<uint4*>(srow + c * 64 + i * 2) = pk;
                 }
             } else {
-                float* prow = a.part_o + (((size_t)t * a.n_split + split) * 128 + h) * kDv + dv0 + c * 32;
 #pragma unroll
                 for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4*>(prow + i) =
+                    *reinterpret_cast<float4*>(srow + c * 128 + i * 4) =
                         make_float4(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv,
                                     __uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv);
             }
         }
-        if (half == 0) {
+        tc::fence_proxy_async_smem();
+        named_bar_sync(5, kSmx * 128);               // every column of every row is staged
+        if (wg == 0) {
+            const int dv0 = half * kHalf;
+            void* dst = bf16_out ? static_cast<void*>(a.o + ((size_t)t * 128 + h) * kDv + dv0)
+                                 : static_cast<void*>(a.part_o + (((size_t)t * a.n_split + split) * 128 + h) * kDv + dv0);
+            tc::bulk_store(dst, srow, row_bytes);
+            tc::bulk_commit();
+            tc::bulk_wait_all();
+        }
+        if (half == 0 && wg == 0) {
             if (a.n_split == 1) { if (a.lse) a.lse[(size_t)t * 128 + h] = lse; }
             else a.part_lse[((size_t)t * a.n_split + split) * 128 + h] = lse;
         }
-    } else {
-        // ---------------- send warps 12..15: warp q pushes heads [32q, 32q + 32) of every partial S
+    } else if (send_warp) {
+        // ---------------- send warps: warp q (mod 4) pushes heads [32q, 32q + 32) of every partial S
         // to the peer -- staged in shared memory, then one 4 KB bulk copy that completes on the
         // peer's rx_full -- as soon as the MMA has produced it, off the softmax's path.
         const int quarter = warp & 3;
@@ -555,6 +665,8 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
         }
     }
 
+    __syncwarp();
+    if (!remote_warp) tc::cluster_wait();
     tc::tc_fence_before();
     __syncthreads();
     tc::cluster_sync_all();                      // no CTA leaves while its peer may still store into it
@@ -566,18 +678,30 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
 }
 
 template <bool KV_FP8, bool TMA>
-cudaError_t launch_t(const CUtensorMap& m, const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_t(const CUtensorMap& qm, const CUtensorMap& m, const AttnArgs& a, cudaStream_t st) {
     const size_t smem = sizeof(AttnSmem) + 1024;
     auto kern = sparse_attn_tc_kernel<KV_FP8, TMA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_split, 2, a.T);
-    kern<<<grid, kAThreads, smem, st>>>(m, a);
+    kern<<<grid, kAThreads, smem, st>>>(qm, m, a);
     return cudaGetLastError();
 }
 
 // The BF16 cache as one 2-D tensor of rows (row of sequence b, token i = b * (kv_seq_b / kv_tok_b)
 // + i) for tile::gather4.  False when the layout or the driver does not allow it.
+// The queries [T][128][576] as a 2-D tensor of T * 128 rows, box 64 dims x 128 heads.
+bool make_q_map(const AttnArgs& a, CUtensorMap* m) {
+    if (tc::encode_tiled() == nullptr || a.T < 1 || (int64_t)a.T * 128 >= ((int64_t)1 << 31)) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)a.T * 128};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    return tc::encode_tiled()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.q), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_kv_map(const AttnArgs& a, CUtensorMap* m) {
     if (tc::encode_tiled() == nullptr || a.B < 1 || a.kv_tok_b <= 0 || a.kv_seq_b % a.kv_tok_b != 0) return false;
     const int64_t rps = a.kv_seq_b / a.kv_tok_b;
@@ -596,16 +720,18 @@ bool make_kv_map(const AttnArgs& a, CUtensorMap* m) {
 
 bool sparse_attn_tc_supported(const AttnArgs& a, int DQK, int DV, bool sep_v) {
     return DQK == kD && DV == kDv && !sep_v && a.H == 128 && (a.kv_tok_b % 16) == 0 && (a.kv_seq_b % 16) == 0 &&
-           ((uintptr_t)a.kv % 16) == 0 && ((uintptr_t)a.q % 16) == 0;
+           ((uintptr_t)a.kv % 16) == 0 && ((uintptr_t)a.q % 16) == 0 && ((uintptr_t)a.o % 16) == 0 &&
+           ((uintptr_t)a.part_o % 16) == 0 && tc::encode_tiled() != nullptr;
 }
 
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, bool kv_fp8, cudaStream_t st) {
-    CUtensorMap m;
+    CUtensorMap qm, m;
     memset(&m, 0, sizeof(m));
-    if (kv_fp8) return launch_t<true, false>(m, a, st);
-    if (make_kv_map(a, &m)) return launch_t<false, true>(m, a, st);
+    if (!make_q_map(a, &qm)) return cudaErrorInvalidValue;
+    if (kv_fp8) return launch_t<true, false>(qm, m, a, st);
+    if (make_kv_map(a, &m)) return launch_t<false, true>(qm, m, a, st);
     memset(&m, 0, sizeof(m));
-    return launch_t<false, false>(m, a, st);
+    return launch_t<false, false>(qm, m, a, st);
 }
 
 }  // namespace lsa
