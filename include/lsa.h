@@ -231,8 +231,13 @@ typedef struct {
 } lsa_decode_params;
 
 /* Runs indexer (flat, or HI: block scores -> recall -> fine scores), top-k + union, then
- * attention for every layer, all on `stream`, with no host synchronisation.  Scores,
- * index lists and split partials live in `ws` (lsa_decode_workspace_size bytes). */
+ * attention for every layer, with no host synchronisation.  Everything is ordered after the
+ * work already queued on `stream`, and work queued on `stream` afterwards runs after all of
+ * it.  With two or more layers the layers alternate between `stream` and a second stream of
+ * the calling thread (created on first use, with two events; forked from `stream` after
+ * top-k and joined back before returning), so that two layers' attention kernels can share
+ * the GPU; captured into a CUDA graph this becomes two branches.  Scores, index lists and the
+ * split partials of each branch live in `ws` (lsa_decode_workspace_size bytes). */
 lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_bytes,
                             int32_t* dev_status, void* stream);
 

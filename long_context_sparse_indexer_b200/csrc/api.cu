@@ -1,5 +1,5 @@
 // C ABI of the LSA library: host-side validation, workspace carving and kernel dispatch.
-// No allocation, no synchronisation (except lsa_read_device_status), no exceptions.
+// No device allocation, no synchronisation (except lsa_read_device_status), no exceptions.
 #include <cmath>
 #include <cstring>
 
@@ -151,7 +151,7 @@ lsa_status attn_impl(const lsa_batch* batch, const void* q, int H, int Dqk, cons
 
 // Workspace plan of the fused path.
 struct FusedPlan {
-    size_t scores = 0, bscores = 0, cand = 0, ccount = 0, idx = 0, count = 0, attn = 0, total = 0;
+    size_t scores = 0, bscores = 0, cand = 0, ccount = 0, idx = 0, count = 0, attn = 0, attn_one = 0, total = 0;
     int n_cols = 0, nblk = 0, cap = 0;
     int64_t ld = 0, bld = 0;
 };
@@ -174,9 +174,39 @@ bool plan_fused(const lsa_decode_params* p, FusedPlan& f) {
     f.scores = off; off += align_up((size_t)T * f.ld * 4);
     f.idx = off; off += align_up((size_t)T * f.cap * 4);
     f.count = off; off += align_up((size_t)T * 4);
-    f.attn = off; off += attn_ws(T, p->H, p->Dv, p->n_split);
+    // One split-partial area per attention branch (layers alternate between two branches).
+    f.attn_one = attn_ws(T, p->H, p->Dv, p->n_split);
+    f.attn = off; off += (size_t)(p->n_layers > 1 ? 2 : 1) * f.attn_one;
     f.total = off;
     return true;
+}
+
+// A second stream of the calling thread on the current device, created on first use, with
+// the two events that fork it from the caller's stream and join it back.  Under stream capture
+// the fork and the join become dependencies of the captured graph.
+struct AuxStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+AuxStream* aux_stream() {
+    static thread_local AuxStream aux[16];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return nullptr;
+    AuxStream& a = aux[dev];
+    if (!a.s) {
+        cudaStream_t s = nullptr;
+        cudaEvent_t f = nullptr, j = nullptr;
+        if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+        if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+            if (f) cudaEventDestroy(f);
+            cudaStreamDestroy(s);
+            return nullptr;
+        }
+        a.s = s; a.fork = f; a.join = j;
+    }
+    return &a;
 }
 
 }  // namespace
@@ -305,14 +335,28 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
                       0, idx, ld_idx, count, dev_status, st);
         if (s != LSA_OK) return s;
     }
-    float* part = reinterpret_cast<float*>(w + f.attn);
+    // The layers depend only on the shared index list, not on one another: layer l runs on
+    // branch l mod 2 (the caller's stream, and a second stream forked from it after top-k),
+    // each branch with its own split partials, so that one layer's CTAs fill the SMs the
+    // other's leave.  Without a second stream the layers run in order on the caller's.
+    AuxStream* aux = p->n_layers > 1 ? aux_stream() : nullptr;
+    if (aux) {
+        if (cudaEventRecord(aux->fork, st) != cudaSuccess || cudaStreamWaitEvent(aux->s, aux->fork, 0) != cudaSuccess)
+            return LSA_ERR_CUDA;
+    }
     for (int l = 0; l < p->n_layers; ++l) {
         const lsa_layer& L = p->layers[l];
+        const int br = aux ? (l & 1) : 0;
+        float* part = reinterpret_cast<float*>(w + f.attn + (size_t)(l & 1) * f.attn_one);
         s = attn_impl(batch, L.q, p->H, p->Dqk, &L.kv, L.v.data ? &L.v : nullptr, p->Dv, idx, ld_idx, count,
-                      p->sm_scale, p->n_split, L.o, L.lse, part, attn_ws(batch->T, p->H, p->Dv, p->n_split),
-                      dev_status, st);
-        if (s != LSA_OK) return s;
+                      p->sm_scale, p->n_split, L.o, L.lse, part, f.attn_one, dev_status, br ? aux->s : st);
+        if (s != LSA_OK) break;
     }
+    if (aux) {                                   // join, also after an error, so the caller's stream waits
+        if (cudaEventRecord(aux->join, aux->s) != cudaSuccess || cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess)
+            return LSA_ERR_CUDA;
+    }
+    if (s != LSA_OK) return s;
     return LSA_OK;
 }
 
