@@ -243,6 +243,43 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
 
 size_t lsa_decode_workspace_size(const lsa_decode_params* p);
 
+/* ---------------------------------------------------------------- pipelined host I/O
+ * A decode driver for callers whose queries and outputs live in host memory (pinned, so that
+ * the copies are asynchronous).  Each lsa_pipeline_step copies one step's inputs from host to
+ * device buffers (`h2d`, one cudaMemcpyAsync each, in order), runs lsa_decode_fused for each of
+ * the step's `n_params` parameter sets (with workspace ws[i] of ws_bytes[i] bytes), then copies
+ * the outputs back (`d2h`): the copy-in on a stream of the pipeline, the decode on the stream
+ * given at creation, the copy-out on a second stream of the pipeline, ordered by events, so that
+ * one step's copies overlap the decode of the steps next to it.  The caller keeps `n_slots`
+ * sets of device input / output buffers and passes slot = step index mod n_slots: a slot's
+ * copy-in waits until the decode that last read that slot's inputs has finished, and its
+ * decode waits until the copy-out that last read that slot's outputs has finished.
+ * Workspaces, dev_status and the index outputs may be shared between slots (the decodes run in
+ * order on one stream).  Host buffers must stay valid and unchanged until the copies that
+ * read or write them have run.
+ *
+ * lsa_pipeline_create: n_slots in [1, 8]; creates two streams and 3 n_slots + 1 events on the
+ *   current device (no device memory).  *out receives the pipeline.
+ * lsa_pipeline_step: LSA_ERR_INVALID_ARG for a bad slot, count or NULL array; any error of
+ *   lsa_decode_fused; LSA_ERR_CUDA when a copy or event call fails.  Nothing is synchronised.
+ * lsa_pipeline_join: makes the decode stream wait for every copy issued so far, so that work
+ *   queued on it afterwards (an event, a synchronisation) follows all of the host outputs.
+ * lsa_pipeline_destroy: waits for the pipeline's streams, then releases them and its events. */
+typedef struct {
+    void*       dst;
+    const void* src;
+    size_t      bytes;
+} lsa_copy;
+
+typedef struct lsa_pipeline lsa_pipeline;
+
+lsa_status lsa_pipeline_create(lsa_pipeline** out, int n_slots, void* stream);
+lsa_status lsa_pipeline_step(lsa_pipeline* pl, int slot, const lsa_decode_params* const* params, int n_params,
+                             void* const* ws, const size_t* ws_bytes, const lsa_copy* h2d, int n_h2d,
+                             const lsa_copy* d2h, int n_d2h, int32_t* dev_status);
+lsa_status lsa_pipeline_join(lsa_pipeline* pl);
+lsa_status lsa_pipeline_destroy(lsa_pipeline* pl);
+
 /* ---------------------------------------------------------------- helpers
  * Synchronises `stream`, then returns the status stored at dev_status (LSA_OK when 0),
  * or LSA_ERR_CUDA if the copy fails. */

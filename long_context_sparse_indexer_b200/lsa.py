@@ -78,6 +78,17 @@ _lib.lsa_decode_fused.argtypes = [_P(CDecodeParams), c_vp, c_size, c_vp, c_vp]
 _lib.lsa_decode_workspace_size.argtypes = [_P(CDecodeParams)]
 _lib.lsa_decode_workspace_size.restype = c_size
 _lib.lsa_read_device_status.argtypes = [c_vp, c_vp]
+
+
+class CCopy(ctypes.Structure):
+    _fields_ = [("dst", c_vp), ("src", c_vp), ("bytes", c_size)]
+
+
+_lib.lsa_pipeline_create.argtypes = [ctypes.POINTER(c_vp), c_i32, c_vp]
+_lib.lsa_pipeline_step.argtypes = [c_vp, c_i32, ctypes.POINTER(_P(CDecodeParams)), c_i32, ctypes.POINTER(c_vp),
+                                   ctypes.POINTER(c_size), _P(CCopy), c_i32, _P(CCopy), c_i32, c_vp]
+_lib.lsa_pipeline_join.argtypes = [c_vp]
+_lib.lsa_pipeline_destroy.argtypes = [c_vp]
 _lib.lsa_status_string.argtypes = [c_i32]
 _lib.lsa_status_string.restype = ctypes.c_char_p
 _lib.lsa_version.restype = c_i32
@@ -87,7 +98,8 @@ for _f in ("lsa_index_score", "lsa_block_keys", "lsa_block_score", "lsa_topk", "
 
 EXPORTS = ("lsa_index_score", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
            "lsa_sparse_attn_noalloc", "lsa_attn_workspace_size", "lsa_decode_fused", "lsa_decode_workspace_size", "lsa_read_device_status",
-           "lsa_status_string", "lsa_version")
+           "lsa_status_string", "lsa_version", "lsa_pipeline_create", "lsa_pipeline_step", "lsa_pipeline_join",
+           "lsa_pipeline_destroy")
 
 
 def library() -> ctypes.CDLL:
@@ -262,6 +274,61 @@ class DecodeStep:
     def __call__(self, ws: torch.Tensor, dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
         _check(_lib.lsa_decode_fused(ctypes.byref(self.p), _ptr(ws), ws.numel() * ws.element_size(),
                                      _ptr(dev_status), _stream(stream)), "lsa_decode_fused")
+
+
+class Pipeline:
+    """lsa_pipeline_*: pipelined host-buffer decode (copy-in, fused decode, copy-out on three
+    streams, ordered per device-buffer slot).  `prepare` marshals one slot's step once; `run`
+    issues it (no synchronisation); `join` orders the decode stream after every copy issued."""
+
+    class Prepared:
+        def __init__(self, slot, steps, wss, h2d, d2h, dev_status):
+            self.slot = int(slot)
+            self._keep = (steps, wss, h2d, d2h, dev_status)
+            n = len(steps)
+            self.params = (_P(CDecodeParams) * max(1, n))(*[ctypes.pointer(st.p) for st in steps])
+            self.ws = (c_vp * max(1, n))(*[_ptr(w) for w in wss])
+            self.ws_bytes = (c_size * max(1, n))(*[w.numel() * w.element_size() for w in wss])
+            self.n = n
+            self.h2d = (CCopy * max(1, len(h2d)))(*[CCopy(_ptr(d), _ptr(h), h.numel() * h.element_size())
+                                                    for d, h in h2d])
+            self.n_h2d = len(h2d)
+            self.d2h = (CCopy * max(1, len(d2h)))(*[CCopy(_ptr(h), _ptr(d), d.numel() * d.element_size())
+                                                    for h, d in d2h])
+            self.n_d2h = len(d2h)
+            self.dev_status = _ptr(dev_status)
+
+    def __init__(self, n_slots: int = 2, stream=None):
+        h = c_vp()
+        _check(_lib.lsa_pipeline_create(ctypes.byref(h), int(n_slots), _stream(stream)), "lsa_pipeline_create")
+        self._h = h
+
+    def prepare(self, slot: int, steps: Sequence["DecodeStep"], wss: Sequence[torch.Tensor],
+                h2d: Sequence[tuple], d2h: Sequence[tuple], dev_status: Optional[torch.Tensor] = None) -> "Pipeline.Prepared":
+        """h2d: (device tensor, pinned host tensor) pairs; d2h: (pinned host tensor, device tensor) pairs."""
+        for d, h in list(h2d) + [(d, h) for h, d in d2h]:
+            assert d.is_cuda and not h.is_cuda and d.is_contiguous() and h.is_contiguous()
+            assert d.numel() * d.element_size() == h.numel() * h.element_size()
+        return Pipeline.Prepared(slot, list(steps), list(wss), list(h2d), list(d2h), dev_status)
+
+    def run(self, pr: "Pipeline.Prepared") -> None:
+        _check(_lib.lsa_pipeline_step(self._h, pr.slot, pr.params, pr.n, pr.ws, pr.ws_bytes, pr.h2d, pr.n_h2d,
+                                      pr.d2h, pr.n_d2h, pr.dev_status), "lsa_pipeline_step")
+
+    def join(self) -> None:
+        _check(_lib.lsa_pipeline_join(self._h), "lsa_pipeline_join")
+
+    def close(self) -> None:
+        if self._h:
+            _check(_lib.lsa_pipeline_destroy(self._h), "lsa_pipeline_destroy")
+            self._h = c_vp()
+
+    def __del__(self):
+        try:
+            if self._h:
+                _lib.lsa_pipeline_destroy(self._h)
+        except Exception:
+            pass
 
 
 def read_device_status(dev_status: torch.Tensor, stream=None) -> int:

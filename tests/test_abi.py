@@ -116,3 +116,15 @@ def test_binding_refuses_to_run_without_cuda_library_on_missing_build(tmp_path, 
         importlib.reload(mod)
     monkeypatch.undo()
     importlib.reload(mod)
+
+
+def test_pipeline_rejects_bad_arguments():
+    """lsa_pipeline_*: argument checks happen before any CUDA call (no device needed)."""
+    lib = lsa.library()
+    out = ctypes.c_void_p()
+    assert lib.lsa_pipeline_create(None, 2, None) == lsa.ERR_INVALID_ARG
+    assert lib.lsa_pipeline_create(ctypes.byref(out), 0, None) == lsa.ERR_INVALID_ARG
+    assert lib.lsa_pipeline_create(ctypes.byref(out), 9, None) == lsa.ERR_INVALID_ARG
+    assert lib.lsa_pipeline_step(None, 0, None, 0, None, None, None, 0, None, 0, None) == lsa.ERR_INVALID_ARG
+    assert lib.lsa_pipeline_join(None) == lsa.ERR_INVALID_ARG
+    assert lib.lsa_pipeline_destroy(None) == lsa.ERR_INVALID_ARG

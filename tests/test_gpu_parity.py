@@ -272,6 +272,46 @@ def test_fused_path_end_to_end(cuda, name):
                     assert mx < 1e-2 and rl2 < 5e-3, (t, li, mx, rl2)
 
 
+@pytest.mark.parametrize("name", ["cli_small", "mtp_small"])
+def test_pipeline_host_io_matches_device_path(cuda, name):
+    """lsa_pipeline_*: queries copied in from pinned host memory into two slots of device
+    buffers (which start zeroed), the fused decode, outputs copied back into host buffers
+    (which start as garbage); after three steps every host output equals, bit for bit, the
+    output of lsa_decode_fused called directly on the same queries."""
+    w = SMALL[name]
+    wt = wt_of(name)
+    pi, pt = 0, wt.passes[0]
+    step, ws, idx, cnt, layers = H.decode_step(wt, pi, n_split=3)
+    step(ws)
+    torch.cuda.synchronize()
+    ref = [L.o.cpu() for L in layers]
+    slots = []
+    for s in range(2):
+        q_idx, wv = torch.zeros_like(pt.q_idx), torch.zeros_like(pt.w)
+        ins, lay = [q_idx, wv], []
+        for L in layers:
+            q = torch.zeros_like(L.q)
+            ins.append(q)
+            lay.append(lsa.Layer(q, L.kv, torch.zeros_like(L.o), torch.empty_like(L.lse), L.v))
+        dec = lsa.DecodeStep(H.batch_of(wt, pi), q_idx, wv, H.idx_cache(wt, pi), w.k, w.n_sink, w.window, lay,
+                             w.H, w.D, w.Dv, w.sm_scale, n_split=3, idx_out=idx, count_out=cnt)
+        host_in = [t.cpu().contiguous().pin_memory() for t in [pt.q_idx, pt.w] + [L.q for L in layers]]
+        host_out = [torch.full(L.o.shape, 7.0, dtype=L.o.dtype).pin_memory() for L in layers]
+        slots.append((dec, list(zip(ins, host_in)), list(zip(host_out, [L.o for L in lay])), host_out))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pl = lsa.Pipeline(2)
+    preps = [pl.prepare(s, [dec], [ws], h2d, d2h, st) for s, (dec, h2d, d2h, _) in enumerate(slots)]
+    for i in range(3):
+        pl.run(preps[i % 2])
+    pl.join()
+    torch.cuda.synchronize()
+    assert lsa.read_device_status(st) == lsa.OK
+    for _, _, _, host_out in slots:
+        for li, h in enumerate(host_out):
+            assert torch.equal(h, ref[li]), (li, (h.float() - ref[li].float()).abs().max())
+    pl.close()
+
+
 @pytest.mark.parametrize("name", FLAT)
 def test_oracle_selection_on_gpu_scores_is_bit_exact(cuda, name):
     """The oracle's top-k + union, run on the GPU's own scores, gives the GPU's index list exactly."""
