@@ -256,15 +256,21 @@ size_t lsa_decode_workspace_size(const lsa_decode_params* p);
  * decode waits until the copy-out that last read that slot's outputs has finished.
  * Workspaces, dev_status and the index outputs may be shared between slots (the decodes run in
  * order on one stream).  Host buffers must stay valid and unchanged until the copies that
- * read or write them have run.
+ * read or write them have run.  A slot's decode is captured into a CUDA graph on its first
+ * step (on a stream of the pipeline) and replayed while the slot's parameter sets, workspaces
+ * and dev_status are the same as at the capture (compared byte for byte, layer arrays
+ * included); otherwise it is captured again.  When the decode stream is itself being
+ * captured, or a capture fails, the decode is launched directly. 
  *
  * lsa_pipeline_create: n_slots in [1, 8]; creates two streams and 3 n_slots + 1 events on the
- *   current device (no device memory).  *out receives the pipeline.
+ *   current device (a third stream and the slot graphs on first use; no device memory of
+ *   its own).  *out receives the pipeline.
  * lsa_pipeline_step: LSA_ERR_INVALID_ARG for a bad slot, count or NULL array; any error of
  *   lsa_decode_fused; LSA_ERR_CUDA when a copy or event call fails.  Nothing is synchronised.
  * lsa_pipeline_join: makes the decode stream wait for every copy issued so far, so that work
  *   queued on it afterwards (an event, a synchronisation) follows all of the host outputs.
- * lsa_pipeline_destroy: waits for the pipeline's streams, then releases them and its events. */
+ * lsa_pipeline_destroy: waits for the pipeline's streams, then releases them, its events and
+ *   its graphs. */
 typedef struct {
     void*       dst;
     const void* src;

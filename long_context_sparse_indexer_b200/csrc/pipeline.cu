@@ -1,6 +1,9 @@
 // Pipelined host I/O around lsa_decode_fused: copy-in, decode and copy-out of consecutive
-// steps on three streams, ordered per buffer slot by events (see lsa.h).
+// steps on three streams, ordered per buffer slot by events (see lsa.h).  A slot's decode is
+// captured once into a CUDA graph and replayed while its parameters stay the same.
+#include <cstring>
 #include <new>
+#include <vector>
 
 #include "kernels.cuh"
 
@@ -12,6 +15,9 @@ struct lsa_pipeline {
     cudaEvent_t in_done[kMaxSlots] = {}, dec_done[kMaxSlots] = {}, out_done[kMaxSlots] = {};
     cudaEvent_t joined = nullptr;
     bool used[kMaxSlots] = {};                   // the slot has events recorded
+    cudaStream_t cap = nullptr;                  // capture stream of the slot graphs
+    cudaGraphExec_t exec[kMaxSlots] = {};        // the slot's captured decode
+    std::vector<unsigned char> sig[kMaxSlots];   // the parameters it was captured with
 };
 
 namespace {
@@ -23,12 +29,82 @@ void release(lsa_pipeline* pl) {
         if (pl->out_done[i]) cudaEventDestroy(pl->out_done[i]);
     }
     if (pl->joined) cudaEventDestroy(pl->joined);
+    for (int i = 0; i < lsa_pipeline::kMaxSlots; ++i)
+        if (pl->exec[i]) cudaGraphExecDestroy(pl->exec[i]);
+    if (pl->cap) cudaStreamDestroy(pl->cap);
     if (pl->in) cudaStreamDestroy(pl->in);
     if (pl->out) cudaStreamDestroy(pl->out);
     delete pl;
 }
 
 inline bool ok(cudaError_t e) { return e == cudaSuccess; }
+
+void append(std::vector<unsigned char>& v, const void* p, size_t n) {
+    const unsigned char* c = static_cast<const unsigned char*>(p);
+    v.insert(v.end(), c, c + n);
+}
+
+// Everything a captured decode depends on: every parameter set with its layer array, the
+// workspaces and the status word.
+std::vector<unsigned char> signature(const lsa_decode_params* const* params, int n, void* const* ws,
+                                     const size_t* ws_bytes, const int32_t* dev_status) {
+    std::vector<unsigned char> v;
+    append(v, &n, sizeof(n));
+    append(v, &dev_status, sizeof(dev_status));
+    for (int i = 0; i < n; ++i) {
+        append(v, params[i], sizeof(lsa_decode_params));
+        if (params[i]->n_layers > 0 && params[i]->layers)
+            append(v, params[i]->layers, sizeof(lsa_layer) * (size_t)params[i]->n_layers);
+        append(v, &ws[i], sizeof(ws[i]));
+        append(v, &ws_bytes[i], sizeof(ws_bytes[i]));
+    }
+    return v;
+}
+
+lsa_status decode_eager(const lsa_decode_params* const* params, int n, void* const* ws, const size_t* ws_bytes,
+                        int32_t* dev_status, cudaStream_t st) {
+    lsa_status s = LSA_OK;
+    for (int i = 0; i < n && s == LSA_OK; ++i) s = lsa_decode_fused(params[i], ws[i], ws_bytes[i], dev_status, st);
+    return s;
+}
+
+// Runs the slot's decode on pl->st: its graph when the parameters match the capture, else a new
+// capture (on the pipeline's own stream, so the caller's stream is never in capture mode).
+// Eager launches when the caller's stream is itself being captured or a capture fails.
+lsa_status decode_slot(lsa_pipeline* pl, int slot, const lsa_decode_params* const* params, int n, void* const* ws,
+                       const size_t* ws_bytes, int32_t* dev_status) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (!ok(cudaStreamIsCapturing(pl->st, &cs)) || cs != cudaStreamCaptureStatusNone)
+        return decode_eager(params, n, ws, ws_bytes, dev_status, pl->st);
+    std::vector<unsigned char> sig = signature(params, n, ws, ws_bytes, dev_status);
+    if (!pl->exec[slot] || sig != pl->sig[slot]) {
+        if (pl->exec[slot]) {
+            cudaGraphExecDestroy(pl->exec[slot]);
+            pl->exec[slot] = nullptr;
+        }
+        if (!pl->cap && !ok(cudaStreamCreateWithFlags(&pl->cap, cudaStreamNonBlocking)))
+            return decode_eager(params, n, ws, ws_bytes, dev_status, pl->st);
+        if (!ok(cudaStreamBeginCapture(pl->cap, cudaStreamCaptureModeThreadLocal)))
+            return decode_eager(params, n, ws, ws_bytes, dev_status, pl->st);
+        const lsa_status s = decode_eager(params, n, ws, ws_bytes, dev_status, pl->cap);
+        cudaGraph_t g = nullptr;
+        const bool captured = ok(cudaStreamEndCapture(pl->cap, &g)) && g != nullptr;
+        if (s != LSA_OK) {                       // invalid parameters: nothing was launched
+            if (g) cudaGraphDestroy(g);
+            return s;
+        }
+        cudaGraphExec_t e = nullptr;
+        const bool inst = captured && ok(cudaGraphInstantiate(&e, g, 0));
+        if (g) cudaGraphDestroy(g);
+        if (!inst) {
+            cudaGetLastError();
+            return decode_eager(params, n, ws, ws_bytes, dev_status, pl->st);
+        }
+        pl->exec[slot] = e;
+        pl->sig[slot] = std::move(sig);
+    }
+    return ok(cudaGraphLaunch(pl->exec[slot], pl->st)) ? LSA_OK : LSA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -73,8 +149,7 @@ lsa_status lsa_pipeline_step(lsa_pipeline* pl, int slot, const lsa_decode_params
         return LSA_ERR_CUDA;
     // Decode, once the copy-out that last read this slot's outputs has finished.
     if (again && !ok(cudaStreamWaitEvent(pl->st, pl->out_done[slot], 0))) return LSA_ERR_CUDA;
-    lsa_status s = LSA_OK;
-    for (int i = 0; i < n_params && s == LSA_OK; ++i) s = lsa_decode_fused(params[i], ws[i], ws_bytes[i], dev_status, pl->st);
+    lsa_status s = n_params ? decode_slot(pl, slot, params, n_params, ws, ws_bytes, dev_status) : LSA_OK;
     // The events below are recorded also after an error, so that the slot's ordering holds.
     if (!ok(cudaEventRecord(pl->dec_done[slot], pl->st)) || !ok(cudaStreamWaitEvent(pl->out, pl->dec_done[slot], 0)))
         return LSA_ERR_CUDA;
