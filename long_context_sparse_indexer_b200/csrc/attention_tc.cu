@@ -60,10 +60,10 @@ constexpr int kAThreads = 512;
 constexpr int kRows = 32;                    // KV rows per tile
 constexpr int kStagesA = 8;                  // KV tile ring
 constexpr int kXB = 2;                       // partial-S exchange buffers (staging and receive)
-constexpr int kSP = 3;                       // S / P buffers in TMEM (P overwrites its own S)
+constexpr int kSP = 4;                       // S / P buffers in TMEM (P overwrites its own S)
 constexpr int kD = 576, kDv = 512, kHalf = 256;
 constexpr int kKSteps = 4 * 4 + 2;           // 16-dim K steps of S per CTA (288 dims)
-constexpr int kQCols = kKSteps * 8;          // TMEM columns of the query slice (144)
+constexpr int kQCols = 16 * 8;               // TMEM columns of the query's V-half dims (128)
 constexpr int kVBytes = 4 * kRows * 128;                  // a tile's 4 V-half atoms, 16 KB
 constexpr int kRopeBytes = kRows * 128;                   // one rope atom, shared by two stages
 static_assert(256 + kSP * 32 + kQCols <= 512, "TMEM columns: O half, S / P buffers, query slice");
@@ -76,6 +76,9 @@ struct AttnSmem {
     // 4 KB of heads [32q, 32q + 32) in each.
     alignas(1024) uint8_t xs[kXB][kXBytes];      // the peer's partial S
     alignas(1024) uint8_t stg[kXB][kXBytes];     // this CTA's partial S, the source of the copy to the peer
+    // The query's 32 rope dims of this CTA, K-major without swizzle: head h, 8-dim chunk c at
+    // (h / 8) * 512 + c * 128 + (h % 8) * 16 -- the A operand of the two rope K steps of S.
+    alignas(1024) uint8_t q_rope[128 * 64];
     alignas(16) float kscale[kStagesA][kRows];   // per-row FP8 scale x softmax scale (0 for masked rows)
     alignas(16) float kmask[kStagesA][kRows];    // 0, or -inf for masked rows (added to the scaled score)
     alignas(16) float vscale[kStagesA][kRows];   // per-row FP8 scale (1 for BF16)
@@ -207,16 +210,15 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             }
             tc::tmem_st32(qt_col + at * 32 + lane_off, w);
         }
-        if (kSmx == 1 || wg == 1) {                  // this CTA's rope chunks: 4 half .. 4 half + 3
+        if (kSmx == 1 || wg == 1) {                  // this CTA's rope chunks 4 half .. 4 half + 3
             const uint8_t* row = q_atom(4) + h * 128;
-            uint32_t w[16];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const uint4 v = got ? *reinterpret_cast<const uint4*>(row + (((4 * half + c) ^ (h & 7)) << 4))
                                     : make_uint4(0, 0, 0, 0);
-                w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+                *reinterpret_cast<uint4*>(sm.q_rope + (h >> 3) * 512 + c * 128 + (h & 7) * 16) = v;
             }
-            tc::tmem_st16(qt_col + 128 + lane_off, w);
+            tc::fence_proxy_async_smem();            // for the tensor cores
         }
         tc::tmem_wait_st();
         tc::tc_fence_before();
@@ -359,6 +361,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
         // ---------------- MMA issuer: S_j and P_j V_j, each in order, whichever is ready
         const uint32_t idesc_s = tc::idesc_f16(128, kRows, 1);
         const uint32_t idesc_o = tc::idesc_f16_bmn(128, kHalf, 1);
+        const uint32_t qraddr = tc::smem_u32(sm.q_rope);
         if (tc::elect_one() && n_tiles > 0 && tc::mbar_wait(&sm.q_ready, 0, abort_flag)) {
             tc::tc_fence_after();
             int ns = 0, npv = 0;                 // next S tile, next P V tile
@@ -379,10 +382,14 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                     const int rh = half ^ (st & 1);
 #pragma unroll
                     for (int kk = 0; kk < kKSteps; ++kk) {
-                        const uint32_t aaddr = kk < 16 ? kaddr + (kk >> 2) * (kRows * 128) + (kk & 3) * 32
-                                                       : raddr + (2 * rh + kk - 16) * 32;
-                        const uint64_t bd = tc::sdesc_sw128(aaddr);
-                        tc::mma_f16_ts(s_col + sb * 32, qt_col + kk * 8, bd, idesc_s, kk > 0);
+                        if (kk < 16) {                   // V-half dims: A (query) from TMEM
+                            const uint64_t bd = tc::sdesc_sw128(kaddr + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+                            tc::mma_f16_ts(s_col + sb * 32, qt_col + kk * 8, bd, idesc_s, kk > 0);
+                        } else {                         // rope dims: A from shared memory
+                            const uint64_t ad = tc::sdesc_none(qraddr + (kk - 16) * 256, 128, 512);
+                            const uint64_t bd = tc::sdesc_sw128(raddr + (2 * rh + kk - 16) * 32);
+                            tc::mma_f16_ss(s_col + sb * 32, ad, bd, idesc_s, 1u);
+                        }
                     }
                     tc::mma_commit(&sm.s_full[sb]);
                     ++ns;
@@ -473,6 +480,16 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
 #pragma unroll
                 for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
             const float mt = mx[0];
+            // Every lane's tile max depends on every word it read from buffer xb, so once this vote
+            // has run the warp's reads of the buffer are complete: the peer may overwrite it (a
+            // release arrive would stall the warp for about half a tile's time).  Released this
+            // early, the peer's next copy into the buffer is not held up by this tile's softmax.
+            {
+                uint32_t v;                          // a warp vote on every lane's max (kept by volatile)
+                asm volatile("{ .reg .pred p, q; setp.ne.f32 p, %1, %1; vote.sync.any.pred q, p, 0xffffffff; selp.u32 %0, 1, 0, q; }"
+                             : "=r"(v) : "f"(mt));
+                if (lane == 0) tc::mbar_arrive_remote_relaxed(tc::peer_smem(&sm.tx_free[xb][quarter], peer));
+            }
             // The reference max is raised to the tile max only when that exceeds it by more than
             // 2^8 (lazy rescaling).  With two warpgroups the decisions form one chain over the
             // tiles: tile j's starts from tile j-1's, handed over through shared memory.
@@ -535,12 +552,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                 break;
             }
             tc::tmem_st16(s_col + sb * 32 + lane_off, pw);
-            // Every lane's max depends on every word it read from buffer xb, so once this vote has
-            // run, the warp's reads of the buffer are complete and the peer may overwrite it.  (A
-            // release arrive here stalls the warp for about half a tile's time.)
-            const bool any_rescale = __any_sync(0xffffffffu, rescale);
-            if (lane == 0) tc::mbar_arrive_remote_relaxed(tc::peer_smem(&sm.tx_free[xb][quarter], peer));
-            if (any_rescale) {
+            if (__any_sync(0xffffffffu, rescale)) {
                 // O must hold P V_{j-1} before it is rescaled.
                 if (j >= 1 &&
                     !__all_sync(0xffffffffu, tc::mbar_wait(&sm.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {

@@ -183,6 +183,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128_lbo(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// Shared-memory matrix descriptor, K-major, no swizzle: core matrices of 8 rows x 16 bytes
+// (128 contiguous bytes); the two 16-byte K chunks of a 16-element K step are `lbo` bytes
+// apart and successive 8-row groups `sbo` bytes apart.
+__device__ __forceinline__ uint64_t sdesc_none(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;                             // descriptor version (sm_100); layout 0: no swizzle
+    return d;
+}
+
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     uint64_t d = 0;
@@ -285,10 +297,12 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t dst, uint4 v) {
 
 // mbar_wait with acquire at cluster scope, for phases completed by a peer CTA's remote arrivals
 // (the peer's stores before its release-arrive are visible afterwards).  Bounded as mbar_wait.
+// Polls with test_wait (never suspends): a thread suspended in try_wait was seen to resume
+// well after a remote arrival completed the phase.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        "{ .reg .pred p; mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
