@@ -253,7 +253,10 @@ def run_gpu(args, rank, world, local_rank):
     w = rank_workload(w, rank, world)
     wt = D.build_workload(w, dev)
     stream = torch.cuda.current_stream()
-    sds = [build_step(w, wt, pi, launch.split_for(w.T(p), w.H, w.cap)) for pi, p in enumerate(w.passes)]
+    forced = [int(x) for x in args.n_split.split(",")] if args.n_split else []
+    sds = [build_step(w, wt, pi, forced[min(pi, len(forced) - 1)] if forced
+                      else launch.split_for(w.T(p), w.H, w.cap, layers=len(p.layers)))
+           for pi, p in enumerate(w.passes)]
 
     def step():
         for sd in sds:
@@ -494,6 +497,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the sequence count (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--n-split", default="", help="override the split-KV chunk count: one value, or one per pass")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

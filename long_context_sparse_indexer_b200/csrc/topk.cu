@@ -102,6 +102,88 @@ __device__ int cluster_threshold(cg::cluster_group& cl, int rank, int* hist, int
     return total;
 }
 
+// One warp: over 64 counts c[0..63] taken from the top (index 63 first) after `base` counts
+// above them, the index where the running count first reaches `need` (run < need <= run + c)
+// and the count above it; lane 0 writes them to *bin / *above (-1 / unchanged when there is
+// none) and, if `total` is given, the sum of the 64 counts to *total.
+__device__ __forceinline__ void top_crossing(const int* c, int base, int need, int* bin, int* above, int* total) {
+    const int lane = threadIdx.x & 31;
+    const int hi = c[63 - 2 * lane], lo = c[62 - 2 * lane];
+    int incl = hi + lo;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    const int run = base + incl - hi - lo;
+    int found = -1, fa = 0;
+    if (run < need && run + hi >= need) { found = 63 - 2 * lane; fa = run; }
+    else if (run + hi < need && run + hi + lo >= need) { found = 62 - 2 * lane; fa = run + hi; }
+    const uint32_t m = __ballot_sync(0xffffffffu, found >= 0);
+    const int src = m ? __ffs(m) - 1 : 0;
+    const int f = __shfl_sync(0xffffffffu, found, src), a = __shfl_sync(0xffffffffu, fa, src);
+    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0) {
+        *bin = m ? f : -1;
+        if (m) *above = a;
+        if (total) *total = tot;
+    }
+}
+
+// Two-level form of cluster_threshold for the 4096-bin histogram of the top 12 bits, with one
+// cluster barrier.  Each CTA folds its histogram into 64 super-bins of 64 bins (`sup`); after
+// the barrier every CTA reads the cluster's 8 x 64 super-bin counts, finds the super-bin where
+// the count from the top reaches `need`, then reads the 8 x 64 bin counts inside it and finds
+// the bin (the same rule, so the same bin, as the one-level form).  Peers read `hist` and `sup`
+// after this returns: the caller must pass another cluster barrier before changing either.
+// Returns the cluster's total count; *s_bin / *s_above are left unchanged when no bin reaches
+// `need` (need <= 0 or need > total).
+__device__ int cluster_threshold_4096(cg::cluster_group& cl, const int* hist, int* sup, int need, int* s_red,
+                                      int* s_bin, int* s_above, int* s_total) {
+    const int t = threadIdx.x, lane = t & 31;
+    static_assert(kTopkThreads == 512 && kTopkCluster == 8, "one thread per 8 bins, 8 lanes per super-bin");
+    __syncthreads();                                     // the local histogram is complete
+    {
+        int s = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s += hist[8 * t + i];
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        if ((t & 7) == 0) sup[t >> 3] = s;
+    }
+    cl.sync();                                           // every CTA's histogram and super-bins complete
+    // Thread t: super-bin t >> 3 of CTA t & 7; the 8 lanes of a super-bin add up the CTAs.
+    {
+        int v = cl.map_shared_rank(sup, t & 7)[t >> 3];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        if ((t & 7) == 0) s_red[t >> 3] = v;
+    }
+    __syncthreads();
+    // Warp 0 walks the 64 totals from the top (lane l: super-bins 63 - 2l and 62 - 2l).
+    if (t < 32) top_crossing(s_red, 0, need, s_red + 64, s_red + 65, s_total);
+    __syncthreads();
+    const int sb = s_red[64];
+    if (sb >= 0) {
+        // Thread t: bin 64 sb + (t >> 3) of CTA t & 7.
+        int v = cl.map_shared_rank(hist, t & 7)[64 * sb + (t >> 3)];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        if ((t & 7) == 0) s_red[66 + (t >> 3)] = v;
+        __syncthreads();
+        if (t < 32) {
+            int bin = -1, above = 0;
+            top_crossing(s_red + 66, s_red[65], need, &bin, &above, nullptr);
+            if (lane == 0 && bin >= 0) { *s_bin = 64 * sb + bin; *s_above = above; }
+        }
+    }
+    __syncthreads();
+    return *s_total;
+}
+
 // Cluster-wide exclusive prefix of one int per CTA (the value in `slot` of each CTA).  Every
 // exchange uses its own slot, so the slot is never rewritten while a peer may still read it.
 __device__ int cluster_exclusive(cg::cluster_group& cl, int* slot, int rank, int& total) {
@@ -152,7 +234,8 @@ topk_kernel(TopkArgs a) {
     __shared__ int hsum[4096];
     __shared__ int s_warp[kTopkWarps];
     __shared__ int s_bin, s_above, s_slot[3], s_wmax;
-    __shared__ int s_wcnt[kTopkWarps];
+    __shared__ int s_wcnt[kTopkWarps], s_wk[kTopkWarps];
+    __shared__ int s_sup[64], s_red[130], s_total, hist3[256];
     extern __shared__ uint32_t s_keys[];          // CACHED: order key of each column of the segment, 0 = invalid
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
@@ -234,7 +317,7 @@ topk_kernel(TopkArgs a) {
         hist_add(hist, (int)(key >> 20), key != 0u);
     }
     // Cluster histogram of the top 12 bits; its total is the number of candidates.
-    const int n_valid = cluster_threshold(cl, rank, hist, hsum, 4096, a.k, s_warp, &s_bin, &s_above);
+    const int n_valid = cluster_threshold_4096(cl, hist, s_sup, a.k, s_red, &s_bin, &s_above, &s_total);
     const bool take_all = n_valid <= a.k;
     const int a_lo = a.raw ? 0 : min(a.n_sink, pos + 1);
     const int b_hi = a.raw ? 0x7fffffff : (a.window > 0 ? max(a_lo, pos - a.window + 1) : pos + 1);
@@ -292,17 +375,20 @@ topk_kernel(TopkArgs a) {
                     dc[wb + i] = lcol[warp * kTopkWarpCap + i];
                 }
             }
+            // No peer reads `hist` any more (the count barrier above): CTA 0 clears its
+            // histograms for passes 2 and 3 while the candidates arrive.
+            if (rank == 0) {
+                for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
+                if (threadIdx.x < 256) hist3[threadIdx.x] = 0;
+            }
             cl.sync();                                   // every candidate has reached CTA 0
             if (rank != 0) return;
-            __syncthreads();
             const int n = total;
             uint32_t vs = 0;
-            int m_keep = 0;
+            int m_keep = 0, n_eq = 0;
             if (!take_all && a.k > 0) {
                 const uint32_t b1 = (uint32_t)s_bin;
                 int above = s_above;
-                for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
-                __syncthreads();
                 for (int i = threadIdx.x; i < n; i += kTopkThreads) {
                     const uint32_t key = ckey[i];
                     if ((key >> 20) == b1) atomicAdd(&hist[(key >> 8) & 0xfff], 1);
@@ -311,51 +397,70 @@ topk_kernel(TopkArgs a) {
                 local_threshold(hist, 4096, a.k - above, s_warp, &s_bin, &s_above);
                 const uint32_t pre = (b1 << 12) | (uint32_t)s_bin;
                 above += s_above;
-                for (int i = threadIdx.x; i < 256; i += kTopkThreads) hist[i] = 0;
-                __syncthreads();
                 for (int i = threadIdx.x; i < n; i += kTopkThreads) {
                     const uint32_t key = ckey[i];
-                    if ((key >> 8) == pre) atomicAdd(&hist[key & 0xff], 1);
+                    if ((key >> 8) == pre) atomicAdd(&hist3[key & 0xff], 1);
                 }
                 __syncthreads();
-                local_threshold(hist, 256, a.k - above, s_warp, &s_bin, &s_above);
+                local_threshold(hist3, 256, a.k - above, s_warp, &s_bin, &s_above);
                 above += s_above;
                 vs = (pre << 8) | (uint32_t)s_bin;
                 m_keep = a.k - above;                    // keys == vs to keep, lowest columns first
+                n_eq = hist3[s_bin];                     // keys == vs among the candidates
             }
             const bool every = take_all || a.k <= 0;     // every candidate is selected (none when k = 0)
-            // Emission in column order: thread = contiguous chunk of the candidates.
-            const int chunk = (n + kTopkThreads - 1) / kTopkThreads;
-            const int i0 = min(n, (int)threadIdx.x * chunk), i1 = min(n, i0 + chunk);
-            int eq_t = 0;
-            if (!every)
-                for (int i = i0; i < i1; ++i) eq_t += ckey[i] == vs;
-            int eq_tot;
-            const int eq_base = cta_inclusive_scan(eq_t, s_warp, eq_tot) - eq_t;
-            auto kept = [&](int i, int& eq_seen) -> bool {
-                const uint32_t key = ckey[i];
-                bool sel;
-                if (every) sel = a.k > 0;
-                else if (key > vs) sel = true;
-                else if (key == vs) sel = eq_base + eq_seen++ < m_keep;
-                else sel = false;
-                if (!sel) return false;
-                if (a.raw) return true;
-                const int p = position(ccol[i]);
-                return p >= a_lo && p < b_hi;
+            const bool ties_all = every || m_keep >= n_eq;
+            // Emission in column order: warp w owns a contiguous range of the candidates and walks
+            // it 32 at a time; in-warp ranks come from ballots, warp bases from per-warp counts.
+            const uint32_t lt = (1u << lane) - 1;
+            const int cw = ((n + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
+            const int e0 = min(n, warp * cw), e1 = min(n, e0 + cw);
+            int eq_base = 0;
+            if (!ties_all) {                             // ties at vs are cut: ranks among them needed
+                int c = 0;
+                for (int i = e0; i < e1; i += 32)
+                    c += __popc(__ballot_sync(0xffffffffu, i + lane < e1 && ckey[i + lane] == vs));
+                if (lane == 0) s_wcnt[warp] = c;
+                __syncthreads();
+                for (int w = 0; w < warp; ++w) eq_base += s_wcnt[w];
+            }
+            // kept(i): selected, and (unless raw) its position outside the sinks and the window.
+            auto walk = [&](bool write, int o) -> int {
+                int eq_run = eq_base, cnt = 0;
+                for (int i = e0; i < e1; i += 32) {
+                    const int ii = i + lane;
+                    const bool in = ii < e1;
+                    const uint32_t key = in ? ckey[ii] : 0u;
+                    bool keep;
+                    if (every) {
+                        keep = in && a.k > 0;
+                    } else {
+                        const bool eq = in && key == vs;
+                        const uint32_t em = ties_all ? 0u : __ballot_sync(0xffffffffu, eq);
+                        keep = in && (key > vs || (eq && (ties_all || eq_run + __popc(em & lt) < m_keep)));
+                        eq_run += __popc(em);
+                    }
+                    int pv = 0;
+                    if (keep) {
+                        pv = a.raw ? ccol[ii] : position(ccol[ii]);
+                        if (!a.raw) keep = pv >= a_lo && pv < b_hi;
+                    }
+                    const uint32_t km = __ballot_sync(0xffffffffu, keep);
+                    if (write && keep) out[o + cnt + __popc(km & lt)] = pv;
+                    cnt += __popc(km);
+                }
+                return cnt;
             };
-            int keep_t = 0;
-            {
-                int eq_seen = 0;
-                for (int i = i0; i < i1; ++i) keep_t += kept(i, eq_seen);
+            const int kept_w = walk(false, 0);
+            if (lane == 0) s_wk[warp] = kept_w;
+            __syncthreads();
+            int keep_base = 0, written = 0;
+            for (int w = 0; w < kTopkWarps; ++w) {
+                const int v = s_wk[w];
+                if (w < warp) keep_base += v;
+                written += v;
             }
-            int written;
-            const int keep_base = cta_inclusive_scan(keep_t, s_warp, written) - keep_t;
-            {
-                int eq_seen = 0, o = a_lo + keep_base;
-                for (int i = i0; i < i1; ++i)
-                    if (kept(i, eq_seen)) out[o++] = a.raw ? ccol[i] : position(ccol[i]);
-            }
+            walk(true, a_lo + keep_base);
             int n_out = a_lo + written;
             if (!a.raw) {
                 for (int i = threadIdx.x; i < a_lo; i += kTopkThreads) out[i] = i;

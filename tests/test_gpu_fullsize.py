@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 
 def _check(w, wt, pi, samples):
     p = w.passes[pi]
-    n_split = launch.split_for(w.T(p), w.H, w.cap)
+    n_split = launch.split_for(w.T(p), w.H, w.cap, layers=len(p.layers))
     step, ws, idx, cnt, layers = H.decode_step(wt, pi, n_split=n_split)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     step(ws, st)
