@@ -343,9 +343,10 @@ def run_gpu(args, rank, world, local_rank):
     # pinned host memory into one of two slots of device buffers, runs the fused calls on that
     # slot and copies every layer's output back to pinned host memory; the copies of one step
     # overlap the decode of its neighbours.  The timed region ends after the last step's copy-out.
-    pl = lsa.Pipeline(2, stream)
+    n_slots = max(2, args.slots)
+    pl = lsa.Pipeline(n_slots, stream)
     preps, h2d_bytes, d2h_bytes = [], 0, 0
-    for slot in range(2):
+    for slot in range(n_slots):
         decs, h2d, d2h = [], [], []
         for pi, pt in enumerate(wt.passes):
             sd = sds[pi]
@@ -366,7 +367,7 @@ def run_gpu(args, rank, world, local_rank):
 
     def e2e_run(n):
         for i in range(n):
-            pl.run(preps[i % 2])
+            pl.run(preps[i % n_slots])
         pl.join()
 
     e2e_run(4)
@@ -497,6 +498,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the sequence count (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--slots", type=int, default=2, help="device buffer slots of the host-buffer pipeline")
     ap.add_argument("--n-split", default="", help="override the split-KV chunk count: one value, or one per pass")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

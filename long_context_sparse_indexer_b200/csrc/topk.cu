@@ -9,7 +9,7 @@
 // Method: radix select on the order-preserving 32-bit key of each score, 12 + 12 + 8 bits.
 // One query row is handled by a cluster of kTopkCluster CTAs; CTA r owns the r-th
 // contiguous segment of the row.  Each pass builds integer shared-memory histograms of
-// its segment (warp-aggregated atomics; counts do not depend on atomic order), every CTA
+// its segment (shared-memory atomics; counts do not depend on atomic order), every CTA
 // then reads all the cluster's histograms through distributed shared memory and finds
 // the same threshold bin.  The result is the k-th key v* and the number m of ties at v*
 // to keep.  The emission pass keeps every key > v* and the first m keys == v* (lowest
