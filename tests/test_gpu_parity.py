@@ -149,6 +149,9 @@ def _host_score_rows(rng, T, n_cols, tie_levels):
 @pytest.mark.parametrize("n_cols,k,n_sink,window,tie_levels", [
     (5000, 256, 4, 128, 3), (5000, 256, 4, 128, 1000), (3000, 2048, 4, 512, 5), (100, 300, 4, 16, 2),
     (70000, 2048, 4, 512, 50), (4097, 0, 4, 128, 3), (4097, 33, 0, 0, 4),
+    # ~30000 keys share the threshold bin: more candidates than CTA 0's merged list holds, so
+    # the cluster finishes with the full passes over its segments
+    (70000, 2048, 4, 512, 2),
 ])
 def test_topk_matches_oracle_exactly(cuda, n_cols, k, n_sink, window, tie_levels):
     rng = np.random.default_rng(n_cols + k)
@@ -175,6 +178,30 @@ def test_topk_matches_oracle_exactly(cuda, n_cols, k, n_sink, window, tie_levels
         want = olsa.union_fixed(picks, int(pos[t]), n_sink, window)
         assert got[t].tolist() == want.tolist()
         assert np.all(idx[t, cnt[t]:].cpu().numpy() == -1)
+
+
+@pytest.mark.parametrize("n_cols", [3000, 70000])
+def test_topk_all_equal_scores(cuda, n_cols):
+    """Every visible score equal (as when every weighted ReLU sum is 0): the selection is the
+    k lowest positions, then the union with the sinks and the window."""
+    T, k, n_sink, window = 3, 2048, 4, 512
+    pos = np.array([n_cols - 1, n_cols // 3, 100])
+    s = np.zeros((T, n_cols), dtype=np.float32)
+    for t in range(T):
+        s[t, pos[t] + 1:] = -np.inf
+    batch = lsa.Batch(torch.tensor([n_cols], dtype=torch.int32, device="cuda"),
+                      torch.zeros(T, dtype=torch.int32, device="cuda"),
+                      torch.from_numpy(pos.astype(np.int32)).cuda(), n_cols)
+    idx = torch.empty((T, k + n_sink + window), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(T, dtype=torch.int32, device="cuda")
+    lsa.topk(batch, torch.from_numpy(s).cuda(), n_cols, k, n_sink, window, idx, cnt)
+    got = H.index_lists(idx, cnt)
+    for t in range(T):
+        cols = np.arange(pos[t] + 1)
+        picks = olsa.topk(s[t, cols].astype(np.float64), cols, k)
+        assert picks.tolist() == list(range(min(k, pos[t] + 1)))      # ties: lowest positions
+        want = olsa.union_fixed(picks, int(pos[t]), n_sink, window)
+        assert got[t].tolist() == want.tolist()
 
 
 def test_topk_raw_and_candidate_blocks(cuda):
