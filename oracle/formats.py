@@ -44,3 +44,21 @@ def decode_rows(data: np.ndarray, scale: np.ndarray | None) -> np.ndarray:
     if scale is None:
         return bf16_to_f64(data)
     return e4m3_to_f64(data, scale)
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Nearest e4m3 value to each float64 x, ties to the even mantissa, magnitudes beyond 448
+    saturated to 448 (round-to-nearest-even with saturation to the largest finite value).
+
+    The e4m3 grid from the definition above: in the binade [2**e, 2**(e+1)), e >= -6, the
+    values are spaced 2**(e-3); below 2**-6 the subnormals are spaced 2**-9.  Returns values,
+    not codes.  NaN stays NaN.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, E = np.frexp(np.where(a > 0, a, 1.0))          # a = f * 2**E with f in [0.5, 1)
+    e = np.maximum(E - 1, -6)                          # floor(log2 a), at least the smallest normal binade
+    quantum = np.ldexp(1.0, e - 3)
+    v = np.minimum(np.rint(a / quantum) * quantum, 448.0)   # np.rint: half to even
+    v = np.where(a > 0, v, 0.0)
+    return np.where(np.isnan(x), np.nan, np.copysign(v, x))

@@ -33,6 +33,32 @@ def indexer_scores(q: np.ndarray, w: np.ndarray, K: np.ndarray) -> np.ndarray:
     return np.maximum(logits, 0.0) @ np.asarray(w, dtype=np.float64)
 
 
+def fp8_queries(q: np.ndarray) -> np.ndarray:
+    """The indexer queries of the FP8-query mode: each row q_h (one head of one token) scaled by
+    the power of two 2**s that brings its largest magnitude m into [128, 256)
+    (s = 7 - floor(log2 m), clamped to [-126, 126]; s = 0 for an all-zero row), rounded to
+    e4m3 (``formats.e4m3_round``) and scaled back by 2**-s.
+
+    The DSA-style indexer usually runs its queries in FP8 ([release] "LongCat 稀疏注意力":
+    LSA grows out of DSA's lightning indexer, whose scoring cost is the bottleneck).  The pages
+    fix no quantisation; the per-row power-of-two scale is this library's reading (exact to
+    undo, so the score differs from the BF16-query score only by the e4m3 rounding of q).
+    q: [H_I, d_I] -> [H_I, d_I] float64.
+    """
+    from .formats import e4m3_round
+    q = np.asarray(q, dtype=np.float64)
+    m = np.max(np.abs(q), axis=-1)
+    _, E = np.frexp(np.where(m > 0, m, 1.0))
+    s = np.where(m > 0, np.clip(7 - (E - 1), -126, 126), 0)
+    sc = np.ldexp(1.0, s)[..., None]
+    return e4m3_round(q * sc) / sc
+
+
+def indexer_scores_fp8q(q: np.ndarray, w: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """``indexer_scores`` with the queries of the FP8-query mode (``fp8_queries``)."""
+    return indexer_scores(fp8_queries(q), w, K)
+
+
 def topk(scores: np.ndarray, positions: np.ndarray, k: int) -> np.ndarray:
     """The min(k, n) positions ranked first by (score descending, position ascending).
 

@@ -62,6 +62,68 @@ def test_scaled_rows_decode():
     assert np.array_equal(v, [[0.5, -0.5], [896.0, 2.0 ** -8]])
 
 
+def test_e4m3_round_matches_torch_float8():
+    rng = np.random.default_rng(3)
+    x = np.concatenate([
+        rng.normal(size=20000) * 40.0,                         # normals up to ~180
+        rng.uniform(-2.0 ** -5, 2.0 ** -5, size=20000),        # around and below the smallest normal
+        rng.uniform(-440.0, 440.0, size=5000),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(formats.e4m3_round(x.astype(np.float64)), ref)
+
+
+def test_e4m3_round_grid_and_ties():
+    t = formats.E4M3_TABLE
+    pos = np.sort(np.unique(t[np.isfinite(t) & (t >= 0)]))
+    assert np.array_equal(formats.e4m3_round(pos), pos)              # every value maps to itself
+    assert np.array_equal(formats.e4m3_round(-pos), -pos)
+    mids = (pos[:-1] + pos[1:]) / 2                                   # exact midpoints: ties to even code
+    got = formats.e4m3_round(mids)
+    code_of = {v: c for c, v in enumerate(t[:0x7F]) if np.isfinite(v)}
+    for lo, hi, g in zip(pos[:-1], pos[1:], got):
+        even = lo if code_of[lo] % 2 == 0 else hi
+        assert g == even, (lo, hi, g)
+    assert formats.e4m3_round(np.array([500.0, -1e6]))[0] == 448.0     # saturation
+    assert formats.e4m3_round(np.array([-1e6]))[0] == -448.0
+    assert formats.e4m3_round(np.array([2.0 ** -10]))[0] == 0.0         # half the smallest subnormal: tie to 0
+
+
+def test_fp8_queries_scale_and_error_bound():
+    rng = np.random.default_rng(4)
+    # rows of very different magnitudes: the scale is per row (head), not per token
+    q = rng.normal(size=(6, 128)) * np.array([1e3, 1.0, 1e-3, 3.0, 1e-6, 0.0])[:, None]
+    q8 = lsa.fp8_queries(q)
+    for h in range(6):
+        m = np.abs(q[h]).max()
+        if m == 0:
+            assert np.all(q8[h] == 0)
+            continue
+        s = 7 - math.floor(math.log2(m))
+        assert 128 <= m * 2.0 ** s < 256
+        big = np.abs(q[h]) * 2.0 ** s >= 2.0 ** -6                   # normal after scaling
+        err = np.abs(q8[h] - q[h])
+        assert np.all(err[big] <= 2.0 ** -4 * np.abs(q[h][big]))      # 3 mantissa bits, round to nearest
+        assert np.all(err[~big] <= 2.0 ** -10 * 2.0 ** -s)            # half a subnormal step
+    assert np.abs(q8[0] - q[0]).max() > 0                             # it does round
+
+
+def test_fp8_query_scores_on_representable_queries():
+    rng = np.random.default_rng(5)
+    # entries k / 4 with |k| <= 15: exactly representable after any power-of-two scale that
+    # keeps the row maximum in [128, 256) (4 significant bits), so the rounding is the identity
+    q = rng.integers(-15, 16, size=(8, 128)) / 4.0 * np.array([2.0 ** j for j in range(-3, 5)])[:, None]
+    q[:, 0] = 3.75 * np.array([2.0 ** j for j in range(-3, 5)])           # a known maximum per row
+    K = rng.normal(size=(50, 128))
+    w = rng.normal(size=8)
+    assert np.array_equal(lsa.fp8_queries(q), q)
+    assert np.array_equal(lsa.indexer_scores_fp8q(q, w, K), lsa.indexer_scores(q, w, K))
+    # and a query that is not representable scores differently
+    q2 = q.copy()
+    q2[:, 1] = 0.123456
+    assert not np.array_equal(lsa.indexer_scores_fp8q(q2, w, K), lsa.indexer_scores(q2, w, K))
+
+
 # ------------------------------------------------------------------ worked example
 
 def test_worked_indexer():
