@@ -119,7 +119,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the GPU arm
 
-def build_step(w, wt, pi, n_split):
+def build_step(w, wt, pi, n_split, q8=False):
     from long_context_sparse_indexer_b200 import lsa
     pt = wt.passes[pi]
     p = w.passes[pi]
@@ -141,9 +141,9 @@ def build_step(w, wt, pi, n_split):
     cnt = torch.empty((T,), dtype=torch.int32, device=dev)
     step = lsa.DecodeStep(batch, pt.q_idx, pt.w, lsa.Cache(pt.k_idx, pt.k_scale), w.k, w.n_sink, w.window, layers,
                           w.H, w.D, w.Dv, w.sm_scale, n_split=n_split, hi=w.hi, block_size=w.block_size,
-                          n_recall=w.n_recall, kbar=kbar, idx_out=idx, count_out=cnt)
+                          n_recall=w.n_recall, kbar=kbar, idx_out=idx, count_out=cnt, idx_q_fp8=q8)
     ws = torch.empty(max(256, step.workspace_size()), dtype=torch.uint8, device=dev)
-    return dict(step=step, ws=ws, idx=idx, cnt=cnt, layers=layers, batch=batch, kbar=kbar, T=T, n_split=n_split)
+    return dict(step=step, ws=ws, idx=idx, cnt=cnt, layers=layers, batch=batch, kbar=kbar, T=T, n_split=n_split, q8=q8)
 
 
 def slot_copy(w, wt, pi, sd):
@@ -160,7 +160,8 @@ def slot_copy(w, wt, pi, sd):
         layers.append(lsa.Layer(q, Ls.kv, torch.empty_like(Ls.o), torch.empty_like(Ls.lse), Ls.v))
     step = lsa.DecodeStep(sd["batch"], q_idx, wv, lsa.Cache(pt.k_idx, pt.k_scale), w.k, w.n_sink, w.window, layers,
                           w.H, w.D, w.Dv, w.sm_scale, n_split=sd["n_split"], hi=w.hi, block_size=w.block_size,
-                          n_recall=w.n_recall, kbar=sd["kbar"], idx_out=sd["idx"], count_out=sd["cnt"])
+                          n_recall=w.n_recall, kbar=sd["kbar"], idx_out=sd["idx"], count_out=sd["cnt"],
+                          idx_q_fp8=sd["q8"])
     return step, [q_idx, wv] + qs, [L.o for L in layers]
 
 
@@ -255,7 +256,7 @@ def run_gpu(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     forced = [int(x) for x in args.n_split.split(",")] if args.n_split else []
     sds = [build_step(w, wt, pi, forced[min(pi, len(forced) - 1)] if forced
-                      else launch.split_for(w.T(p), w.H, w.cap, layers=len(p.layers)))
+                      else launch.split_for(w.T(p), w.H, w.cap, layers=len(p.layers)), q8=args.idx_q8)
            for pi, p in enumerate(w.passes)]
 
     def step():
@@ -308,8 +309,8 @@ def run_gpu(args, rank, world, local_rank):
         ld = (wt.L_alloc + 3) // 4 * 4
         sc = torch.empty((sd0["T"], ld), dtype=torch.float32, device=dev)
         idx_fn = lambda: lsa.index_score(sd0["batch"], pt0.q_idx, pt0.w, k_cache, sc, n_cols=wt.L_alloc,  # noqa
-                                         stream=stream)
-        kern = "index_score (flat indexer)"
+                                         stream=stream, q_fp8=args.idx_q8)
+        kern = "index_score (flat indexer, FP8 queries)" if args.idx_q8 else "index_score (flat indexer)"
     else:
         nblk = (wt.L_alloc + w.block_size - 1) // w.block_size
         sc = torch.empty((sd0["T"], (nblk + 3) // 4 * 4), dtype=torch.float32, device=dev)
@@ -389,6 +390,7 @@ def run_gpu(args, rank, world, local_rank):
                    "queries_per_step_per_gpu": q_per_step, "ctx": [int(W.lengths(w).min()), int(W.lengths(w).max())],
                    "k": w.k, "n_sink": w.n_sink, "window": w.window, "hi": w.hi,
                    "layers_per_index": [len(p.layers) for p in w.passes],
+                   "indexer_queries": "fp8 (per-head power-of-two scale)" if args.idx_q8 else "bf16 (exact)",
                    "n_split": [sd["n_split"] for sd in sds], "parallelism": f"replicas x{world} (batch per GPU)",
                    "launch": "cuda_graph" if graph is not None else "eager",
                    "l2": "inputs larger than L2 (indexer keys + selected KV rows per step >> 126 MB)"},
@@ -499,6 +501,7 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the sequence count (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--slots", type=int, default=2, help="device buffer slots of the host-buffer pipeline")
+    ap.add_argument("--idx-q8", action="store_true", help="indexer in FP8-query mode (lsa_index_score_q8)")
     ap.add_argument("--n-split", default="", help="override the split-KV chunk count: one value, or one per pass")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

@@ -107,6 +107,18 @@ lsa_status lsa_index_score(const lsa_batch* batch, const void* q_idx, const floa
                            int block_size, float* scores, int64_t ld_scores, int n_cols,
                            int32_t* dev_status, void* stream);
 
+/* lsa_index_score in FP8-query mode: the DSA-style indexer's e4m3 queries.  Each row
+ * q_idx[t,h,:] is scaled by the power of two 2^s (s = 7 - floor(log2 max|q_idx[t,h,:]|),
+ * clamped to [-126, 126]; 0 for an all-zero row), rounded to e4m3 (nearest, ties to even,
+ * saturating) and scaled back, and the scores use those queries: half the tensor-core work of
+ * the exact BF16-query mode.  Same arguments and results otherwise.  Needs the tensor-core
+ * path (FP8 keys, d_I = 128, H_I a multiple of 32, block_size 64 for HI); returns
+ * LSA_ERR_UNSUPPORTED elsewhere. */
+lsa_status lsa_index_score_q8(const lsa_batch* batch, const void* q_idx, const float* w, int H_I,
+                              const lsa_cache* k_idx, const int32_t* cand_blocks, int n_cand,
+                              int block_size, float* scores, int64_t ld_scores, int n_cols,
+                              int32_t* dev_status, void* stream);
+
 /* ---------------------------------------------------------------- a2: HI block keys
  * Block key of block j of sequence b = arithmetic mean of the dequantised indexer keys
  * of rows j*block_size .. min(seq_len[b], (j+1)*block_size) - 1 ([release] HI bullet:
@@ -228,6 +240,9 @@ typedef struct {
     int32_t*         idx_out;
     int64_t          idx_ld;
     int32_t*         count_out;
+    /* indexer queries: 0 = BF16 (exact), 1 = FP8-query mode (as lsa_index_score_q8; flat and
+     * the fine stage of HI -- HI block scores keep the BF16 queries) */
+    int32_t          idx_q_fp8;
 } lsa_decode_params;
 
 /* Runs indexer (flat, or HI: block scores -> recall -> fine scores), top-k + union, then

@@ -57,7 +57,8 @@ IndexArgs make_index_args(const lsa_batch* batch, const void* q_idx, const float
 
 lsa_status index_score_impl(const lsa_batch* batch, const void* q_idx, const float* w, int H_I,
                             const lsa_cache* k_idx, const int32_t* cand, int n_cand, int block_size,
-                            float* scores, int64_t ld, int n_cols, int32_t* st, cudaStream_t stream) {
+                            float* scores, int64_t ld, int n_cols, int32_t* st, cudaStream_t stream,
+                            bool q_fp8 = false) {
     lsa_status s = check_batch(batch);
     if (s != LSA_OK) return s;
     if ((s = check_cache(k_idx, 0)) != LSA_OK) return s;
@@ -71,6 +72,9 @@ lsa_status index_score_impl(const lsa_batch* batch, const void* q_idx, const flo
         if (n_cols < 0 || n_cols > ld || n_cols > batch->L_alloc) return LSA_ERR_INVALID_ARG;
     }
     IndexArgs a = make_index_args(batch, q_idx, w, k_idx, cand, n_cand, block_size, scores, ld, n_cols, st);
+    a.q_fp8 = q_fp8 ? 1 : 0;
+    // The FP8-query mode exists on the tensor-core path only.
+    if (q_fp8 && !index_score_tc_supported(a, H_I, k_idx->dim, k_idx->dtype == LSA_FP8_E4M3)) return LSA_ERR_UNSUPPORTED;
     return cuda_status(launch_index_score(a, H_I, k_idx->dim, k_idx->dtype == LSA_FP8_E4M3, stream));
 }
 
@@ -220,6 +224,13 @@ lsa_status lsa_index_score(const lsa_batch* batch, const void* q_idx, const floa
                             n_cols, dev_status, static_cast<cudaStream_t>(stream));
 }
 
+lsa_status lsa_index_score_q8(const lsa_batch* batch, const void* q_idx, const float* w, int H_I,
+                              const lsa_cache* k_idx, const int32_t* cand_blocks, int n_cand, int block_size,
+                              float* scores, int64_t ld_scores, int n_cols, int32_t* dev_status, void* stream) {
+    return index_score_impl(batch, q_idx, w, H_I, k_idx, cand_blocks, n_cand, block_size, scores, ld_scores,
+                            n_cols, dev_status, static_cast<cudaStream_t>(stream), true);
+}
+
 lsa_status lsa_block_keys(const lsa_batch* batch, const lsa_cache* k_idx, int block_size, float* kbar,
                           int64_t kbar_seq_stride, int32_t* dev_status, void* stream) {
     lsa_status s = check_batch(batch);
@@ -313,7 +324,7 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
 
     if (!p->hi) {
         s = index_score_impl(batch, p->q_idx, p->w, p->H_I, &p->k_idx, nullptr, 0, 0, scores, f.ld, f.n_cols,
-                             dev_status, st);
+                             dev_status, st, p->idx_q_fp8 != 0);
         if (s != LSA_OK) return s;
         s = topk_impl(batch, scores, f.ld, f.n_cols, nullptr, 0, 0, p->k, p->n_sink, p->window, 0, idx, ld_idx,
                       count, dev_status, st);
@@ -329,7 +340,7 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
                       p->n_recall, ccount, dev_status, st);
         if (s != LSA_OK) return s;
         s = index_score_impl(batch, p->q_idx, p->w, p->H_I, &p->k_idx, cand, p->n_recall, p->block_size, scores,
-                             f.ld, 0, dev_status, st);
+                             f.ld, 0, dev_status, st, p->idx_q_fp8 != 0);
         if (s != LSA_OK) return s;
         s = topk_impl(batch, scores, f.ld, f.n_cols, cand, p->n_recall, p->block_size, p->k, p->n_sink, p->window,
                       0, idx, ld_idx, count, dev_status, st);

@@ -14,6 +14,10 @@
 // against hi then lo), so the FP32 accumulator holds 2^s_h (q_h . k); products of e4m3 values are
 // exact.  2^-s_h is folded into the head weight.
 //
+// FP8-query mode (IndexArgs::q_fp8): the query row is hi alone, rn(q_h 2^s_h) 2^-s_h, the
+// per-(token, head) e4m3 query of the DSA-style indexer; the MMA runs over K = 128, half the
+// tensor-core work.  Scores then differ from the BF16-query ones by the rounding of q.
+//
 // Scheduling.  Query tokens come in groups of G <= 4 tokens of one sequence (N = G*H_I <= 256
 // query rows share every key row).  A group's key range is cut into 128-key tiles; only tiles
 // holding a visible key are active.  Every CTA counts the active tiles of all groups, takes an
@@ -24,7 +28,7 @@
 //   warp 0      : TMA producer -- key tiles (two 64-row boxes, 128-byte swizzle, which is the
 //                 K-major operand layout) and their per-token scales into a KS-stage ring;
 //                 allocates / frees TMEM.
-//   warp 1      : MMA issuer -- per tile, 8 x tcgen05.mma kind::f8f6f4 (M = 128 keys, N, K = 32)
+//   warp 1      : MMA issuer -- per tile, 8 (FP8 queries: 4) x tcgen05.mma kind::f8f6f4 (M = 128 keys, N, K = 32)
 //                 into one of 512 / N accumulator slots; its commit frees the key stage.
 //   warps 2..3  : query preparation, once per epoch (hi / lo split, 128-byte-swizzled K-major).
 //   warps 4..11 : epilogue, two warpgroups taking alternate tiles -- thread = key row (= TMEM
@@ -197,8 +201,9 @@ __device__ void prepare_queries(const IndexArgs& a, int t0, int H_I, int ct, int
                 const float x0 = v[4 * e] * sc, x1 = v[4 * e + 1] * sc, x2 = v[4 * e + 2] * sc, x3 = v[4 * e + 3] * sc;
                 const uint16_t h01 = f32x2_to_e4m3x2(x0, x1), h23 = f32x2_to_e4m3x2(x2, x3);
                 const float2 d01 = e4m3x2_to_f32x2(h01), d23 = e4m3x2_to_f32x2(h23);
-                const uint16_t l01 = f32x2_to_e4m3x2(x0 - d01.x, x1 - d01.y);
-                const uint16_t l23 = f32x2_to_e4m3x2(x2 - d23.x, x3 - d23.y);
+                // FP8-query mode: the row is its rounded hi part alone (lo is never read).
+                const uint16_t l01 = a.q_fp8 ? 0 : f32x2_to_e4m3x2(x0 - d01.x, x1 - d01.y);
+                const uint16_t l23 = a.q_fp8 ? 0 : f32x2_to_e4m3x2(x2 - d23.x, x3 - d23.y);
                 hw[e] = (uint32_t)h01 | ((uint32_t)h23 << 16);
                 lw[e] = (uint32_t)l01 | ((uint32_t)l23 << 16);
             }
@@ -381,6 +386,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         // 128-byte swizzled row starts kk * 32 bytes in, i.e. 2 * kk in the descriptor's address
         // field, which cannot carry since shared addresses are below 256 KB)
         const uint32_t idesc = tc::idesc_f16(128, N, 0);      // e4m3 x e4m3 -> f32, both K-major
+        const int n_k8 = a.q_fp8 ? 4 : 8;                      // FP8-query mode: no lo half
         if (tc::elect_one()) {
             const uint64_t da0 = tc::sdesc_sw128(tc::smem_u32(sm.keys[0]));
             const uint64_t dh0 = tc::sdesc_sw128(tc::smem_u32(sm.q[0][0])), dl0 = tc::sdesc_sw128(tc::smem_u32(sm.q[0][1]));
@@ -399,8 +405,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                     const uint64_t da = da0 + (uint64_t)((s * NB + b) * (kBlockBytes >> 4));
                     const uint32_t dc = d_col + slot * SW + b * N;
 #pragma unroll
-                    for (int k8 = 0; k8 < 8; ++k8)
-                        tc::mma_f8_ss(dc, da + 2 * (k8 & 3), (k8 < 4 ? dh : dl) + 2 * (k8 & 3), idesc, k8 > 0);
+                    for (int k8 = 0; k8 < 8; ++k8)               // K steps 0..3: q_hi; 4..7: q_lo
+                        if (k8 < n_k8)
+                            tc::mma_f8_ss(dc, da + 2 * (k8 & 3), (k8 < 4 ? dh : dl) + 2 * (k8 & 3), idesc, k8 > 0);
                 }
                 tc::mma_commit(&sm.empty_k[s]);
                 tc::mma_commit(&sm.d_full[slot]);

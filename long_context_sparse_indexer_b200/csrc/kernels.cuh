@@ -21,6 +21,7 @@ struct IndexArgs {
     int64_t ld;
     int n_cols;              // columns to write
     int group;               // tokens per CTA (<= 4)
+    int q_fp8;               // 1: FP8-query mode (queries rounded once to e4m3, tensor-core path only)
     int32_t* status;
 };
 

@@ -57,12 +57,13 @@ class CDecodeParams(ctypes.Structure):
                 ("kbar_seq_stride", c_i64),
                 ("H", c_i32), ("Dqk", c_i32), ("Dv", c_i32), ("sm_scale", c_f32), ("n_split", c_i32),
                 ("n_layers", c_i32), ("layers", ctypes.POINTER(CLayer)),
-                ("idx_out", c_vp), ("idx_ld", c_i64), ("count_out", c_vp)]
+                ("idx_out", c_vp), ("idx_ld", c_i64), ("count_out", c_vp), ("idx_q_fp8", c_i32)]
 
 
 _P = ctypes.POINTER
 _lib.lsa_index_score.argtypes = [_P(CBatch), c_vp, c_vp, c_i32, _P(CCache), c_vp, c_i32, c_i32, c_vp, c_i64,
                                  c_i32, c_vp, c_vp]
+_lib.lsa_index_score_q8.argtypes = _lib.lsa_index_score.argtypes
 _lib.lsa_block_keys.argtypes = [_P(CBatch), _P(CCache), c_i32, c_vp, c_i64, c_vp, c_vp]
 _lib.lsa_block_score.argtypes = [_P(CBatch), c_vp, c_vp, c_i32, c_i32, c_vp, c_i64, c_i32, c_vp, c_i64, c_i32,
                                  c_vp, c_vp]
@@ -92,11 +93,11 @@ _lib.lsa_pipeline_destroy.argtypes = [c_vp]
 _lib.lsa_status_string.argtypes = [c_i32]
 _lib.lsa_status_string.restype = ctypes.c_char_p
 _lib.lsa_version.restype = c_i32
-for _f in ("lsa_index_score", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
+for _f in ("lsa_index_score", "lsa_index_score_q8", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
            "lsa_sparse_attn_noalloc", "lsa_decode_fused", "lsa_read_device_status"):
     getattr(_lib, _f).restype = c_i32
 
-EXPORTS = ("lsa_index_score", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
+EXPORTS = ("lsa_index_score", "lsa_index_score_q8", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
            "lsa_sparse_attn_noalloc", "lsa_attn_workspace_size", "lsa_decode_fused", "lsa_decode_workspace_size", "lsa_read_device_status",
            "lsa_status_string", "lsa_version", "lsa_pipeline_create", "lsa_pipeline_step", "lsa_pipeline_join",
            "lsa_pipeline_destroy")
@@ -166,13 +167,15 @@ _EMPTY_CACHE = CCache(None, None, 0, 0, 0, 0, 0)
 
 def index_score(batch: Batch, q_idx: torch.Tensor, w: torch.Tensor, k_idx: Cache, scores: torch.Tensor,
                 n_cols: int = 0, cand_blocks: Optional[torch.Tensor] = None, block_size: int = 0,
-                dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
-    """lsa_index_score: flat scores (cand_blocks None) or HI fine scores over recalled blocks."""
+                dev_status: Optional[torch.Tensor] = None, stream=None, q_fp8: bool = False) -> None:
+    """lsa_index_score (lsa_index_score_q8 with q_fp8): flat scores (cand_blocks None) or HI fine
+    scores over recalled blocks."""
     cb, ck = batch.c(), k_idx.c()
     n_cand = int(cand_blocks.shape[1]) if cand_blocks is not None else 0
-    _check(_lib.lsa_index_score(ctypes.byref(cb), _ptr(q_idx), _ptr(w), int(q_idx.shape[1]), ctypes.byref(ck),
-                                _ptr(cand_blocks), n_cand, int(block_size), _ptr(scores), int(scores.stride(0)),
-                                int(n_cols), _ptr(dev_status), _stream(stream)), "lsa_index_score")
+    fn, name = (_lib.lsa_index_score_q8, "lsa_index_score_q8") if q_fp8 else (_lib.lsa_index_score, "lsa_index_score")
+    _check(fn(ctypes.byref(cb), _ptr(q_idx), _ptr(w), int(q_idx.shape[1]), ctypes.byref(ck),
+              _ptr(cand_blocks), n_cand, int(block_size), _ptr(scores), int(scores.stride(0)),
+              int(n_cols), _ptr(dev_status), _stream(stream)), name)
 
 
 def block_keys(batch: Batch, k_idx: Cache, block_size: int, kbar: torch.Tensor,
@@ -256,7 +259,8 @@ class DecodeStep:
     def __init__(self, batch: Batch, q_idx: torch.Tensor, w: torch.Tensor, k_idx: Cache, k: int, n_sink: int,
                  window: int, layers: Sequence[Layer], H: int, Dqk: int, Dv: int, sm_scale: float, n_split: int = 1,
                  hi: bool = False, block_size: int = 64, n_recall: int = 0, kbar: Optional[torch.Tensor] = None,
-                 idx_out: Optional[torch.Tensor] = None, count_out: Optional[torch.Tensor] = None):
+                 idx_out: Optional[torch.Tensor] = None, count_out: Optional[torch.Tensor] = None,
+                 idx_q_fp8: bool = False):
         self._keep = (batch, q_idx, w, k_idx, list(layers), kbar, idx_out, count_out)
         arr = (CLayer * max(1, len(layers)))()
         for i, L in enumerate(layers):
@@ -266,7 +270,8 @@ class DecodeStep:
                                int(window), int(bool(hi)), int(block_size), int(n_recall), _ptr(kbar),
                                int(kbar.stride(0)) if kbar is not None else 0, int(H), int(Dqk), int(Dv),
                                float(sm_scale), int(n_split), len(layers), arr, _ptr(idx_out),
-                               int(idx_out.stride(0)) if idx_out is not None else 0, _ptr(count_out))
+                               int(idx_out.stride(0)) if idx_out is not None else 0, _ptr(count_out),
+                               int(bool(idx_q_fp8)))
 
     def workspace_size(self) -> int:
         return int(_lib.lsa_decode_workspace_size(ctypes.byref(self.p)))

@@ -25,12 +25,13 @@ def kv_cache(wt: D.WorkloadTensors, pi: int, li: int):
     return lsa.Cache(L["kv"], L["kv_scale"]), (lsa.Cache(L["v"]) if L["v"] is not None else None)
 
 
-def flat_scores(wt: D.WorkloadTensors, pi: int = 0, status=None) -> torch.Tensor:
+def flat_scores(wt: D.WorkloadTensors, pi: int = 0, status=None, q_fp8: bool = False) -> torch.Tensor:
     pt = wt.passes[pi]
     T = pt.q_idx.shape[0]
     ld = (wt.L_alloc + 3) // 4 * 4
     sc = torch.full((T, ld), float("nan"), dtype=torch.float32, device=pt.q_idx.device)
-    lsa.index_score(batch_of(wt, pi), pt.q_idx, pt.w, idx_cache(wt, pi), sc, n_cols=wt.L_alloc, dev_status=status)
+    lsa.index_score(batch_of(wt, pi), pt.q_idx, pt.w, idx_cache(wt, pi), sc, n_cols=wt.L_alloc, dev_status=status,
+                    q_fp8=q_fp8)
     return sc
 
 
@@ -42,7 +43,8 @@ def block_keys(wt: D.WorkloadTensors, pi: int = 0, status=None) -> torch.Tensor:
     return kbar
 
 
-def decode_step(wt: D.WorkloadTensors, pi: int = 0, n_split: int = 1, kbar=None, cap_extra: int = 0):
+def decode_step(wt: D.WorkloadTensors, pi: int = 0, n_split: int = 1, kbar=None, cap_extra: int = 0,
+                idx_q_fp8: bool = False):
     """Builds lsa.DecodeStep for a pass plus its output tensors."""
     w = wt.w
     pt = wt.passes[pi]
@@ -61,7 +63,7 @@ def decode_step(wt: D.WorkloadTensors, pi: int = 0, n_split: int = 1, kbar=None,
         kbar = block_keys(wt, pi)
     step = lsa.DecodeStep(batch_of(wt, pi), pt.q_idx, pt.w, idx_cache(wt, pi), w.k, w.n_sink, w.window, layers,
                           w.H, w.D, w.Dv, w.sm_scale, n_split=n_split, hi=w.hi, block_size=w.block_size,
-                          n_recall=w.n_recall, kbar=kbar, idx_out=idx, count_out=cnt)
+                          n_recall=w.n_recall, kbar=kbar, idx_out=idx, count_out=cnt, idx_q_fp8=idx_q_fp8)
     ws = torch.empty(max(256, step.workspace_size()), dtype=torch.uint8, device=dev)
     return step, ws, idx, cnt, layers
 

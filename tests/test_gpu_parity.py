@@ -114,6 +114,98 @@ def test_flat_index_scores(cuda, name):
             assert np.all(np.isneginf(sc[t, pos + 1:wt.L_alloc]))
 
 
+# The FP8-query mode needs the tensor-core indexer (FP8 keys, d_I = 128, H_I a multiple of 32).
+Q8 = ["cli_small", "mtp_small", "prefill_small", "cli_unaligned"]
+
+
+@pytest.mark.parametrize("name", Q8)
+def test_fp8_query_index_scores(cuda, name):
+    """FP8-query mode against the oracle's FP8-query scores (same query rounding; products of
+    e4m3 values are exact, so only the FP32 accumulation differs), and visibly different from
+    the exact BF16-query scores."""
+    w = SMALL[name]
+    wt = wt_of(name)
+    for pi, p in enumerate(w.passes):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sc = H.flat_scores(wt, pi, st, q_fp8=True).cpu().numpy().astype(np.float64)
+        assert lsa.read_device_status(st) == lsa.OK
+        plan = W.plant_plan(w, p) if p.name == "target" and (w.plant_frac or w.plant_blocks) else None
+        moved = 0.0
+        for t in tokens_to_check(w, p):
+            b, pos, L, qi, wi = run.query_context(w, p, t)
+            K = run.index_keys(w, p, b, np.arange(pos + 1), plan)
+            ref = olsa.indexer_scores_fp8q(qi, wi, K)
+            assert H.score_close(sc[t, :pos + 1], ref) < 1e-4
+            assert np.all(np.isneginf(sc[t, pos + 1:wt.L_alloc]))
+            moved = max(moved, H.score_close(olsa.indexer_scores(qi, wi, K), ref))
+        assert moved > 1e-3                      # the rounding of q is real: the mode changes the scores
+
+
+def test_fp8_query_mode_unsupported_shapes(cuda):
+    for name in ("tiny_decode", "cli_d64"):
+        wt = wt_of(name)
+        with pytest.raises(lsa.LsaError) as e:
+            H.flat_scores(wt, 0, q_fp8=True)
+        assert e.value.status == lsa.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name", ["cli_small", "mtp_small"])
+def test_fp8_query_fused_selection(cuda, name):
+    """The fused step in FP8-query mode selects what the oracle's top-k selects on the GPU's own
+    FP8-query scores, and its attention matches the oracle on that index list."""
+    w = SMALL[name]
+    wt = wt_of(name)
+    p = w.passes[0]
+    sc = H.flat_scores(wt, 0, q_fp8=True).cpu().numpy().astype(np.float64)
+    step, ws, idx, cnt, layers = H.decode_step(wt, 0, n_split=2, idx_q_fp8=True)
+    step(ws)
+    got = H.index_lists(idx, cnt)
+    _, q_pos = W.query_rows(w, p)
+    for t in range(w.T(p)):
+        pos = int(q_pos[t])
+        picks = olsa.topk(sc[t, :pos + 1], np.arange(pos + 1), w.k)
+        assert got[t].tolist() == olsa.union_fixed(picks, pos, w.n_sink, w.window).tolist()
+
+
+def test_hi_fine_scores_fp8_query(cuda):
+    """HI fine stage in FP8-query mode: scores over recalled blocks equal the oracle's FP8-query
+    scores at the blocks' positions."""
+    w = SMALL["hi_small"]
+    wt = wt_of("hi_small")
+    p = w.passes[0]
+    pt = wt.passes[0]
+    T = pt.q_idx.shape[0]
+    nblk = (wt.L_alloc + w.block_size - 1) // w.block_size
+    n_cand = 6
+    cand = torch.full((T, n_cand), -1, dtype=torch.int32)
+    _, q_pos = W.query_rows(w, p)
+    for t in range(T):
+        vis = int(q_pos[t]) // w.block_size + 1
+        picks = sorted({0, vis - 1, vis // 2, vis // 3, max(0, vis - 7)})
+        cand[t, :len(picks)] = torch.tensor(picks, dtype=torch.int32)
+    cand = cand.cuda()
+    sc = torch.empty((T, n_cand * w.block_size), dtype=torch.float32, device="cuda")
+    lsa.index_score(H.batch_of(wt), pt.q_idx, pt.w, H.idx_cache(wt), sc, cand_blocks=cand, block_size=w.block_size,
+                    q_fp8=True)
+    sc = sc.cpu().numpy().astype(np.float64)
+    cand = cand.cpu().numpy()
+    plan = W.plant_plan(w, p)
+    assert nblk >= n_cand
+    for t in tokens_to_check(w, p):
+        b, pos, L, qi, wi = run.query_context(w, p, t)
+        for j, blk in enumerate(cand[t]):
+            cols = sc[t, j * w.block_size:(j + 1) * w.block_size]
+            if blk < 0:
+                assert np.all(np.isneginf(cols))
+                continue
+            rows = np.arange(blk * w.block_size, (blk + 1) * w.block_size)
+            vis = rows <= pos
+            K = run.index_keys(w, p, b, rows[vis], plan)
+            ref = olsa.indexer_scores_fp8q(qi, wi, K)
+            assert H.score_close(cols[vis], ref) < 1e-4
+            assert np.all(np.isneginf(cols[~vis]))
+
+
 def test_block_keys_and_block_scores(cuda):
     w = SMALL["hi_small"]
     wt = wt_of("hi_small")
