@@ -89,6 +89,26 @@ def union_fixed(selected: np.ndarray, pos: int, n_sink: int, window: int) -> np.
     return np.union1d(np.union1d(np.asarray(selected, dtype=np.int64), sinks), win)
 
 
+def union_fixed_budget(scores: np.ndarray, positions: np.ndarray, k: int, pos: int, n_sink: int,
+                       window: int) -> np.ndarray:
+    """Fixed-budget SI selection: the sinks and the window as in ``union_fixed``, plus the top-k
+    (``topk`` order) of the visible positions OUTSIDE both, so the three sets are disjoint and
+    the list holds min(k, outside) + |sinks| + |window| positions, ascending.
+
+    [release] SI bullet: the selection budget is split between a contiguous, hardware-aligned
+    part and the dynamic picks.  Read as a budget, the dynamic part should not spend picks on
+    positions the fixed part already holds; ``union_fixed`` is the other reading (top-k over all
+    visible positions, then the union).  scores / positions: the visible keys (any order).
+    """
+    scores = np.asarray(scores, dtype=np.float64)
+    positions = np.asarray(positions, dtype=np.int64)
+    a = min(n_sink, pos + 1)
+    b = max(a, pos - window + 1) if window > 0 else pos + 1
+    outside = (positions >= a) & (positions < b)
+    picks = topk(scores[outside], positions[outside], k)
+    return union_fixed(picks, pos, n_sink, window)
+
+
 def block_keys(K: np.ndarray, length: int, block_size: int) -> np.ndarray:
     """Block key = arithmetic mean of the (dequantised) keys of the block's existing tokens.
 

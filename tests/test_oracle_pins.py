@@ -354,3 +354,38 @@ def test_hi_candidates_are_whole_recalled_blocks():
     J = lsa.indexer_scores(q, w, kbar[:250 // bs + 1])
     best = sorted(np.argsort(-J, kind="stable")[:3].tolist())
     assert blocks == best
+
+
+# ------------------------------------------------------------------ fixed-budget SI selection
+
+def test_fixed_budget_union_brute_force():
+    rng = np.random.default_rng(11)
+    for trial in range(300):
+        n = int(rng.integers(1, 40))
+        pos = int(rng.integers(0, n))
+        k = int(rng.integers(0, 12))
+        n_sink = int(rng.integers(0, 5))
+        window = int(rng.integers(0, 8))
+        sc = rng.integers(0, 4, size=pos + 1).astype(np.float64)       # many ties
+        got = lsa.union_fixed_budget(sc, np.arange(pos + 1), k, pos, n_sink, window)
+        sinks = set(range(min(n_sink, pos + 1)))
+        win = set(range(max(0, pos - window + 1), pos + 1)) if window > 0 else set()
+        rest = [j for j in range(pos + 1) if j not in sinks and j not in win]
+        # brute force: rank the rest by (score desc, position asc), take k
+        best = sorted(rest, key=lambda j: (-sc[j], j))[:k]
+        want = sorted(sinks | win | set(best))
+        assert got.tolist() == want
+        assert len(got) == len(sinks | win) + min(k, len(rest))          # exact budget, disjoint parts
+
+
+def test_fixed_budget_equals_plain_union_when_picks_avoid_the_fixed_sets():
+    pos, k, n_sink, window = 999, 50, 4, 100
+    sc = np.zeros(pos + 1)
+    sc[300:350] = 10.0 + np.arange(50)                 # the top-50 lie outside sinks and window
+    cols = np.arange(pos + 1)
+    plain = lsa.union_fixed(lsa.topk(sc, cols, k), pos, n_sink, window)
+    assert np.array_equal(lsa.union_fixed_budget(sc, cols, k, pos, n_sink, window), plain)
+    sc[995] = 100.0                                    # a top score inside the window
+    plain = lsa.union_fixed(lsa.topk(sc, cols, k), pos, n_sink, window)
+    budget = lsa.union_fixed_budget(sc, cols, k, pos, n_sink, window)
+    assert len(budget) == len(plain) + 1               # the budget spends that pick elsewhere
