@@ -58,6 +58,7 @@ typedef enum { LSA_BF16 = 0, LSA_FP8_E4M3 = 1, LSA_FP32 = 2 } lsa_dtype;
 
 /* lsa_topk flags */
 #define LSA_TOPK_RAW (1u << 0) /* output the selected COLUMN ids, no sink/window union (HI recall) */
+#define LSA_TOPK_EXCLUDES_FIXED (1u << 1) /* fixed-budget SI: top-k drawn outside sinks and window */
 
 /* A per-sequence cache: row r of sequence b starts at
  *   data + b * seq_stride + r * tok_stride            (elements of `dtype`),
@@ -149,6 +150,10 @@ lsa_status lsa_block_score(const lsa_batch* batch, const void* q_idx, const floa
  *   SI bullet: a contiguous, hardware-aligned window beside the dynamic picks).
  *   LSA_TOPK_RAW: the output is the selected column ids, ascending (HI coarse recall);
  *   n_sink and window must be 0.
+ *   LSA_TOPK_EXCLUDES_FIXED: fixed-budget SI -- columns at sink or window positions are no
+ *   candidates, so the k picks come from the other visible positions and the (disjoint) list
+ *   holds min(k, those) + the sinks + the window ([release] SI bullet, read as a budget split
+ *   between the contiguous part and the dynamic picks).  Not with LSA_TOPK_RAW.
  *   idx [T][ld_idx] int32, entries beyond count[t] set to -1; count [T] int32.
  *   ld_idx >= k + n_sink + window. */
 lsa_status lsa_topk(const lsa_batch* batch, const float* scores, int64_t ld_scores, int n_cols,
@@ -243,6 +248,9 @@ typedef struct {
     /* indexer queries: 0 = BF16 (exact), 1 = FP8-query mode (as lsa_index_score_q8; flat and
      * the fine stage of HI -- HI block scores keep the BF16 queries) */
     int32_t          idx_q_fp8;
+    /* selection: 0 = top-k over all visible keys, then the union with sinks and window;
+     * 1 = fixed budget (LSA_TOPK_EXCLUDES_FIXED) */
+    int32_t          si_fixed_budget;
 } lsa_decode_params;
 
 /* Runs indexer (flat, or HI: block scores -> recall -> fine scores), top-k + union, then

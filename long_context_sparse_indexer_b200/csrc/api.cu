@@ -85,11 +85,13 @@ lsa_status topk_impl(const lsa_batch* batch, const float* scores, int64_t ld, in
     lsa_status s = check_batch(batch);
     if (s != LSA_OK) return s;
     const bool raw = flags & LSA_TOPK_RAW;
+    const bool fixed = flags & LSA_TOPK_EXCLUDES_FIXED;
     if (k < 0 || n_sink < 0 || window < 0 || n_cols < 0 || n_cols > ld) return LSA_ERR_INVALID_ARG;
     if (raw && (n_sink || window || cand)) return LSA_ERR_INVALID_ARG;
     if ((int64_t)k + n_sink + window > ld_idx) return LSA_ERR_INVALID_ARG;
     if (cand && (n_cand < 1 || block_size < 1 || n_cols > (int64_t)n_cand * block_size)) return LSA_ERR_INVALID_ARG;
-    if (flags & ~LSA_TOPK_RAW) return LSA_ERR_UNSUPPORTED;
+    if (flags & ~(LSA_TOPK_RAW | LSA_TOPK_EXCLUDES_FIXED)) return LSA_ERR_UNSUPPORTED;
+    if (raw && fixed) return LSA_ERR_INVALID_ARG;
     if (batch->T == 0) return LSA_OK;
     if (!scores || !idx || !count) return LSA_ERR_INVALID_ARG;
     TopkArgs a{};
@@ -97,7 +99,7 @@ lsa_status topk_impl(const lsa_batch* batch, const float* scores, int64_t ld, in
     a.B = batch->B; a.T = batch->T; a.L_alloc = batch->L_alloc;
     a.scores = scores; a.ld = ld; a.n_cols = n_cols;
     a.cand = cand; a.n_cand = n_cand; a.block_size = block_size;
-    a.k = k; a.n_sink = n_sink; a.window = window; a.raw = raw;
+    a.k = k; a.n_sink = n_sink; a.window = window; a.raw = raw; a.fixed_budget = fixed;
     a.idx = idx; a.ld_idx = ld_idx; a.count = count; a.status = st;
     return cuda_status(launch_topk(a, stream));
 }
@@ -321,13 +323,14 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
     int32_t* idx = p->idx_out ? p->idx_out : reinterpret_cast<int32_t*>(w + f.idx);
     int32_t* count = p->count_out ? p->count_out : reinterpret_cast<int32_t*>(w + f.count);
     const int64_t ld_idx = p->idx_out ? p->idx_ld : f.cap;
+    const uint32_t topk_flags = p->si_fixed_budget ? LSA_TOPK_EXCLUDES_FIXED : 0u;
 
     if (!p->hi) {
         s = index_score_impl(batch, p->q_idx, p->w, p->H_I, &p->k_idx, nullptr, 0, 0, scores, f.ld, f.n_cols,
                              dev_status, st, p->idx_q_fp8 != 0);
         if (s != LSA_OK) return s;
-        s = topk_impl(batch, scores, f.ld, f.n_cols, nullptr, 0, 0, p->k, p->n_sink, p->window, 0, idx, ld_idx,
-                      count, dev_status, st);
+        s = topk_impl(batch, scores, f.ld, f.n_cols, nullptr, 0, 0, p->k, p->n_sink, p->window, topk_flags, idx,
+                      ld_idx, count, dev_status, st);
         if (s != LSA_OK) return s;
     } else {
         float* bscores = reinterpret_cast<float*>(w + f.bscores);
@@ -343,7 +346,7 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
                              f.ld, 0, dev_status, st, p->idx_q_fp8 != 0);
         if (s != LSA_OK) return s;
         s = topk_impl(batch, scores, f.ld, f.n_cols, cand, p->n_recall, p->block_size, p->k, p->n_sink, p->window,
-                      0, idx, ld_idx, count, dev_status, st);
+                      topk_flags, idx, ld_idx, count, dev_status, st);
         if (s != LSA_OK) return s;
     }
     // The layers depend only on the shared index list, not on one another: layer l runs on

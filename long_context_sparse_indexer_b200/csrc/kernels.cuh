@@ -66,6 +66,7 @@ struct TopkArgs {
     int n_cand, block_size;
     int k, n_sink, window;
     bool raw;
+    bool fixed_budget;       // top-k drawn outside the sinks and the window
     int32_t* idx;
     int64_t ld_idx;
     int32_t* count;

@@ -16,7 +16,9 @@
 // columns first); ranks across CTAs, warps and lanes come from cluster-wide prefix
 // counts, ballots and popcounts.  Positions are written in ascending order and merged
 // with the sinks [0, a) and the window [b, pos], so the list comes out sorted and
-// de-duplicated.  Segments of up to 40960 columns are first cached in shared memory as
+// de-duplicated.  Fixed-budget mode: sink and window positions are no candidates at all, so the
+// top-k is drawn from the other positions and the list holds exactly min(k, those) + a + (pos + 1
+// - b) entries.  Segments of up to 40960 columns are first cached in shared memory as
 // order keys (one coalesced read of the row); longer ones are re-read from global memory.
 #include <algorithm>
 #include <cooperative_groups.h>
@@ -266,12 +268,26 @@ topk_kernel(TopkArgs a) {
     const int per_warp = ((c1 - c0 + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
     const int w0 = min(c1, c0 + warp * per_warp), w1 = min(c1, w0 + per_warp);
 
+    // Sinks [0, a_lo) and window [b_hi, pos] (positions), and the position of column cc.
+    const int a_lo = a.raw ? 0 : min(a.n_sink, pos + 1);
+    const int b_hi = a.raw ? 0x7fffffff : (a.window > 0 ? max(a_lo, pos - a.window + 1) : pos + 1);
+    auto position = [&](int cc) -> int {
+        if (a.raw || !a.cand) return cc;
+        return a.cand[(size_t)t * a.n_cand + cc / a.block_size] * a.block_size + cc % a.block_size;
+    };
+    // Fixed-budget selection: a column at a sink or window position is no candidate.
+    auto fixed_pos = [&](int cc) -> bool {
+        if (!a.fixed_budget) return false;
+        const int p = position(cc);
+        return p < a_lo || p >= b_hi;
+    };
+
     // Order key of column cc of this warp's segment (0 = not a candidate; valid keys are > 0).
     auto key_at = [&](int cc) -> uint32_t {
         if (cc >= w1) return 0u;
         if (CACHED) return s_keys[cc - c0];
         const float f = row[cc];
-        return (f != f || f == kNegInf) ? 0u : order_key(f);
+        return (f != f || f == kNegInf || fixed_pos(cc)) ? 0u : order_key(f);
     };
 
     // ---- pass 1: top 12 bits (and, when cached, the segment's keys into shared memory)
@@ -301,7 +317,7 @@ topk_kernel(TopkArgs a) {
                     if (cc + e >= c1) break;
                     const float x = f[u][e];
                     if (x != x) report(a.status, LSA_ERR_DEVICE_DATA);
-                    s_keys[cc + e - c0] = (x != x || x == kNegInf) ? 0u : order_key(x);
+                    s_keys[cc + e - c0] = (x != x || x == kNegInf || fixed_pos(cc + e)) ? 0u : order_key(x);
                 }
             }
         }
@@ -319,12 +335,6 @@ topk_kernel(TopkArgs a) {
     // Cluster histogram of the top 12 bits; its total is the number of candidates.
     const int n_valid = cluster_threshold_4096(cl, hist, s_sup, a.k, s_red, &s_bin, &s_above, &s_total);
     const bool take_all = n_valid <= a.k;
-    const int a_lo = a.raw ? 0 : min(a.n_sink, pos + 1);
-    const int b_hi = a.raw ? 0x7fffffff : (a.window > 0 ? max(a_lo, pos - a.window + 1) : pos + 1);
-    auto position = [&](int cc) -> int {
-        if (a.raw || !a.cand) return cc;
-        return a.cand[(size_t)t * a.n_cand + cc / a.block_size] * a.block_size + cc % a.block_size;
-    };
 
     // ---- compacted finish.  The top-k lies in the threshold bin b1 of pass 1 or above it, a few
     // thousand columns of the row: every warp lists its candidates (column order) in its region

@@ -24,6 +24,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_DATA, ERR_TIMEOUT = range(7)
 BF16, FP8_E4M3, FP32 = 0, 1, 2
 TOPK_RAW = 1
+TOPK_EXCLUDES_FIXED = 2
 
 c_i32, c_i64, c_u32, c_f32, c_vp, c_size = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float,
                                              ctypes.c_void_p, ctypes.c_size_t)
@@ -57,7 +58,8 @@ class CDecodeParams(ctypes.Structure):
                 ("kbar_seq_stride", c_i64),
                 ("H", c_i32), ("Dqk", c_i32), ("Dv", c_i32), ("sm_scale", c_f32), ("n_split", c_i32),
                 ("n_layers", c_i32), ("layers", ctypes.POINTER(CLayer)),
-                ("idx_out", c_vp), ("idx_ld", c_i64), ("count_out", c_vp), ("idx_q_fp8", c_i32)]
+                ("idx_out", c_vp), ("idx_ld", c_i64), ("count_out", c_vp), ("idx_q_fp8", c_i32),
+                ("si_fixed_budget", c_i32)]
 
 
 _P = ctypes.POINTER
@@ -195,11 +197,12 @@ def block_score(batch: Batch, q_idx: torch.Tensor, w: torch.Tensor, kbar: torch.
 
 def topk(batch: Batch, scores: torch.Tensor, n_cols: int, k: int, n_sink: int, window: int, idx: torch.Tensor,
          count: torch.Tensor, cand_blocks: Optional[torch.Tensor] = None, block_size: int = 0, raw: bool = False,
-         dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+         dev_status: Optional[torch.Tensor] = None, stream=None, fixed_budget: bool = False) -> None:
     cb = batch.c()
     n_cand = int(cand_blocks.shape[1]) if cand_blocks is not None else 0
     _check(_lib.lsa_topk(ctypes.byref(cb), _ptr(scores), int(scores.stride(0)), int(n_cols), _ptr(cand_blocks),
-                         n_cand, int(block_size), int(k), int(n_sink), int(window), TOPK_RAW if raw else 0,
+                         n_cand, int(block_size), int(k), int(n_sink), int(window),
+                         (TOPK_RAW if raw else 0) | (TOPK_EXCLUDES_FIXED if fixed_budget else 0),
                          _ptr(idx), int(idx.stride(0)), _ptr(count), _ptr(dev_status), _stream(stream)), "lsa_topk")
 
 
@@ -260,7 +263,7 @@ class DecodeStep:
                  window: int, layers: Sequence[Layer], H: int, Dqk: int, Dv: int, sm_scale: float, n_split: int = 1,
                  hi: bool = False, block_size: int = 64, n_recall: int = 0, kbar: Optional[torch.Tensor] = None,
                  idx_out: Optional[torch.Tensor] = None, count_out: Optional[torch.Tensor] = None,
-                 idx_q_fp8: bool = False):
+                 idx_q_fp8: bool = False, si_fixed_budget: bool = False):
         self._keep = (batch, q_idx, w, k_idx, list(layers), kbar, idx_out, count_out)
         arr = (CLayer * max(1, len(layers)))()
         for i, L in enumerate(layers):
@@ -271,7 +274,7 @@ class DecodeStep:
                                int(kbar.stride(0)) if kbar is not None else 0, int(H), int(Dqk), int(Dv),
                                float(sm_scale), int(n_split), len(layers), arr, _ptr(idx_out),
                                int(idx_out.stride(0)) if idx_out is not None else 0, _ptr(count_out),
-                               int(bool(idx_q_fp8)))
+                               int(bool(idx_q_fp8)), int(bool(si_fixed_budget)))
 
     def workspace_size(self) -> int:
         return int(_lib.lsa_decode_workspace_size(ctypes.byref(self.p)))

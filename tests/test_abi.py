@@ -67,6 +67,7 @@ def test_topk_rejects_bad_arguments():
     assert call(k=-1) == lsa.ERR_INVALID_ARG
     assert call(flags=lsa.TOPK_RAW) == lsa.ERR_INVALID_ARG                 # raw mode takes no sinks/window
     assert call(flags=8) == lsa.ERR_UNSUPPORTED
+    assert call(flags=lsa.TOPK_RAW | lsa.TOPK_EXCLUDES_FIXED, ns=0, win=0) == lsa.ERR_INVALID_ARG   # raw has no fixed part
 
 
 def test_attention_rejects_bad_arguments():

@@ -296,6 +296,76 @@ def test_topk_all_equal_scores(cuda, n_cols):
         assert got[t].tolist() == want.tolist()
 
 
+@pytest.mark.parametrize("n_cols,k,n_sink,window,tie_levels", [
+    (5000, 256, 4, 128, 3), (70000, 2048, 4, 512, 50), (70000, 2048, 4, 512, 2), (100, 300, 4, 16, 2),
+])
+def test_topk_fixed_budget(cuda, n_cols, k, n_sink, window, tie_levels):
+    """Fixed-budget SI: the oracle's top-k over the positions outside the sinks and the window,
+    then the (disjoint) union; the list holds exactly min(k, outside) + sinks + window."""
+    rng = np.random.default_rng(n_cols + k + 7)
+    T = 4
+    s = _host_score_rows(rng, T, n_cols, tie_levels)
+    pos = np.array([n_cols - 1, n_cols // 2, 10, n_cols - 2])
+    for t in range(T):
+        s[t, pos[t] + 1:] = -np.inf
+    # the best scores of every row sit in its window and its sinks: the budget must skip them
+    for t in range(T):
+        s[t, max(0, pos[t] - 3):pos[t] + 1] = 1e6
+        s[t, :2] = 1e6
+    batch = lsa.Batch(torch.tensor([n_cols], dtype=torch.int32, device="cuda"),
+                      torch.zeros(T, dtype=torch.int32, device="cuda"),
+                      torch.from_numpy(pos.astype(np.int32)).cuda(), n_cols)
+    idx = torch.empty((T, k + n_sink + window), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(T, dtype=torch.int32, device="cuda")
+    lsa.topk(batch, torch.from_numpy(s).cuda(), n_cols, k, n_sink, window, idx, cnt, fixed_budget=True)
+    got = H.index_lists(idx, cnt)
+    for t in range(T):
+        cols = np.nonzero(~np.isneginf(s[t]))[0]
+        want = olsa.union_fixed_budget(s[t, cols].astype(np.float64), cols, k, int(pos[t]), n_sink, window)
+        assert got[t].tolist() == want.tolist()
+        a = min(n_sink, pos[t] + 1)
+        b = max(a, pos[t] - window + 1)
+        outside = int(np.sum((cols >= a) & (cols < b)))
+        assert len(got[t]) == min(k, outside) + a + (pos[t] + 1 - b)
+        assert np.all(idx[t, cnt[t]:].cpu().numpy() == -1)
+
+
+def test_topk_fixed_budget_candidate_blocks(cuda):
+    rng = np.random.default_rng(2)
+    T, bs, n_cand = 3, 64, 40
+    blocks = np.stack([np.sort(rng.choice(500, size=n_cand, replace=False)) for _ in range(T)])
+    blocks[:, 0] = 0                                          # the sinks' block is recalled
+    blocks[2, -5:] = -1
+    pos = np.array([500 * 64 - 1, 250 * 64 + 17, 30000])
+    for t in range(T):                                        # and the window's last block
+        last = int(pos[t]) // bs
+        if last not in blocks[t]:
+            blocks[t, 1] = last
+        blocks[t] = np.sort(np.where(blocks[t] < 0, 10 ** 6, blocks[t]))
+        blocks[t] = np.where(blocks[t] == 10 ** 6, -1, blocks[t])
+    s = rng.integers(0, 20, size=(T, n_cand * bs)).astype(np.float32)
+    for t in range(T):
+        p_of_col = (blocks[t][:, None] * bs + np.arange(bs)[None, :]).reshape(-1)
+        bad = (np.repeat(blocks[t], bs) < 0) | (p_of_col > pos[t])
+        s[t, bad] = -np.inf
+        s[t, (p_of_col <= pos[t]) & (p_of_col > pos[t] - 50) & ~bad] = 1e6     # top scores in the window
+    batch = lsa.Batch(torch.tensor([500 * 64], dtype=torch.int32, device="cuda"),
+                      torch.zeros(T, dtype=torch.int32, device="cuda"), torch.from_numpy(pos.astype(np.int32)).cuda(),
+                      500 * 64)
+    cb = torch.from_numpy(blocks.astype(np.int32)).cuda()
+    k, ns, win = 300, 4, 100
+    idx = torch.empty((T, k + ns + win), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(T, dtype=torch.int32, device="cuda")
+    lsa.topk(batch, torch.from_numpy(s).cuda(), n_cand * bs, k, ns, win, idx, cnt, cand_blocks=cb, block_size=bs,
+             fixed_budget=True)
+    got = H.index_lists(idx, cnt)
+    for t in range(T):
+        p_of_col = (blocks[t][:, None] * bs + np.arange(bs)[None, :]).reshape(-1)
+        valid = ~np.isneginf(s[t])
+        want = olsa.union_fixed_budget(s[t, valid].astype(np.float64), p_of_col[valid], k, int(pos[t]), ns, win)
+        assert got[t].tolist() == want.tolist()
+
+
 def test_topk_raw_and_candidate_blocks(cuda):
     rng = np.random.default_rng(1)
     T, bs, n_cand = 3, 64, 40
