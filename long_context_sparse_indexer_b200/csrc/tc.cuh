@@ -240,13 +240,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                  :: "r"(smem_u32(bar)) : "memory");
 }
 
-// Arrives on the mbarrier at the same shared-memory offset in every CTA of the cluster whose bit
-// is set in cta_mask, once every tcgen05.mma issued so far by this thread has completed.
-__device__ __forceinline__ void mma_commit_cluster(uint64_t* bar, uint16_t cta_mask) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-                 :: "r"(smem_u32(bar)), "h"(cta_mask) : "memory");
-}
-
 // ---------------------------------------------------------------- clusters
 
 // Shared::cluster address of this CTA's shared-memory location p in cluster CTA `rank`.
