@@ -13,9 +13,10 @@
 // runs the same softmax (so both hold the same P) and accumulates O[:, V half h] += P V_h from
 // its own rows.  Every byte of a row is read once and no product is computed twice.
 //
-// Memory plan.  TMEM (512 columns): O half [0,256), three S / P buffers [256,352) -- the
-// softmax writes P (BF16) over the S it has just read, so S can run two tiles ahead of P V --
-// and the query slice Q[:, D_h] [352,496) as the A operand of S.  Shared memory: an 8-stage
+// Memory plan.  TMEM (512 columns): O half [0,256), four S / P buffers [256,384) -- the
+// softmax writes P (BF16) over the S it has just read, so S can run three tiles ahead of P V --
+// and the query's V-half dims [384,512) as the A operand of S; the query's 32 rope dims sit in
+// shared memory (no swizzle, K-major) as the A operand of S's two rope steps.  Shared memory: an 8-stage
 // ring of 32-row KV tiles, read as the B operand of S (K-major) and of P V (MN-major): each
 // stage has its 4 swizzled 64-dim V-half atoms (16 KB), and two stages share one 64-dim rope
 // atom, each in the half of its 128-byte rows that the other leaves (only 32 rope dims are this
@@ -27,8 +28,8 @@
 //                tile::gather4 (4 rows x 64 dims per load) and the 4 rope chunks of each row with
 //                16-byte cp.async; both complete on the tile's barrier by themselves, so the warp
 //                moves on at once.  (Without a tensor map for the cache, cp.async does it all.)
-//   warp 1     : MMA issuer -- S_j (18 TS MMAs, N = 32) once tile j has landed, P V_{j-3} has
-//                been issued and S_{j-3} has been sent; O += P_j V_j (2 TS MMAs, N = 256) once
+//   warp 1     : MMA issuer -- S_j (16 TS + 2 SS MMAs, N = 32) once tile j has landed, P V_{j-4}
+//                has been issued and S_{j-4} has been sent; O += P_j V_j (2 TS MMAs, N = 256) once
 //                the softmax of tile j is done; whichever is ready, each kind in order.
 //   warps 4..7 : send -- warp q (mod 4) stages heads [32q, 32q + 32) of each partial S in shared
 //                memory and pushes the 4 KB to the peer with one bulk shared-to-shared copy that
@@ -165,7 +166,8 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
         sm.abort = 0;
         tc::fence_barrier_init();
         // Q[:, V half] as 4 swizzled 64-dim atoms into the exchange buffers and its rope atom into
-        // KV stage 7, all idle until the softmax warps have moved Q to TMEM.
+        // KV stage 7, all idle until the softmax warps have moved Q to TMEM (the rope part to
+        // shared memory).
         tc::prefetch_tmap(&qmap);
         tc::mbar_expect_tx(&sm.q_tma, 5 * 128 * 128);
         for (int at = 0; at < 5; ++at)
@@ -231,7 +233,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
     if (remote_warp) tc::cluster_wait();
 
     if (kAsync ? (warp == 0 || warp == 2 || warp == 3) : warp < kGatherFp8) {
-        // ---------------- gather producers: tiles j = first, first + step, ... into stage j % 7
+        // ---------------- gather producers: tiles j = first, first + step, ... into stage j % 8
         const int first = kAsync ? (warp == 0 ? 0 : warp - 1) : warp, step = kAsync ? 3 : kGatherFp8;
         auto fetch_row = [&](int j) -> int {                       // lane l: index of row l of tile j
             if (j >= n_tiles) return -1;
@@ -369,7 +371,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             uint32_t polls = 0;
             while (npv < n_tiles) {
                 bool progressed = false;
-                // S_ns needs its KV tile and its S / P buffer free: P V_{ns-3} issued and S_{ns-3}
+                // S_ns needs its KV tile and its S / P buffer free: P V_{ns-4} issued and S_{ns-4}
                 // read by the send warps.
                 if (ns < n_tiles && ns <= npv + kSP - 1 &&
                     (ns < kSP || tc::mbar_test_wait(&sm.s_sent[ns % kSP], ((ns / kSP) - 1) & 1)) &&
