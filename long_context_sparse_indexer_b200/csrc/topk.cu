@@ -7,19 +7,23 @@
 // first, which makes the selection unique and the output deterministic.
 //
 // Method: radix select on the order-preserving 32-bit key of each score, 12 + 12 + 8 bits.
-// One query row is handled by a cluster of kTopkCluster CTAs; CTA r owns the r-th
-// contiguous segment of the row.  Each pass builds integer shared-memory histograms of
-// its segment (shared-memory atomics; counts do not depend on atomic order), every CTA
-// then reads all the cluster's histograms through distributed shared memory and finds
-// the same threshold bin.  The result is the k-th key v* and the number m of ties at v*
-// to keep.  The emission pass keeps every key > v* and the first m keys == v* (lowest
-// columns first); ranks across CTAs, warps and lanes come from cluster-wide prefix
-// counts, ballots and popcounts.  Positions are written in ascending order and merged
-// with the sinks [0, a) and the window [b, pos], so the list comes out sorted and
-// de-duplicated.  Fixed-budget mode: sink and window positions are no candidates at all, so the
-// top-k is drawn from the other positions and the list holds exactly min(k, those) + a + (pos + 1
-// - b) entries.  Segments of up to 40960 columns are first cached in shared memory as
-// order keys (one coalesced read of the row); longer ones are re-read from global memory.
+// One query row is handled by a cluster of kTopkCluster CTAs; CTA r owns the r-th contiguous
+// segment of the row (cached in shared memory as order keys when it has at most 40960 columns,
+// else re-read from global memory).  Histograms are integer shared-memory counts (atomics;
+// counts do not depend on atomic order).
+//   1. Top 12 bits over the cluster: each CTA folds its 4096 bins into 64 super-bins; after one
+//      cluster barrier every CTA reads the 8 x 64 super-bin counts, then the 8 x 64 bins inside
+//      the threshold super-bin, through distributed shared memory, and finds the same bin b1.
+//   2. The keys at or above b1 (usually a few thousand) are compacted, in column order, into
+//      CTA 0's shared memory; CTA 0 alone finds the next 12 and the last 8 bits, i.e. the k-th
+//      key v* and the number m of ties at v* to keep, and emits: every key > v* and the first
+//      m keys == v* (lowest columns first), ranks from per-warp counts, ballots and popcounts.
+//      When the candidates do not fit, the cluster runs passes 2 and 3 over its segments and
+//      emits with cluster-wide prefix counts instead.
+// Positions are written in ascending order and merged with the sinks [0, a) and the window
+// [b, pos], so the list comes out sorted and de-duplicated.  Fixed-budget mode: sink and window
+// positions are no candidates at all, so the top-k is drawn from the other positions and the
+// list holds exactly min(k, those) + a + (pos + 1 - b) entries.
 #include <algorithm>
 #include <cooperative_groups.h>
 
