@@ -129,3 +129,36 @@ def test_pipeline_rejects_bad_arguments():
     assert lib.lsa_pipeline_step(None, 0, None, 0, None, None, None, 0, None, 0, None) == lsa.ERR_INVALID_ARG
     assert lib.lsa_pipeline_join(None) == lsa.ERR_INVALID_ARG
     assert lib.lsa_pipeline_destroy(None) == lsa.ERR_INVALID_ARG
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """Every ctypes mirror of a header struct has the header's size and field offsets (checked
+    by compiling a C program against include/lsa.h)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    mirrors = {"lsa_cache": lsa.CCache, "lsa_batch": lsa.CBatch, "lsa_layer": lsa.CLayer,
+               "lsa_decode_params": lsa.CDecodeParams, "lsa_copy": lsa.CCopy}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "lsa.h"', "int main(void) {"]
+    for cname, cls in mirrors.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run([gcc, "-std=c11", "-I", inc, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {}
+    for line in out:
+        if line:
+            parts = line.split()
+            got[tuple(parts[:-1])] = int(parts[-1])
+    for cname, cls in mirrors.items():
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for fname, _ in cls._fields_:
+            assert got[(cname, fname)] == getattr(cls, fname).offset, (cname, fname)
