@@ -33,6 +33,9 @@
  *   - Element strides are counted in elements of the cache's dtype.
  *   - No exception crosses this boundary.  Calls on different streams may run
  *     concurrently as long as their output buffers do not overlap.
+ *   - One call handles at most 65,535 query tokens and 65,535 sequences (some kernels put
+ *     the token in a grid dimension of that size); larger batches return
+ *     LSA_ERR_UNSUPPORTED before anything is launched.
  */
 #ifndef LSA_H_
 #define LSA_H_
@@ -196,9 +199,13 @@ size_t lsa_attn_workspace_size(int T, int H, int Dv, int n_split);
  *   - Returns LSA_ERR_WORKSPACE when lsa_attn_workspace_size(T, H, Dv, n_split) exceeds
  *     LSA_NOALLOC_SCRATCH_BYTES (at Dv = 512: T * n_split * H at most 16,352);
  *     n_split == 1 needs no scratch.
+ *   - Arguments are checked exactly as lsa_sparse_attn checks them (same statuses); the
+ *     scratch size is checked after those checks.
  *   - The first call with n_split > 1 on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is kept per device and CUDA context: after a device
+ *     reset (which destroys the context and the array with it) the next call looks it up
+ *     again in the new context, so that call too should come before any capture.
  *   - Every call shares the one array and it keeps the last call's contents; nothing in
  *     it needs to start at zero (each call writes every partial it reads).  Calls whose
  *     execution overlaps on the GPU (other streams, other threads, concurrent graphs)

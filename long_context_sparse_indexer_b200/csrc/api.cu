@@ -10,6 +10,7 @@ using namespace lsa;
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr int kMaxTokens = 65535;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 inline int elem_bytes(int dtype) { return dtype == LSA_FP8_E4M3 ? 1 : (dtype == LSA_BF16 ? 2 : 4); }
@@ -17,6 +18,8 @@ inline int elem_bytes(int dtype) { return dtype == LSA_FP8_E4M3 ? 1 : (dtype == 
 lsa_status check_batch(const lsa_batch* b) {
     if (!b || b->B < 1 || b->T < 0 || b->q_group < 1 || b->L_alloc < 1) return LSA_ERR_INVALID_ARG;
     if (b->T % b->q_group) return LSA_ERR_INVALID_ARG;
+    // Several kernels put the query token in a grid dimension limited to 65535 blocks.
+    if (b->T > kMaxTokens || b->B > kMaxTokens) return LSA_ERR_UNSUPPORTED;
     if (b->T > 0 && (!b->seq_len || !b->q_seq || !b->q_pos)) return LSA_ERR_INVALID_ARG;
     return LSA_OK;
 }
@@ -109,10 +112,13 @@ size_t attn_ws(int T, int H, int Dv, int n_split) {
     return align_up((size_t)T * n_split * H * Dv * 4) + align_up((size_t)T * n_split * H * 4);
 }
 
-lsa_status attn_impl(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,
-                     const lsa_cache* v, int Dv, const int32_t* idx, int64_t ld_idx, const int32_t* count,
-                     float sm_scale, int n_split, void* o, float* lse, void* ws, size_t ws_bytes,
-                     int32_t* st, cudaStream_t stream) {
+}  // namespace
+
+// Argument checks of lsa_sparse_attn that do not involve the workspace (shared with the
+// no-allocation entry point, which checks its own scratch size after these).
+lsa_status lsa::attn_validate(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,
+                              const lsa_cache* v, int Dv, const int32_t* idx, int64_t ld_idx, const int32_t* count,
+                              float sm_scale, int n_split, const void* o) {
     lsa_status s = check_batch(batch);
     if (s != LSA_OK) return s;
     const bool sep_v = v && v->data;
@@ -127,6 +133,18 @@ lsa_status attn_impl(const lsa_batch* batch, const void* q, int H, int Dqk, cons
     if (batch->T == 0) return LSA_OK;
     if (!q || !idx || !count || !o) return LSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(o)) return LSA_ERR_INVALID_ARG;
+    return LSA_OK;
+}
+
+namespace {
+
+lsa_status attn_impl(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,
+                     const lsa_cache* v, int Dv, const int32_t* idx, int64_t ld_idx, const int32_t* count,
+                     float sm_scale, int n_split, void* o, float* lse, void* ws, size_t ws_bytes,
+                     int32_t* st, cudaStream_t stream) {
+    lsa_status s = attn_validate(batch, q, H, Dqk, kv, v, Dv, idx, ld_idx, count, sm_scale, n_split, o);
+    if (s != LSA_OK || batch->T == 0) return s;
+    const bool sep_v = v && v->data;
     const size_t need = attn_ws(batch->T, H, Dv, n_split);
     if (need && (!ws || ws_bytes < need || ((uintptr_t)ws % kAlign))) return LSA_ERR_WORKSPACE;
     AttnArgs a{};

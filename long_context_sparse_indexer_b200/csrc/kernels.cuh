@@ -107,4 +107,9 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, int DQK, int DV, bool kv_fp8, 
 bool sparse_attn_tc_supported(const AttnArgs& a, int DQK, int DV, bool sep_v);
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, bool kv_fp8, cudaStream_t st);
 
+// Host-side checks of lsa_sparse_attn's arguments other than its workspace (api.cu).
+lsa_status attn_validate(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,
+                         const lsa_cache* v, int Dv, const int32_t* idx, int64_t ld_idx, const int32_t* count,
+                         float sm_scale, int n_split, const void* o);
+
 }  // namespace lsa

@@ -89,6 +89,38 @@ def test_attention_rejects_bad_arguments():
     assert lsa.attn_workspace_size(5, 128, 512, 1) == 0
 
 
+def test_noalloc_attention_checks_shapes_before_its_scratch_size():
+    """The no-allocation entry point returns what lsa_sparse_attn returns for the same bad
+    arguments, and LSA_ERR_WORKSPACE only for a valid request its static scratch cannot hold
+    (no GPU: every one of these returns before the first CUDA call)."""
+    lib = lsa.library()
+    kv = _cache(dtype=lsa.BF16, dim=576, scale=None)
+    big = _batch(T=200)
+    call = lambda b, H=128, ns=64: lib.lsa_sparse_attn_noalloc(  # noqa
+        ctypes.byref(b), 4096, H, 576, ctypes.byref(kv), None, 512, 16, 100, 16, 0.04, ns, 4096, 16, None, None)
+    assert call(big, H=100) == lsa.ERR_UNSUPPORTED          # shape first, although 200 x 64 x 100 rows > scratch
+    assert call(big, ns=0) == lsa.ERR_INVALID_ARG
+    assert call(big) == lsa.ERR_WORKSPACE                   # 200 x 64 x 128 partial rows of 2 KB > 32 MiB
+    assert lsa.attn_workspace_size(200, 128, 512, 64) > lsa.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    m = re.search(r"#define\s+LSA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", open(HDR).read())
+    assert m, "LSA_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert int(m.group(1)) << int(m.group(2)) == lsa.NOALLOC_SCRATCH_BYTES
+
+
+def test_batches_beyond_the_grid_limit_are_refused():
+    """More than 65,535 query tokens in one call: LSA_ERR_UNSUPPORTED before any launch."""
+    lib = lsa.library()
+    b = _batch(T=65536)
+    kv = _cache(dtype=lsa.BF16, dim=576, scale=None)
+    assert lib.lsa_sparse_attn(ctypes.byref(b), 4096, 128, 576, ctypes.byref(kv), None, 512, 16, 100, 16, 0.04, 1,
+                               4096, 16, None, 0, None, None) == lsa.ERR_UNSUPPORTED
+    assert lib.lsa_topk(ctypes.byref(b), 16, 100, 100, None, 0, 0, 10, 0, 0, 0, 16, 10, 16, None,
+                        None) == lsa.ERR_UNSUPPORTED
+
+
 def test_fused_rejects_bad_arguments():
     lib = lsa.library()
     p = lsa.CDecodeParams()

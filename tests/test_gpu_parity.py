@@ -455,10 +455,12 @@ def test_fused_path_end_to_end(cuda, name):
             a, b = set(got[t].tolist()), set(ref["idx"].tolist())
             assert len(a & b) >= 0.999 * len(b) and len(a) == len(b), (t, len(a), len(b), len(a & b))
             assert np.all(np.diff(got[t]) > 0)
-            if a == b:
-                for li, (o_ref, lse_ref) in enumerate(ref["layers"]):
-                    mx, rl2 = H.attn_errors(outs[li][0][t], o_ref)
-                    assert mx < 1e-2 and rl2 < 5e-3, (t, li, mx, rl2)
+            for li, layer in enumerate(p.layers):
+                # where the lists differ (near-ties decided in FP32), the attention is checked on
+                # the GPU's own list
+                o_ref = ref["layers"][li][0] if a == b else run.attend(w, p, layer, t, got[t])[0]
+                mx, rl2 = H.attn_errors(outs[li][0][t], o_ref)
+                assert mx < 1e-2 and rl2 < 5e-3, (t, li, mx, rl2, a == b)
 
 
 @pytest.mark.parametrize("name", ["cli_small", "mtp_small"])
