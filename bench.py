@@ -134,8 +134,7 @@ def build_step(w, wt, pi, n_split, q8=False):
                                 lsa.Cache(L["v"]) if L["v"] is not None else None))
     kbar = None
     if w.hi:
-        nblk = (wt.L_alloc + w.block_size - 1) // w.block_size
-        kbar = torch.empty((w.B, nblk, w.d_I), dtype=torch.float32, device=dev)
+        kbar = lsa.block_keys_buffer(w.B, wt.L_alloc, w.block_size, w.d_I, dev)
         lsa.block_keys(batch, lsa.Cache(pt.k_idx, pt.k_scale), w.block_size, kbar)
     idx = torch.empty((T, w.cap), dtype=torch.int32, device=dev)
     cnt = torch.empty((T,), dtype=torch.int32, device=dev)
@@ -242,46 +241,67 @@ def time_region(fn, steps, stream):
     return e0.elapsed_time(e1) / steps
 
 
-def run_gpu(args, rank, world, local_rank):
+def attention_flops(w, steps_data):
+    """Algorithmic flops of the attention of one step: 2 * H * (Dqk + Dv) per (query, selected row,
+    layer) -- the QK^T and PV contractions."""
+    tot = 0.0
+    for p, sd in zip(w.passes, steps_data):
+        rows = float(sd["cnt"].sum().item())
+        tot += 2.0 * w.H * (w.D + w.Dv) * rows * len(p.layers)
+    return tot
+
+
+def graph_of(fn):
+    """fn captured once into a CUDA graph (on a side stream), or None if capture fails."""
+    try:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                fn(s)
+        torch.cuda.synchronize()
+        return g
+    except Exception as e:  # capture unsupported: eager launches
+        print(f"[bench] graph capture failed, timing eager launches: {e}", file=sys.stderr)
+        return None
+
+
+def time_alone(fn, stream, n):
+    """Average CUDA-event duration of fn() on `stream` over n back-to-back launches (after 3 warm)."""
+    for _ in range(3):
+        fn()
+    return time_region(fn, n, stream)
+
+
+def measure(name, args, rank, world, local_rank, headline):
+    """One workload: its step (all passes, all layers) captured in a CUDA graph, W warm-up steps,
+    a sustained untimed load (so the clock samples describe the steady state), then exactly K
+    steps between CUDA events; the dominant kernels timed alone for the rooflines; with
+    `headline`, also the end-to-end rate through the host-buffer pipeline."""
     from lsa_synth import device as D
     from long_context_sparse_indexer_b200 import launch, lsa
 
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = W.WORKLOADS[args.workload]
-    if args.batch:
-        w = W.scaled(args.workload, B=args.batch)
+    w = W.WORKLOADS[name]
+    if args.batch and headline:
+        w = W.scaled(name, B=args.batch)
     w = rank_workload(w, rank, world)
     wt = D.build_workload(w, dev)
     stream = torch.cuda.current_stream()
-    forced = [int(x) for x in args.n_split.split(",")] if args.n_split else []
+    forced = [int(x) for x in args.n_split.split(",")] if (args.n_split and headline) else []
     sds = [build_step(w, wt, pi, forced[min(pi, len(forced) - 1)] if forced
                       else launch.split_for(w.T(p), w.H, w.cap, layers=len(p.layers)), q8=args.idx_q8)
            for pi, p in enumerate(w.passes)]
 
-    def step():
+    def step(s=None):
         for sd in sds:
-            sd["step"](sd["ws"], stream=stream)
+            sd["step"](sd["ws"], stream=s if s is not None else stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
-
-    graph = None
-    if not args.no_graph:
-        try:
-            g = torch.cuda.CUDAGraph()
-            s = torch.cuda.Stream()
-            s.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(s):
-                with torch.cuda.graph(g, stream=s):
-                    for sd in sds:
-                        sd["step"](sd["ws"], stream=s)
-            torch.cuda.synchronize()
-            graph = g
-        except Exception as e:  # capture unsupported: eager launches
-            print(f"[bench] graph capture failed, timing eager launches: {e}", file=sys.stderr)
-            graph = None
+    graph = None if args.no_graph else graph_of(step)
     fn = (lambda: graph.replay()) if graph is not None else step
     for _ in range(3):
         fn()
@@ -291,7 +311,11 @@ def run_gpu(args, rank, world, local_rank):
         dist.barrier()
     with ClockSampler(local_rank) as clk:
         torch.cuda.synchronize()
-        time.sleep(0.05)                     # let the sampler start before the timed region
+        time.sleep(0.05)                     # let the sampler start
+        # sustained untimed load of about args.load_ms, then the timed region
+        t_one = time_region(fn, 3, stream)
+        for _ in range(max(1, int(args.load_ms / max(t_one, 1e-3)))):
+            fn()
         ms = time_region(fn, args.steps, stream)
     if world > 1:
         dist.barrier()
@@ -300,11 +324,18 @@ def run_gpu(args, rank, world, local_rank):
     q_per_step = w.queries_per_step()
     value = q_per_step * world / (ms / 1e3)
     total_bytes, idx_bytes = algorithmic_bytes(w, wt, sds)
+    hbm, src = peaks()
+    bf16, bsrc = bf16_peak()
+    res = {"workload": w.name, "value": value, "unit": "queries/s", "ms_per_step": ms,
+           "algorithmic_gb_per_step": total_bytes / 1e9, "step_hbm_gbs": total_bytes / (ms / 1e3) / 1e9,
+           "step_hbm_frac": total_bytes / (ms / 1e3) / 1e9 / hbm,
+           "n_split": [sd["n_split"] for sd in sds], "launch": "cuda_graph" if graph is not None else "eager",
+           "clocks": clk.summary()}
 
-    # Dominant kernel: the indexer of the first pass, timed alone on the same inputs.
-    sd0 = sds[0]
-    pt0 = wt.passes[0]
+    # Dominant kernels timed alone on the same inputs, against their rooflines.
+    sd0, pt0 = sds[0], wt.passes[0]
     k_cache = lsa.Cache(pt0.k_idx, pt0.k_scale)
+    n_alone = max(10, args.steps)
     if not w.hi:
         ld = (wt.L_alloc + 3) // 4 * 4
         sc = torch.empty((sd0["T"], ld), dtype=torch.float32, device=dev)
@@ -316,13 +347,10 @@ def run_gpu(args, rank, world, local_rank):
         sc = torch.empty((sd0["T"], (nblk + 3) // 4 * 4), dtype=torch.float32, device=dev)
         idx_fn = lambda: lsa.block_score(sd0["batch"], pt0.q_idx, pt0.w, sd0["kbar"], w.block_size, sc, nblk,  # noqa
                                          stream=stream)
-        kern = "block_score (HI coarse scores)"
+        kern = "block_score (HI coarse scores, tensor cores)"
         lens = W.lengths(w)
         idx_bytes = sum((int(l) - 1) // w.block_size + 1 for l in lens) * w.d_I * 4
-    for _ in range(3):
-        idx_fn()
-    kms = time_region(idx_fn, max(10, args.steps), stream)
-    hbm, src = peaks()
+    kms = time_alone(idx_fn, stream, n_alone)
     achieved = idx_bytes / (kms / 1e3) / 1e9
     roof = {"bound": "hbm", "kernel": kern, "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": indexer_traffic(kern, idx_bytes), "peak_source": f"{src} hbm_gbs",
@@ -332,18 +360,67 @@ def run_gpu(args, rank, world, local_rank):
         # burst x 2 (the nominal FP8 / BF16 ratio).  Tensor-bound when its flops at that peak take
         # longer than its bytes at the HBM peak (prefill; not decode).
         flops = indexer_flops(w, w.passes[0])
-        bf16, bsrc = bf16_peak()
         fp8 = 2.0 * bf16
         if flops / (fp8 * 1e12) > idx_bytes / (hbm * 1e9):
             tf = flops / (kms / 1e3) / 1e12
             roof.update({"bound": "tensor", "achieved": tf, "peak": fp8, "unit": "TFLOP/s", "frac": tf / fp8,
-                         "peak_source": f"{bsrc} bf16_tflops x 2 (FP8 MMA)", "algorithmic_flops_per_launch": flops})
+                         "peak_source": f"{bsrc} bf16_tflops x 2 (FP8 MMA)", "algorithmic_flops_per_launch": flops,
+                         "algorithmic_bytes_per_launch": idx_bytes})
+    res["roofline"] = roof
 
-    # End to end through the public API with host buffers: the pipelined driver of the C ABI
-    # (lsa_pipeline_*).  Every step copies its queries (indexer q and w, every layer's q) from
-    # pinned host memory into one of two slots of device buffers, runs the fused calls on that
-    # slot and copies every layer's output back to pinned host memory; the copies of one step
-    # overlap the decode of its neighbours.  The timed region ends after the last step's copy-out.
+    # Attention of the first pass alone (every layer of the pass, as in the step), against the
+    # tensor roofline when its flops dominate (prefill), else HBM.
+    p0 = w.passes[0]
+    att_layers = sd0["layers"]
+    ws_att = torch.empty(max(256, 2 * lsa.attn_workspace_size(sd0["T"], w.H, w.Dv, sd0["n_split"])),
+                         dtype=torch.uint8, device=dev)
+
+    def att_fn():
+        for L in att_layers:
+            lsa.sparse_attn(sd0["batch"], L.q, L.kv, sd0["idx"], sd0["cnt"], w.sm_scale, L.o, L.lse, v=L.v,
+                            n_split=sd0["n_split"], ws=ws_att, stream=stream)
+    ams = time_alone(att_fn, stream, n_alone)
+    rows = float(sd0["cnt"].sum().item())
+    rowb = w.D * (1 if w.kv_fp8 else 2) + (4 if w.kv_fp8 else 0)
+    att_bytes = len(att_layers) * (rows * rowb + sd0["T"] * (w.H * w.D * 2 + w.H * w.Dv * 2 + w.H * 4))
+    att_flops = 2.0 * w.H * (w.D + w.Dv) * rows * len(att_layers)
+    a_roof = {"kernel": "sparse_attn (+ split merge)", "launch_ms": ams, "algorithmic_bytes_per_launch": att_bytes,
+              "algorithmic_flops_per_launch": att_flops}
+    if att_flops / (bf16 * 1e12) > att_bytes / (hbm * 1e9):
+        tf = att_flops / (ams / 1e3) / 1e12
+        a_roof.update({"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16,
+                       "peak_source": f"{bsrc} bf16_tflops (BF16 MMA)"})
+    else:
+        gb = att_bytes / (ams / 1e3) / 1e9
+        a_roof.update({"bound": "hbm", "achieved": gb, "peak": hbm, "unit": "GB/s", "frac": gb / hbm,
+                       "peak_source": f"{src} hbm_gbs"})
+    res["attention_roofline"] = a_roof
+
+    if headline:
+        res["e2e"] = e2e_rate(w, wt, sds, args, world, dev, stream, q_per_step)
+        res["gpu_launches"] = launches_per_step(w, [sd["n_split"] for sd in sds]) * args.steps
+        res["config"] = {"workload": w.name, "description": w.description, "batch": w.B,
+                         "queries_per_step_per_gpu": q_per_step,
+                         "ctx": [int(W.lengths(w).min()), int(W.lengths(w).max())],
+                         "k": w.k, "n_sink": w.n_sink, "window": w.window, "hi": w.hi,
+                         "layers_per_index": [len(p.layers) for p in w.passes],
+                         "indexer_queries": "fp8 (per-head power-of-two scale)" if args.idx_q8 else "bf16 (exact)",
+                         "n_split": res["n_split"], "parallelism": f"replicas x{world} (batch per GPU)",
+                         "launch": res["launch"],
+                         "l2": "inputs larger than L2 (indexer keys + selected KV rows per step >> 126 MB)"}
+    del sds, wt, graph
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res, w
+
+
+def e2e_rate(w, wt, sds, args, world, dev, stream, q_per_step):
+    """End to end through the public API with host buffers: the pipelined driver of the C ABI
+    (lsa_pipeline_*).  Every step copies its queries (indexer q and w, every layer's q) from
+    pinned host memory into one of two slots of device buffers, runs the fused calls on that
+    slot and copies every layer's output back to pinned host memory; the copies of one step
+    overlap the decode of its neighbours.  The timed region ends after the last step's copy-out."""
+    from long_context_sparse_indexer_b200 import lsa
     n_slots = max(2, args.slots)
     pl = lsa.Pipeline(n_slots, stream)
     preps, h2d_bytes, d2h_bytes = [], 0, 0
@@ -380,51 +457,29 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     pl.close()
-    h2d, d2h = h2d_bytes, d2h_bytes
-
-    res = {
-        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16+fp8", "data": "synthetic (seeded counter-based generator)",
-        "config": {"workload": w.name, "description": w.description, "batch": w.B,
-                   "queries_per_step_per_gpu": q_per_step, "ctx": [int(W.lengths(w).min()), int(W.lengths(w).max())],
-                   "k": w.k, "n_sink": w.n_sink, "window": w.window, "hi": w.hi,
-                   "layers_per_index": [len(p.layers) for p in w.passes],
-                   "indexer_queries": "fp8 (per-head power-of-two scale)" if args.idx_q8 else "bf16 (exact)",
-                   "n_split": [sd["n_split"] for sd in sds], "parallelism": f"replicas x{world} (batch per GPU)",
-                   "launch": "cuda_graph" if graph is not None else "eager",
-                   "l2": "inputs larger than L2 (indexer keys + selected KV rows per step >> 126 MB)"},
-        "algorithmic_gb_per_step": total_bytes / 1e9,
-        "step_hbm_gbs": total_bytes / (ms / 1e3) / 1e9,
-        "roofline": roof,
-        "e2e": {"value": q_per_step * world / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": launches_per_step(w, [sd["n_split"] for sd in sds]) * args.steps,
-        "clocks": clk.summary(),
-    }
-    return res, w, wt
+    return {"value": q_per_step * world / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d_bytes,
+            "d2h_bytes_per_step": d2h_bytes, "ms_per_step": e2e_ms}
 
 
 def indexer_traffic(kern: str, idx_bytes: float):
-    """DRAM bytes per launch of the flat tensor-core indexer, from the committed ncu capture.
+    """DRAM bytes per launch of the flat tensor-core indexer, from the committed ncu figures.
 
-    The capture's summary (profiles/kernels_decode_cli_128k_batch8.md) records the ratio of
-    measured DRAM traffic to algorithmic bytes on a small case and the SHA-256 of the kernel
-    source it was taken on; the ratio is applied only while the source still has that hash
-    (otherwise the counters describe another kernel and the field is null)."""
+    profiles/indexer_traffic.json records the ratio of measured DRAM traffic to algorithmic
+    bytes on a small case of the same kernel and the SHA-256 of the kernel source it was taken
+    on; the ratio is applied only while the source still has that hash (otherwise the counters
+    describe another kernel and the field is null)."""
     import hashlib
-    import re
     if not kern.startswith("index_score"):
         return None
     try:
-        txt = open(os.path.join(ROOT, "profiles", "kernels_decode_cli_128k_batch8.md")).read()
-        m = re.search(r"indexer_traffic_ratio=([0-9.]+) source_sha256=([0-9a-f]{64})", txt)
+        with open(os.path.join(ROOT, "profiles", "indexer_traffic.json")) as f:
+            d = json.load(f)
         src = open(os.path.join(ROOT, "long_context_sparse_indexer_b200", "csrc", "index_score_tc.cu"), "rb").read()
-    except OSError:
+    except (OSError, ValueError):
         return None
-    if not m or hashlib.sha256(src).hexdigest() != m.group(2):
+    if hashlib.sha256(src).hexdigest() != d.get("source_sha256"):
         return None
-    return float(m.group(1)) * idx_bytes
+    return float(d["dram_bytes_over_algorithmic"]) * idx_bytes
 
 
 # ------------------------------------------------------------------ the CPU oracle (baseline / reference arm)
@@ -500,6 +555,11 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the sequence count (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="measure only --workload (by default a single-GPU run of the 128K decode also measures the "
+                         "1M-context HI decode and the 32K prefill chunk)")
+    ap.add_argument("--load-ms", type=float, default=250.0,
+                    help="untimed sustained load before each timed region (clock samples at steady state)")
     ap.add_argument("--slots", type=int, default=2, help="device buffer slots of the host-buffer pipeline")
     ap.add_argument("--idx-q8", action="store_true", help="indexer in FP8-query mode (lsa_index_score_q8)")
     ap.add_argument("--n-split", default="", help="override the split-KV chunk count: one value, or one per pass")
@@ -514,14 +574,31 @@ def main():
         if res is not None:
             print(json.dumps(res), flush=True)
         return
+    torch.cuda.set_device(local_rank)
     if world > 1:
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    res, w, wt = run_gpu(args, rank, world, local_rank)
+    head, w = measure(args.workload, args, rank, world, local_rank, headline=True)
+    res = {
+        "metric": METRIC, "value": head["value"], "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16+fp8", "data": "synthetic (seeded counter-based generator)",
+        "config": head["config"],
+        "algorithmic_gb_per_step": head["algorithmic_gb_per_step"], "step_hbm_gbs": head["step_hbm_gbs"],
+        "step_hbm_frac": head["step_hbm_frac"],
+        "roofline": head["roofline"], "attention_roofline": head["attention_roofline"],
+        "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+    }
+    if world == 1 and not args.no_extras and args.workload == "decode_cli_128k" and not args.batch:
+        # The metric names two context lengths (128K and 1M); the prefill chunk carries the tensor
+        # roofline.  Each is measured the same way (graph, warm-up, sustained load, K timed steps).
+        res["workloads"] = {}
+        for nm in ("decode_hi_1m", "prefill_32k"):
+            r, _ = measure(nm, args, rank, world, local_rank, headline=False)
+            res["workloads"][nm] = r
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             n, dt = oracle_sample(W.WORKLOADS[args.workload], 2, min_seconds=10.0)

@@ -127,18 +127,25 @@ lsa_status lsa_index_score_q8(const lsa_batch* batch, const void* q_idx, const f
  * Block key of block j of sequence b = arithmetic mean of the dequantised indexer keys
  * of rows j*block_size .. min(seq_len[b], (j+1)*block_size) - 1 ([release] HI bullet:
  * block-level approximate scoring; the mean is this library's block summary).
- *   kbar [B][*][d_I] float, sequence b at kbar + b * kbar_seq_stride; blocks
- *   0 .. ceil(seq_len[b] / block_size) - 1 are written.  Cache maintenance: rerun for the
- *   blocks whose rows changed (here: all). */
+ *   kbar: BF16 bits, sequence b at kbar + b * kbar_seq_stride (uint16 elements), 2 * d_I
+ *   per block: row j holds hi[0..d_I) then lo[0..d_I), where m is the mean computed in FP32
+ *   (fixed pairwise summation order), hi = m rounded to BF16 and lo = (m - hi) rounded to
+ *   BF16; the block key is hi + lo (16 significant bits, relative error <= 2^-17 of m).
+ *   Blocks 0 .. ceil(seq_len[b] / block_size) - 1 are written.  Requires
+ *   kbar_seq_stride >= ceil(L_alloc / block_size) * 2 * d_I, a multiple of 8, and kbar
+ *   16-byte aligned.  Cache maintenance: rerun for the blocks whose rows changed (here: all). */
 lsa_status lsa_block_keys(const lsa_batch* batch, const lsa_cache* k_idx, int block_size,
-                          float* kbar, int64_t kbar_seq_stride, int32_t* dev_status, void* stream);
+                          void* kbar, int64_t kbar_seq_stride, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------- a2: HI block scores
- * J(t,j) = sum_h w[t,h] * ReLU(q_idx[t,h,:] . kbar[q_seq[t], j, :]) for block columns
- * j < n_cols: the score when block j is visible (j * block_size <= q_pos[t]), else
- * -INFINITY.  d_I = dimension of q_idx rows (64 or 128). */
+ * J(t,j) = sum_h w[t,h] * ReLU(q_idx[t,h,:] . kbar(q_seq[t], j)) for block columns
+ * j < n_cols, kbar(b, j) = hi + lo as written by lsa_block_keys: the score when block j is
+ * visible (j * block_size <= q_pos[t]), else -INFINITY.  d_I = dimension of q_idx rows
+ * (64 or 128).  Same layout requirements on kbar as lsa_block_keys.  For H_I a multiple of
+ * 32 the scores come from the tensor cores (BF16 MMA over K = 2 d_I: [hi | lo] against
+ * [q | q], exact products, FP32 accumulation); otherwise from FP32 CUDA-core dot products. */
 lsa_status lsa_block_score(const lsa_batch* batch, const void* q_idx, const float* w, int H_I, int d_I,
-                           const float* kbar, int64_t kbar_seq_stride, int block_size,
+                           const void* kbar, int64_t kbar_seq_stride, int block_size,
                            float* scores, int64_t ld_scores, int n_cols,
                            int32_t* dev_status, void* stream);
 
@@ -240,8 +247,8 @@ typedef struct {
     int32_t          k, n_sink, window;
     /* hierarchical indexing (hi != 0): block keys kbar from lsa_block_keys */
     int32_t          hi, block_size, n_recall;
-    const float*     kbar;
-    int64_t          kbar_seq_stride;
+    const void*      kbar;            /* BF16 (hi, lo) pairs, as written by lsa_block_keys */
+    int64_t          kbar_seq_stride; /* uint16 elements between sequences */
     /* attention layers sharing the index */
     int32_t          H, Dqk, Dv;
     float            sm_scale;

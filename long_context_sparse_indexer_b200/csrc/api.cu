@@ -251,14 +251,15 @@ lsa_status lsa_index_score_q8(const lsa_batch* batch, const void* q_idx, const f
                             n_cols, dev_status, static_cast<cudaStream_t>(stream), true);
 }
 
-lsa_status lsa_block_keys(const lsa_batch* batch, const lsa_cache* k_idx, int block_size, float* kbar,
+lsa_status lsa_block_keys(const lsa_batch* batch, const lsa_cache* k_idx, int block_size, void* kbar,
                           int64_t kbar_seq_stride, int32_t* dev_status, void* stream) {
     lsa_status s = check_batch(batch);
     if (s != LSA_OK) return s;
     if ((s = check_cache(k_idx, 0)) != LSA_OK) return s;
     if (!kbar || block_size < 1 || block_size > 1024 || k_idx->dim > 1024) return LSA_ERR_INVALID_ARG;
     const int64_t nblk = (batch->L_alloc + block_size - 1) / block_size;
-    if (kbar_seq_stride < nblk * k_idx->dim || ((uintptr_t)kbar & 15)) return LSA_ERR_INVALID_ARG;
+    if (kbar_seq_stride < nblk * 2 * k_idx->dim || kbar_seq_stride % 8 || ((uintptr_t)kbar & 15)) return LSA_ERR_INVALID_ARG;
+    if (!batch->seq_len) return LSA_ERR_INVALID_ARG;
     BlockKeyArgs a{};
     a.seq_len = batch->seq_len; a.B = batch->B; a.L_alloc = batch->L_alloc;
     const int eb = elem_bytes(k_idx->dtype);
@@ -267,27 +268,27 @@ lsa_status lsa_block_keys(const lsa_batch* batch, const lsa_cache* k_idx, int bl
     a.seq_stride_b = k_idx->seq_stride * eb; a.tok_stride_b = k_idx->tok_stride * eb;
     a.scale_seq_stride = k_idx->scale_seq_stride;
     a.d_I = k_idx->dim; a.block_size = block_size; a.fp8 = k_idx->dtype == LSA_FP8_E4M3;
-    a.kbar = kbar; a.kbar_seq_stride = kbar_seq_stride; a.status = dev_status;
-    if (!batch->seq_len) return LSA_ERR_INVALID_ARG;
+    a.kbar = static_cast<uint16_t*>(kbar); a.kbar_seq_stride = kbar_seq_stride; a.status = dev_status;
     return cuda_status(launch_block_keys(a, static_cast<cudaStream_t>(stream)));
 }
 
 lsa_status lsa_block_score(const lsa_batch* batch, const void* q_idx, const float* w, int H_I, int d_I,
-                           const float* kbar, int64_t kbar_seq_stride, int block_size, float* scores,
+                           const void* kbar, int64_t kbar_seq_stride, int block_size, float* scores,
                            int64_t ld_scores, int n_cols, int32_t* dev_status, void* stream) {
     lsa_status s = check_batch(batch);
     if (s != LSA_OK) return s;
     if (!supported_hi(H_I) || (d_I != 64 && d_I != 128)) return LSA_ERR_UNSUPPORTED;
     if (block_size < 1 || n_cols < 0 || n_cols > ld_scores) return LSA_ERR_INVALID_ARG;
     const int64_t nblk = (batch->L_alloc + block_size - 1) / block_size;
-    if (n_cols > nblk || kbar_seq_stride < nblk * d_I) return LSA_ERR_INVALID_ARG;
+    if (n_cols > nblk || kbar_seq_stride < nblk * 2 * d_I || kbar_seq_stride % 8) return LSA_ERR_INVALID_ARG;
     if (batch->T == 0) return LSA_OK;
-    if (!q_idx || !w || !kbar || !scores || ((uintptr_t)kbar & 15) || (kbar_seq_stride % 4)) return LSA_ERR_INVALID_ARG;
+    if (!q_idx || !w || !kbar || !scores || ((uintptr_t)kbar & 15) || ((uintptr_t)q_idx & 15)) return LSA_ERR_INVALID_ARG;
     BlockScoreArgs a{};
     a.seq_len = batch->seq_len; a.q_seq = batch->q_seq; a.q_pos = batch->q_pos;
-    a.B = batch->B; a.T = batch->T; a.L_alloc = batch->L_alloc;
+    a.B = batch->B; a.T = batch->T; a.L_alloc = batch->L_alloc; a.q_group = batch->q_group;
     a.q = static_cast<const uint16_t*>(q_idx); a.w = w;
-    a.kbar = kbar; a.kbar_seq_stride = kbar_seq_stride; a.d_I = d_I; a.block_size = block_size;
+    a.kbar = static_cast<const uint16_t*>(kbar); a.kbar_seq_stride = kbar_seq_stride; a.L_blocks = (int)nblk;
+    a.d_I = d_I; a.block_size = block_size;
     a.scores = scores; a.ld = ld_scores; a.n_cols = n_cols; a.status = dev_status;
     return cuda_status(launch_block_score(a, H_I, static_cast<cudaStream_t>(stream)));
 }

@@ -33,8 +33,8 @@ struct BlockKeyArgs {
     int64_t seq_stride_b, tok_stride_b, scale_seq_stride;
     int d_I, block_size;
     bool fp8;
-    float* kbar;
-    int64_t kbar_seq_stride;
+    uint16_t* kbar;          // [B][*][2][d_I] bf16 bits: (hi, lo) of each block key
+    int64_t kbar_seq_stride; // uint16 elements between sequences
     int32_t* status;
 };
 
@@ -45,8 +45,10 @@ struct BlockScoreArgs {
     int B, T, L_alloc;
     const uint16_t* q;   // bf16 [T][H_I][d_I]
     const float* w;      // [T][H_I]
-    const float* kbar;
-    int64_t kbar_seq_stride;
+    const uint16_t* kbar;    // [B][*][2][d_I] bf16 bits (hi, lo)
+    int64_t kbar_seq_stride; // uint16 elements between sequences
+    int L_blocks;            // block rows allocated per sequence (ceil(L_alloc / block_size))
+    int q_group;
     int d_I, block_size;
     float* scores;
     int64_t ld;

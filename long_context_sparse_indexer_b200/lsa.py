@@ -180,8 +180,16 @@ def index_score(batch: Batch, q_idx: torch.Tensor, w: torch.Tensor, k_idx: Cache
               int(n_cols), _ptr(dev_status), _stream(stream)), name)
 
 
+def block_keys_buffer(B: int, L_alloc: int, block_size: int, d_I: int, device) -> torch.Tensor:
+    """An (uninitialised) block-key buffer in the layout lsa_block_keys writes:
+    [B, ceil(L_alloc / block_size), 2 * d_I] BF16, each row the (hi, lo) halves of one block key."""
+    nblk = (L_alloc + block_size - 1) // block_size
+    return torch.empty((B, nblk, 2 * d_I), dtype=torch.bfloat16, device=device)
+
+
 def block_keys(batch: Batch, k_idx: Cache, block_size: int, kbar: torch.Tensor,
                dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """lsa_block_keys into `kbar` (see block_keys_buffer for its layout)."""
     cb, ck = batch.c(), k_idx.c()
     _check(_lib.lsa_block_keys(ctypes.byref(cb), ctypes.byref(ck), int(block_size), _ptr(kbar), int(kbar.stride(0)),
                                _ptr(dev_status), _stream(stream)), "lsa_block_keys")

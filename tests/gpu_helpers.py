@@ -37,10 +37,17 @@ def flat_scores(wt: D.WorkloadTensors, pi: int = 0, status=None, q_fp8: bool = F
 
 def block_keys(wt: D.WorkloadTensors, pi: int = 0, status=None) -> torch.Tensor:
     w = wt.w
-    nblk = (wt.L_alloc + w.block_size - 1) // w.block_size
-    kbar = torch.zeros((w.B, nblk, w.d_I), dtype=torch.float32, device=wt.seq_len.device)
+    kbar = lsa.block_keys_buffer(w.B, wt.L_alloc, w.block_size, w.d_I, wt.seq_len.device)
+    kbar.zero_()
     lsa.block_keys(batch_of(wt, pi), idx_cache(wt, pi), w.block_size, kbar, dev_status=status)
     return kbar
+
+
+def block_key_values(kbar: torch.Tensor) -> np.ndarray:
+    """The block keys a block-key buffer holds, hi + lo, in float64: [B, nblk, d_I]."""
+    x = kbar.float().cpu().numpy().astype(np.float64)
+    d = x.shape[-1] // 2
+    return x[..., :d] + x[..., d:]
 
 
 def decode_step(wt: D.WorkloadTensors, pi: int = 0, n_split: int = 1, kbar=None, cap_extra: int = 0,
