@@ -224,6 +224,81 @@ lsa_status lsa_sparse_attn_noalloc(const lsa_batch* batch, const void* q, int H,
                                    float sm_scale, int n_split, void* o, float* lse,
                                    int32_t* dev_status, void* stream);
 
+/* ---------------------------------------------------------------- partial attention and its merge
+ * lsa_sparse_attn with the result in FP32 and not normalised across calls: o_part [T][H][Dv]
+ * float and lse_part [T][H] float (both required), the attention of each (token, head) over the
+ * rows of its list only.  The partial results of disjoint row sets combine with
+ * lsa_merge_partials ([explainer] "③ KVP 解码切分示意": per-shard partial attention, then the
+ * merge).  Same arguments, workspace and determinism as lsa_sparse_attn otherwise. */
+lsa_status lsa_sparse_attn_partial(const lsa_batch* batch, const void* q, int H, int Dqk,
+                                   const lsa_cache* kv, const lsa_cache* v, int Dv,
+                                   const int32_t* idx, int64_t ld_idx, const int32_t* count,
+                                   float sm_scale, int n_split, float* o_part, float* lse_part,
+                                   void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* Log-sum-exp merge of n_parts partial attentions over disjoint row sets, in part order:
+ * with m = max_p lse_p and w_p = exp(lse_p - m), o = sum_p (w_p / sum w) o_p and
+ * lse = m + log(sum w); a part with lse = -inf (no rows) contributes nothing, and all parts
+ * empty give o = 0, lse = -inf.  o_parts [n_parts][T][H][Dv] float, lse_parts [n_parts][T][H]
+ * float, o [T][H][Dv] BF16 (rounded to nearest even), lse [T][H] float or NULL.  Dv a multiple of
+ * 8, 16-byte aligned o_parts and o; 1 <= n_parts <= 1024. */
+lsa_status lsa_merge_partials(const float* o_parts, const float* lse_parts, int n_parts, int T, int H, int Dv,
+                              void* o, float* lse, void* stream);
+
+/* ---------------------------------------------------------------- KVP: one context over several ranks
+ * [explainer] "③ KVP 解码切分示意" and [release] "推理" (decode nodes): the KV cache of a long
+ * sequence is split over devices, each computes partial results over its shard, and the partial
+ * results are merged.  Shard r of sequence b is the contiguous row range
+ * shard_start[b] .. shard_start[b] + shard_len[b] - 1; the rank that holds it stores those rows as
+ * rows 0 .. shard_len[b] - 1 of its own caches (indexer keys and KV).  Shards of a sequence are
+ * disjoint, cover 0 .. seq_len[b] - 1 and are numbered in position order.  One step over R shards:
+ *   1. lsa_kvp_shard_batch: the shard's local batch (local lengths and positions);
+ *   2. lsa_index_score with the local batch and caches: the shard's scores;
+ *   3. lsa_kvp_candidates: the shard's top-k as (global position, score) pairs;
+ *   4. the caller gathers every shard's candidates, in shard order (an all-gather over ranks);
+ *   5. lsa_kvp_select: the global top-k with sinks and window, the same on every rank and the same
+ *      list as the single-device selection (each key of the global top-k is in the top-k of its
+ *      shard, and the order (score desc, position asc) is kept);
+ *   6. lsa_kvp_local_index: the selected rows of this shard, as local rows;
+ *   7. lsa_sparse_attn_partial with the local batch and caches;
+ *   8. the caller gathers every shard's partial results, in shard order;
+ *   9. lsa_merge_partials.
+ * Only the plain union (no LSA_TOPK_EXCLUDES_FIXED) and flat indexing are covered. */
+
+/* local_seq_len[b] = shard_len[b]; local_q_pos[t] = clamp(q_pos[t] - shard_start[b], 0,
+ * shard_len[b] - 1) (device [B] and [T] outputs).  The local batch is the global one with these
+ * two arrays and L_alloc_local.  A shard outside 0 .. seq_len[b] - 1, or longer than
+ * L_alloc_local, is bad device data. */
+lsa_status lsa_kvp_shard_batch(const lsa_batch* global, int L_alloc_local, const int32_t* shard_start,
+                               const int32_t* shard_len, int32_t* local_seq_len, int32_t* local_q_pos,
+                               int32_t* dev_status, void* stream);
+
+/* The top-k of the shard's local scores (scores [T][ld_scores], columns = local rows, as
+ * lsa_index_score wrote them for the local batch) as global positions, ascending, and their
+ * scores: cand_pos [T][k] int32 and cand_score [T][k] float, padded with (-1, -INFINITY);
+ * cand_count [T] the number of pairs.  A token whose global position q_pos_global[t] precedes the
+ * shard sees none of its keys and gets no pair. */
+lsa_status lsa_kvp_candidates(const lsa_batch* local, const int32_t* q_pos_global, const int32_t* shard_start,
+                              const float* scores, int64_t ld_scores, int n_cols, int k, int32_t* cand_pos,
+                              float* cand_score, int32_t* cand_count, int32_t* dev_status, void* stream);
+
+/* The global selection from every shard's candidates: cand_pos / cand_score [n_parts][T][k_part]
+ * in shard order (as lsa_kvp_candidates wrote them, gathered).  The k pairs ranked first by
+ * (score desc, position asc), unioned with the sinks and the window of the global batch, as
+ * lsa_topk's default mode: idx [T][ld_idx] ascending, -1 padded, count [T].
+ * ws: lsa_kvp_select_workspace_size(T, n_parts, k_part) bytes, 256-byte aligned. */
+size_t lsa_kvp_select_workspace_size(int T, int n_parts, int k_part);
+lsa_status lsa_kvp_select(const lsa_batch* global, const int32_t* cand_pos, const float* cand_score, int n_parts,
+                          int k_part, int k, int n_sink, int window, int32_t* idx, int64_t ld_idx, int32_t* count,
+                          void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* The entries of each token's global list idx[t][0..count[t]) that fall in the shard, minus
+ * shard_start (local rows, ascending): local_idx [T][ld_local] (-1 padded), local_count [T].
+ * ld_local >= ld_idx. */
+lsa_status lsa_kvp_local_index(const lsa_batch* global, const int32_t* shard_start, const int32_t* shard_len,
+                               const int32_t* idx, int64_t ld_idx, const int32_t* count, int32_t* local_idx,
+                               int64_t ld_local, int32_t* local_count, int32_t* dev_status, void* stream);
+
 /* ---------------------------------------------------------------- fused decode / prefill step
  * One attention layer consuming a shared index list (cross-layer indexing: [release] CLI
  * bullet, one index serves consecutive layers; MTP paragraph, draft steps 2 and 3 reuse

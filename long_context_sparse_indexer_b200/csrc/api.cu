@@ -138,12 +138,15 @@ lsa_status lsa::attn_validate(const lsa_batch* batch, const void* q, int H, int 
 
 namespace {
 
+// o32 / lse32 (FP32 result, both given) replace o / lse when not NULL.
 lsa_status attn_impl(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,
                      const lsa_cache* v, int Dv, const int32_t* idx, int64_t ld_idx, const int32_t* count,
                      float sm_scale, int n_split, void* o, float* lse, void* ws, size_t ws_bytes,
-                     int32_t* st, cudaStream_t stream) {
-    lsa_status s = attn_validate(batch, q, H, Dqk, kv, v, Dv, idx, ld_idx, count, sm_scale, n_split, o);
+                     int32_t* st, cudaStream_t stream, float* o32 = nullptr, float* lse32 = nullptr) {
+    lsa_status s = attn_validate(batch, q, H, Dqk, kv, v, Dv, idx, ld_idx, count, sm_scale, n_split,
+                                 o32 ? static_cast<const void*>(o32) : o);
     if (s != LSA_OK || batch->T == 0) return s;
+    if (o32 && (!lse32 || ((uintptr_t)lse32 & 3))) return LSA_ERR_INVALID_ARG;
     const bool sep_v = v && v->data;
     const size_t need = attn_ws(batch->T, H, Dv, n_split);
     if (need && (!ws || ws_bytes < need || ((uintptr_t)ws % kAlign))) return LSA_ERR_WORKSPACE;
@@ -168,6 +171,12 @@ lsa_status attn_impl(const lsa_batch* batch, const void* q, int H, int Dqk, cons
     if (n_split > 1) {
         a.part_o = static_cast<float*>(ws);
         a.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up((size_t)batch->T * n_split * H * Dv * 4));
+    }
+    if (o32) {                    // FP32 result: one split writes it directly, more splits merge into it
+        a.f32_out = 1;
+        a.o32 = o32;
+        a.lse32 = lse32;
+        if (n_split == 1) { a.part_o = o32; a.part_lse = lse32; }
     }
     a.status = st;
     return cuda_status(launch_sparse_attn(a, Dqk, Dv, kv->dtype == LSA_FP8_E4M3, sep_v, stream));
@@ -391,6 +400,95 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
     }
     if (s != LSA_OK) return s;
     return LSA_OK;
+}
+
+lsa_status lsa_sparse_attn_partial(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,
+                                   const lsa_cache* v, int Dv, const int32_t* idx, int64_t ld_idx,
+                                   const int32_t* count, float sm_scale, int n_split, float* o_part, float* lse_part,
+                                   void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    if (batch && batch->T > 0 && (!o_part || !lse_part)) return LSA_ERR_INVALID_ARG;
+    return attn_impl(batch, q, H, Dqk, kv, v, Dv, idx, ld_idx, count, sm_scale, n_split, nullptr, nullptr, ws,
+                     ws_bytes, dev_status, static_cast<cudaStream_t>(stream), o_part, lse_part);
+}
+
+lsa_status lsa_merge_partials(const float* o_parts, const float* lse_parts, int n_parts, int T, int H, int Dv,
+                              void* o, float* lse, void* stream) {
+    if (n_parts < 1 || n_parts > 1024 || T < 0 || H < 1 || Dv < 8 || Dv % 8) return LSA_ERR_INVALID_ARG;
+    if (T > kMaxTokens) return LSA_ERR_UNSUPPORTED;
+    if (T == 0) return LSA_OK;
+    if (!o_parts || !lse_parts || !o || !aligned16(o_parts) || !aligned16(o)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_merge_partials(o_parts, lse_parts, n_parts, (int64_t)T * H, H, T, H, Dv,
+                                             static_cast<uint16_t*>(o), nullptr, lse,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+lsa_status lsa_kvp_shard_batch(const lsa_batch* global, int L_alloc_local, const int32_t* shard_start,
+                               const int32_t* shard_len, int32_t* local_seq_len, int32_t* local_q_pos,
+                               int32_t* dev_status, void* stream) {
+    lsa_status s = check_batch(global);
+    if (s != LSA_OK) return s;
+    if (L_alloc_local < 1 || !shard_start || !shard_len || !local_seq_len || (global->T > 0 && !local_q_pos))
+        return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_kvp_shard_batch(global->B, global->T, L_alloc_local, global->seq_len, global->q_seq,
+                                              global->q_pos, shard_start, shard_len, local_seq_len, local_q_pos,
+                                              dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+lsa_status lsa_kvp_candidates(const lsa_batch* local, const int32_t* q_pos_global, const int32_t* shard_start,
+                              const float* scores, int64_t ld_scores, int n_cols, int k, int32_t* cand_pos,
+                              float* cand_score, int32_t* cand_count, int32_t* dev_status, void* stream) {
+    lsa_status s = check_batch(local);
+    if (s != LSA_OK) return s;
+    if (k < 1) return LSA_ERR_INVALID_ARG;
+    if (local->T == 0) return LSA_OK;
+    if (!q_pos_global || !shard_start || !cand_score || !cand_count) return LSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = topk_impl(local, scores, ld_scores, n_cols, nullptr, 0, 0, k, 0, 0, LSA_TOPK_RAW, cand_pos, k, cand_count,
+                  dev_status, st);
+    if (s != LSA_OK) return s;
+    return cuda_status(launch_kvp_candidates(local->T, k, local->q_seq, q_pos_global, shard_start, local->B, scores,
+                                             ld_scores, cand_count, cand_pos, cand_score, st));
+}
+
+size_t lsa_kvp_select_workspace_size(int T, int n_parts, int k_part) {
+    if (T < 0 || n_parts < 0 || k_part < 0) return 0;
+    const size_t n = (size_t)T * n_parts * k_part;
+    return align_up(n * 4) + align_up(n * 4);
+}
+
+lsa_status lsa_kvp_select(const lsa_batch* global, const int32_t* cand_pos, const float* cand_score, int n_parts,
+                          int k_part, int k, int n_sink, int window, int32_t* idx, int64_t ld_idx, int32_t* count,
+                          void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    lsa_status s = check_batch(global);
+    if (s != LSA_OK) return s;
+    if (n_parts < 1 || k_part < 1 || (int64_t)n_parts * k_part > 0x7fffffff) return LSA_ERR_INVALID_ARG;
+    if (global->T == 0) return LSA_OK;
+    if (!cand_pos || !cand_score) return LSA_ERR_INVALID_ARG;
+    const size_t need = lsa_kvp_select_workspace_size(global->T, n_parts, k_part);
+    if (!ws || ws_bytes < need || ((uintptr_t)ws % kAlign)) return LSA_ERR_WORKSPACE;
+    const int n = n_parts * k_part;
+    int32_t* pos_row = static_cast<int32_t*>(ws);
+    float* score_row = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up((size_t)global->T * n * 4));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = cuda_status(launch_kvp_gather(global->T, n_parts, k_part, cand_pos, cand_score, pos_row, score_row, st));
+    if (s != LSA_OK) return s;
+    // Columns in part order, each part's positions ascending and the parts' ranges ascending: the
+    // column order is the position order, so the (score desc, column asc) selection of lsa_topk is
+    // the (score desc, position asc) one; each column maps to its position as a block of one row.
+    return topk_impl(global, score_row, n, n, pos_row, n, 1, k, n_sink, window, 0, idx, ld_idx, count, dev_status, st);
+}
+
+lsa_status lsa_kvp_local_index(const lsa_batch* global, const int32_t* shard_start, const int32_t* shard_len,
+                               const int32_t* idx, int64_t ld_idx, const int32_t* count, int32_t* local_idx,
+                               int64_t ld_local, int32_t* local_count, int32_t* dev_status, void* stream) {
+    lsa_status s = check_batch(global);
+    if (s != LSA_OK) return s;
+    if (ld_idx < 1 || ld_local < ld_idx) return LSA_ERR_INVALID_ARG;
+    if (global->T == 0) return LSA_OK;
+    if (!shard_start || !shard_len || !idx || !count || !local_idx || !local_count) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_kvp_local_index(global->T, global->B, global->q_seq, shard_start, shard_len, idx, ld_idx,
+                                              count, local_idx, ld_local, local_count, dev_status,
+                                              static_cast<cudaStream_t>(stream)));
 }
 
 lsa_status lsa_read_device_status(const int32_t* dev_status, void* stream) {

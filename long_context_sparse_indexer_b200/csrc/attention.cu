@@ -254,7 +254,7 @@ sparse_attn_kernel(AttnArgs a) {
         lse_v[hf] = l_run[hf] > 0.f ? (m_run[hf] + log2f(l_run[hf])) * kLn2 : kNegInf;
     }
     const int dv0 = qw * (DV / 4);
-    if (a.n_split == 1) {
+    if (a.n_split == 1 && !a.f32_out) {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             const int h = h0 + g + 8 * hf;
@@ -282,17 +282,22 @@ sparse_attn_kernel(AttnArgs a) {
 // Split merge: thread = 8 consecutive V dims of one (token, head).  With m = max_s lse_s and
 // w_s = exp(lse_s - m): o = sum_s (w_s / sum w) o_s and lse = m + log(sum w), sums in split
 // order.  Up to kMergeRegs splits are loaded before any arithmetic (one memory round trip).
+// Partial s of (token t, head h) is row s * part_stride + t * tok_stride + h; the splits of one
+// call are [T][n_split][H] (part_stride = H, tok_stride = n_split * H), the per-rank partials of
+// KVP [n_part][T][H] (part_stride = T * H, tok_stride = H).
 constexpr int kMergeThreads = 256;
 constexpr int kMergeRegs = 8;
 
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* part_o, const float* part_lse,
-                                                              int n_split, int H, int DV, uint16_t* o, float* lse) {
+                                                              int n_split, int H, int DV, int64_t part_stride,
+                                                              int64_t tok_stride, uint16_t* o, float* o32,
+                                                              float* lse) {
     const int per_row = DV / 8;
     const int i = blockIdx.x * kMergeThreads + threadIdx.x;       // (head, 8-dim chunk) of token t
     const int t = blockIdx.y;
     if (i >= H * per_row) return;
     const int h = i / per_row, d = (i % per_row) * 8;
-    const size_t row0 = (size_t)t * n_split * H + h;               // (split 0, head h)
+    const size_t row0 = (size_t)t * tok_stride + h;                // (split 0, head h)
     float m = kNegInf, wsum = 0.f;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (n_split <= kMergeRegs) {
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* part_
 #pragma unroll
         for (int s = 0; s < kMergeRegs; ++s) {
             if (s < n_split) {
-                const size_t r = row0 + (size_t)s * H;
+                const size_t r = row0 + (size_t)s * part_stride;
                 l[s] = __ldcg(part_lse + r);
                 const float4* src = reinterpret_cast<const float4*>(part_o + r * DV + d);
                 x0[s] = __ldcg(src);
@@ -326,14 +331,14 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* part_
             }
         }
     } else {
-        for (int s = 0; s < n_split; ++s) m = fmaxf(m, __ldcg(part_lse + row0 + (size_t)s * H));
+        for (int s = 0; s < n_split; ++s) m = fmaxf(m, __ldcg(part_lse + row0 + (size_t)s * part_stride));
         for (int s = 0; s < n_split; ++s) {
-            const float ls = __ldcg(part_lse + row0 + (size_t)s * H);
+            const float ls = __ldcg(part_lse + row0 + (size_t)s * part_stride);
             wsum += m == kNegInf ? 0.f : expf(ls - m);
         }
         const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
         for (int s = 0; s < n_split; ++s) {
-            const size_t r = row0 + (size_t)s * H;
+            const size_t r = row0 + (size_t)s * part_stride;
             const float ws = (m == kNegInf ? 0.f : expf(__ldcg(part_lse + r) - m)) * rs;
             const float4* src = reinterpret_cast<const float4*>(part_o + r * DV + d);
             const float4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
@@ -343,17 +348,33 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* part_
             acc[6] = fmaf(ws, a1.z, acc[6]); acc[7] = fmaf(ws, a1.w, acc[7]);
         }
     }
-    uint4 pk;
-    pk.x = pack_bf16x2(acc[0], acc[1]); pk.y = pack_bf16x2(acc[2], acc[3]);
-    pk.z = pack_bf16x2(acc[4], acc[5]); pk.w = pack_bf16x2(acc[6], acc[7]);
-    *reinterpret_cast<uint4*>(o + ((size_t)t * H + h) * DV + d) = pk;
+    const size_t out = ((size_t)t * H + h) * DV + d;
+    if (o32) {
+        *reinterpret_cast<float4*>(o32 + out) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(o32 + out + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    } else {
+        uint4 pk;
+        pk.x = pack_bf16x2(acc[0], acc[1]); pk.y = pack_bf16x2(acc[2], acc[3]);
+        pk.z = pack_bf16x2(acc[4], acc[5]); pk.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(o + out) = pk;
+    }
     if (lse && d == 0) lse[(size_t)t * H + h] = wsum > 0.f ? m + logf(wsum) : kNegInf;
 }
 
-static cudaError_t launch_merge(const AttnArgs& a, int DV, cudaStream_t st) {
-    dim3 mg((a.H * (DV / 8) + kMergeThreads - 1) / kMergeThreads, a.T);
-    merge_kernel<<<mg, kMergeThreads, 0, st>>>(a.part_o, a.part_lse, a.n_split, a.H, DV, a.o, a.lse);
+cudaError_t launch_merge_partials(const float* part_o, const float* part_lse, int n_part, int64_t part_stride,
+                                  int64_t tok_stride, int T, int H, int DV, uint16_t* o, float* o32, float* lse,
+                                  cudaStream_t st) {
+    if (T <= 0) return cudaSuccess;
+    dim3 mg((H * (DV / 8) + kMergeThreads - 1) / kMergeThreads, T);
+    merge_kernel<<<mg, kMergeThreads, 0, st>>>(part_o, part_lse, n_part, H, DV, part_stride, tok_stride, o, o32, lse);
     return cudaGetLastError();
+}
+
+// The merge of one call's split partials ([T][n_split][H]) into its BF16 (or FP32) result.
+static cudaError_t launch_merge(const AttnArgs& a, int DV, cudaStream_t st) {
+    return launch_merge_partials(a.part_o, a.part_lse, a.n_split, a.H, (int64_t)a.n_split * a.H, a.T, a.H, DV,
+                                 a.f32_out ? nullptr : a.o, a.f32_out ? a.o32 : nullptr,
+                                 a.f32_out ? a.lse32 : a.lse, st);
 }
 
 template <int DQK, int DV, int MT, bool KV_FP8, bool SEP_V>

@@ -598,7 +598,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
         const float lse = l_f > 0.f ? (m_f + log2f(l_f)) * kLn2 : kNegInf;
         // The rows go out through shared memory (the idle KV ring; rows padded by 16 B so that
         // consecutive heads fall in different banks), one bulk copy per head row.
-        const bool bf16_out = a.n_split == 1;
+        const bool bf16_out = a.n_split == 1 && !a.f32_out;
         const int row_bytes = bf16_out ? kHalf * 2 : kHalf * 4, pitch = row_bytes + 16;
         uint8_t* srow = sm.kv[0] + h * pitch;
         const int c_beg = kSmx == 2 ? wg * (kHalf / 64) : 0, c_end = kSmx == 2 ? c_beg + kHalf / 64 : kHalf / 32;
@@ -640,7 +640,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             tc::bulk_wait_all();
         }
         if (half == 0 && wg == 0) {
-            if (a.n_split == 1) { if (a.lse) a.lse[(size_t)t * 128 + h] = lse; }
+            if (bf16_out) { if (a.lse) a.lse[(size_t)t * 128 + h] = lse; }
             else a.part_lse[((size_t)t * a.n_split + split) * 128 + h] = lse;
         }
     } else if (send_warp) {

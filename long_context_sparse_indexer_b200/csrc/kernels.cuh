@@ -94,8 +94,11 @@ struct AttnArgs {
     int n_split;
     uint16_t* o;                // [T][H][DV] bf16
     float* lse;                 // [T][H] or NULL
-    float* part_o;              // [T][n_split][H][DV] (n_split > 1)
+    float* part_o;              // [T][n_split][H][DV] (n_split > 1, or f32_out)
     float* part_lse;            // [T][n_split][H]
+    int f32_out;                // the result in FP32: o32 / lse32 instead of o / lse
+    float* o32;                 // [T][H][DV] (f32_out)
+    float* lse32;               // [T][H] (f32_out)
     int32_t* status;
 };
 
@@ -108,6 +111,26 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int DQK, int DV, bool kv_fp8, bool sep_v, cudaStream_t st);
 bool sparse_attn_tc_supported(const AttnArgs& a, int DQK, int DV, bool sep_v);
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, bool kv_fp8, cudaStream_t st);
+// Log-sum-exp merge of n_part partial attentions: partial p of (token t, head h) at row
+// p * part_stride + t * tok_stride + h of part_o ([row][DV]) and part_lse; result BF16 (o) or
+// FP32 (o32), lse optional.
+cudaError_t launch_merge_partials(const float* part_o, const float* part_lse, int n_part, int64_t part_stride,
+                                  int64_t tok_stride, int T, int H, int DV, uint16_t* o, float* o32, float* lse,
+                                  cudaStream_t st);
+
+// KVP helpers (kvp.cu).
+cudaError_t launch_kvp_shard_batch(int B, int T, int L_alloc_local, const int32_t* seq_len, const int32_t* q_seq,
+                                   const int32_t* q_pos, const int32_t* shard_start, const int32_t* shard_len,
+                                   int32_t* local_seq_len, int32_t* local_q_pos, int32_t* status, cudaStream_t st);
+cudaError_t launch_kvp_candidates(int T, int k, const int32_t* q_seq, const int32_t* q_pos,
+                                  const int32_t* shard_start, int B, const float* scores, int64_t ld,
+                                  const int32_t* count, int32_t* cand_pos, float* cand_score, cudaStream_t st);
+cudaError_t launch_kvp_gather(int T, int n_parts, int k_part, const int32_t* cand_pos, const float* cand_score,
+                              int32_t* pos_out, float* score_out, cudaStream_t st);
+cudaError_t launch_kvp_local_index(int T, int B, const int32_t* q_seq, const int32_t* shard_start,
+                                   const int32_t* shard_len, const int32_t* idx, int64_t ld_idx,
+                                   const int32_t* count, int32_t* local_idx, int64_t ld_local, int32_t* local_count,
+                                   int32_t* status, cudaStream_t st);
 
 // Host-side checks of lsa_sparse_attn's arguments other than its workspace (api.cu).
 lsa_status attn_validate(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,

@@ -81,6 +81,16 @@ _lib.lsa_decode_fused.argtypes = [_P(CDecodeParams), c_vp, c_size, c_vp, c_vp]
 _lib.lsa_decode_workspace_size.argtypes = [_P(CDecodeParams)]
 _lib.lsa_decode_workspace_size.restype = c_size
 _lib.lsa_read_device_status.argtypes = [c_vp, c_vp]
+_lib.lsa_sparse_attn_partial.argtypes = [_P(CBatch), c_vp, c_i32, c_i32, _P(CCache), _P(CCache), c_i32, c_vp, c_i64,
+                                         c_vp, c_f32, c_i32, c_vp, c_vp, c_vp, c_size, c_vp, c_vp]
+_lib.lsa_merge_partials.argtypes = [c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]
+_lib.lsa_kvp_shard_batch.argtypes = [_P(CBatch), c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]
+_lib.lsa_kvp_candidates.argtypes = [_P(CBatch), c_vp, c_vp, c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]
+_lib.lsa_kvp_select_workspace_size.argtypes = [c_i32, c_i32, c_i32]
+_lib.lsa_kvp_select_workspace_size.restype = c_size
+_lib.lsa_kvp_select.argtypes = [_P(CBatch), c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_vp,
+                                c_size, c_vp, c_vp]
+_lib.lsa_kvp_local_index.argtypes = [_P(CBatch), c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp]
 
 
 class CCopy(ctypes.Structure):
@@ -96,13 +106,15 @@ _lib.lsa_status_string.argtypes = [c_i32]
 _lib.lsa_status_string.restype = ctypes.c_char_p
 _lib.lsa_version.restype = c_i32
 for _f in ("lsa_index_score", "lsa_index_score_q8", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
-           "lsa_sparse_attn_noalloc", "lsa_decode_fused", "lsa_read_device_status"):
+           "lsa_sparse_attn_noalloc", "lsa_decode_fused", "lsa_read_device_status", "lsa_sparse_attn_partial",
+           "lsa_merge_partials", "lsa_kvp_shard_batch", "lsa_kvp_candidates", "lsa_kvp_select", "lsa_kvp_local_index"):
     getattr(_lib, _f).restype = c_i32
 
 EXPORTS = ("lsa_index_score", "lsa_index_score_q8", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
            "lsa_sparse_attn_noalloc", "lsa_attn_workspace_size", "lsa_decode_fused", "lsa_decode_workspace_size", "lsa_read_device_status",
            "lsa_status_string", "lsa_version", "lsa_pipeline_create", "lsa_pipeline_step", "lsa_pipeline_join",
-           "lsa_pipeline_destroy")
+           "lsa_pipeline_destroy", "lsa_sparse_attn_partial", "lsa_merge_partials", "lsa_kvp_shard_batch",
+           "lsa_kvp_candidates", "lsa_kvp_select_workspace_size", "lsa_kvp_select", "lsa_kvp_local_index")
 
 
 def library() -> ctypes.CDLL:
@@ -253,6 +265,76 @@ def sparse_attn_noalloc(batch: Batch, q: torch.Tensor, kv: Cache, idx: torch.Ten
                                         ctypes.byref(cv) if cv is not None else None, Dv, _ptr(idx),
                                         int(idx.stride(0)), _ptr(count), float(sm_scale), int(n_split), _ptr(o),
                                         _ptr(lse), _ptr(dev_status), _stream(stream)), "lsa_sparse_attn_noalloc")
+
+
+def sparse_attn_partial(batch: Batch, q: torch.Tensor, kv: Cache, idx: torch.Tensor, count: torch.Tensor,
+                        sm_scale: float, o_part: torch.Tensor, lse_part: torch.Tensor, v: Optional[Cache] = None,
+                        Dv: int = 0, n_split: int = 1, ws: Optional[torch.Tensor] = None,
+                        dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """lsa_sparse_attn_partial: sparse_attn with an FP32 result (o_part [T, H, Dv] float, lse_part [T, H])."""
+    cb, ck = batch.c(), kv.c()
+    cv = v.c() if v is not None else None
+    H, Dqk = int(q.shape[1]), int(q.shape[2])
+    Dv = int(Dv or o_part.shape[2])
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.lsa_sparse_attn_partial(ctypes.byref(cb), _ptr(q), H, Dqk, ctypes.byref(ck),
+                                        ctypes.byref(cv) if cv is not None else None, Dv, _ptr(idx),
+                                        int(idx.stride(0)), _ptr(count), float(sm_scale), int(n_split), _ptr(o_part),
+                                        _ptr(lse_part), _ptr(ws), wsb, _ptr(dev_status), _stream(stream)),
+           "lsa_sparse_attn_partial")
+
+
+def merge_partials(o_parts: torch.Tensor, lse_parts: torch.Tensor, o: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                   stream=None) -> None:
+    """lsa_merge_partials: o_parts [R, T, H, Dv] float, lse_parts [R, T, H] -> o [T, H, Dv] bf16 (+ lse)."""
+    R, T, H, Dv = (int(x) for x in o_parts.shape)
+    assert o_parts.is_contiguous() and lse_parts.is_contiguous() and o.is_contiguous()
+    _check(_lib.lsa_merge_partials(_ptr(o_parts), _ptr(lse_parts), R, T, H, Dv, _ptr(o), _ptr(lse), _stream(stream)),
+           "lsa_merge_partials")
+
+
+def kvp_shard_batch(batch: Batch, L_alloc_local: int, shard_start: torch.Tensor, shard_len: torch.Tensor,
+                    local_seq_len: torch.Tensor, local_q_pos: torch.Tensor, dev_status: Optional[torch.Tensor] = None,
+                    stream=None) -> Batch:
+    """lsa_kvp_shard_batch: the shard's local batch (same q_seq, local lengths and positions)."""
+    cb = batch.c()
+    _check(_lib.lsa_kvp_shard_batch(ctypes.byref(cb), int(L_alloc_local), _ptr(shard_start), _ptr(shard_len),
+                                    _ptr(local_seq_len), _ptr(local_q_pos), _ptr(dev_status), _stream(stream)),
+           "lsa_kvp_shard_batch")
+    return Batch(local_seq_len, batch.q_seq, local_q_pos, int(L_alloc_local), batch.q_group)
+
+
+def kvp_candidates(local: Batch, q_pos_global: torch.Tensor, shard_start: torch.Tensor, scores: torch.Tensor,
+                   n_cols: int, k: int, cand_pos: torch.Tensor, cand_score: torch.Tensor, cand_count: torch.Tensor,
+                   dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    cb = local.c()
+    _check(_lib.lsa_kvp_candidates(ctypes.byref(cb), _ptr(q_pos_global), _ptr(shard_start), _ptr(scores),
+                                   int(scores.stride(0)), int(n_cols), int(k), _ptr(cand_pos), _ptr(cand_score),
+                                   _ptr(cand_count), _ptr(dev_status), _stream(stream)), "lsa_kvp_candidates")
+
+
+def kvp_select_workspace_size(T: int, n_parts: int, k_part: int) -> int:
+    return int(_lib.lsa_kvp_select_workspace_size(T, n_parts, k_part))
+
+
+def kvp_select(batch: Batch, cand_pos: torch.Tensor, cand_score: torch.Tensor, k: int, n_sink: int, window: int,
+               idx: torch.Tensor, count: torch.Tensor, ws: torch.Tensor, dev_status: Optional[torch.Tensor] = None,
+               stream=None) -> None:
+    """lsa_kvp_select: cand_pos / cand_score [n_parts, T, k_part] (shard order) -> idx [T, cap], count [T]."""
+    n_parts, _, k_part = (int(x) for x in cand_pos.shape)
+    cb = batch.c()
+    _check(_lib.lsa_kvp_select(ctypes.byref(cb), _ptr(cand_pos), _ptr(cand_score), n_parts, k_part, int(k),
+                               int(n_sink), int(window), _ptr(idx), int(idx.stride(0)), _ptr(count), _ptr(ws),
+                               ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)), "lsa_kvp_select")
+
+
+def kvp_local_index(batch: Batch, shard_start: torch.Tensor, shard_len: torch.Tensor, idx: torch.Tensor,
+                    count: torch.Tensor, local_idx: torch.Tensor, local_count: torch.Tensor,
+                    dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    cb = batch.c()
+    _check(_lib.lsa_kvp_local_index(ctypes.byref(cb), _ptr(shard_start), _ptr(shard_len), _ptr(idx),
+                                    int(idx.stride(0)), _ptr(count), _ptr(local_idx), int(local_idx.stride(0)),
+                                    _ptr(local_count), _ptr(dev_status), _stream(stream)), "lsa_kvp_local_index")
 
 
 @dataclass
