@@ -74,23 +74,37 @@ def topk(scores: np.ndarray, positions: np.ndarray, k: int) -> np.ndarray:
     return positions[order[:max(0, min(k, scores.size))]]
 
 
-def union_fixed(selected: np.ndarray, pos: int, n_sink: int, window: int) -> np.ndarray:
+def window_start(pos: int, window: int, align: int = 0) -> int:
+    """First position of the SI window: pos-window+1 clipped at 0, or -- with ``align`` > 0 -- that
+    position rounded down to a multiple of ``align`` (the block-aligned window).
+
+    [release] SI bullet: the contiguous part of the selection is read with hardware-aligned
+    accesses.  The plain reading keeps the window's extent exactly ``window`` positions; the
+    aligned reading starts it at the row block that holds pos-window+1, so the window covers
+    whole blocks up to the query (``window`` to ``window + align - 1`` positions).
+    """
+    b = max(0, pos - window + 1)
+    return (b // align) * align if align > 0 else b
+
+
+def union_fixed(selected: np.ndarray, pos: int, n_sink: int, window: int, align: int = 0) -> np.ndarray:
     """Ascending, de-duplicated union of the top-k picks, the sinks and the SI window.
 
     Sinks: positions 0..n_sink-1 ([explainer] "① LSA": a few fixed sink tokens keep the
     sparse softmax stable).  Window: the last ``window`` visible positions
     pos-window+1..pos, the contiguous, sequentially read part of the selection budget
-    that streaming-aware indexing adds to the dynamic picks ([release] SI bullet).  Both
-    are clipped to the visible range 0..pos.
+    that streaming-aware indexing adds to the dynamic picks ([release] SI bullet); with
+    ``align``, from ``window_start(pos, window, align)``.  Both are clipped to the visible
+    range 0..pos.
     """
     sinks = np.arange(0, min(n_sink, pos + 1), dtype=np.int64)
-    win = np.arange(max(0, pos - window + 1), pos + 1, dtype=np.int64) if window > 0 else \
+    win = np.arange(window_start(pos, window, align), pos + 1, dtype=np.int64) if window > 0 else \
         np.zeros(0, dtype=np.int64)
     return np.union1d(np.union1d(np.asarray(selected, dtype=np.int64), sinks), win)
 
 
 def union_fixed_budget(scores: np.ndarray, positions: np.ndarray, k: int, pos: int, n_sink: int,
-                       window: int) -> np.ndarray:
+                       window: int, align: int = 0) -> np.ndarray:
     """Fixed-budget SI selection: the sinks and the window as in ``union_fixed``, plus the top-k
     (``topk`` order) of the visible positions OUTSIDE both, so the three sets are disjoint and
     the list holds min(k, outside) + |sinks| + |window| positions, ascending.
@@ -103,10 +117,10 @@ def union_fixed_budget(scores: np.ndarray, positions: np.ndarray, k: int, pos: i
     scores = np.asarray(scores, dtype=np.float64)
     positions = np.asarray(positions, dtype=np.int64)
     a = min(n_sink, pos + 1)
-    b = max(a, pos - window + 1) if window > 0 else pos + 1
+    b = max(a, window_start(pos, window, align)) if window > 0 else pos + 1
     outside = (positions >= a) & (positions < b)
     picks = topk(scores[outside], positions[outside], k)
-    return union_fixed(picks, pos, n_sink, window)
+    return union_fixed(picks, pos, n_sink, window, align)
 
 
 def block_keys(K: np.ndarray, length: int, block_size: int) -> np.ndarray:

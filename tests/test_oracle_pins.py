@@ -389,3 +389,45 @@ def test_fixed_budget_equals_plain_union_when_picks_avoid_the_fixed_sets():
     plain = lsa.union_fixed(lsa.topk(sc, cols, k), pos, n_sink, window)
     budget = lsa.union_fixed_budget(sc, cols, k, pos, n_sink, window)
     assert len(budget) == len(plain) + 1               # the budget spends that pick elsewhere
+
+
+# ------------------------------------------------------------------ block-aligned SI window
+
+def test_aligned_window_brute_force():
+    """The aligned window covers every position from the 64-row block holding pos-W+1 up to pos:
+    brute force over small cases, its extent between W and W + 63, and the plain window when
+    pos-W+1 is itself on a block boundary."""
+    rng = np.random.default_rng(13)
+    for _ in range(300):
+        pos = int(rng.integers(0, 400))
+        W = int(rng.integers(0, 200))
+        ns = int(rng.integers(0, 6))
+        sel = rng.choice(pos + 1, size=int(rng.integers(0, min(pos + 2, 30))), replace=False)
+        first = max(0, pos - W + 1)
+        blk = first - first % 64
+        win = set(range(blk, pos + 1)) if W > 0 else set()
+        want = set(sel.tolist()) | {j for j in range(ns) if j <= pos} | win
+        assert lsa.union_fixed(sel, pos, ns, W, align=64).tolist() == sorted(want)
+        if W > 0:
+            assert W <= len(win) <= W + 63 or len(win) == pos + 1
+        if W > 0 and first % 64 == 0:
+            assert lsa.union_fixed(sel, pos, ns, W, align=64).tolist() == lsa.union_fixed(sel, pos, ns, W).tolist()
+    assert lsa.window_start(1000, 512, 64) == 448 and lsa.window_start(1000, 512) == 489
+    assert lsa.window_start(100, 512, 64) == 0 and lsa.window_start(575, 512, 64) == 64
+
+
+def test_aligned_window_fixed_budget_brute_force():
+    rng = np.random.default_rng(17)
+    for _ in range(300):
+        pos = int(rng.integers(0, 300))
+        k = int(rng.integers(0, 12))
+        n_sink = int(rng.integers(0, 5))
+        window = int(rng.integers(0, 100))
+        sc = rng.integers(0, 4, size=pos + 1).astype(np.float64)
+        got = lsa.union_fixed_budget(sc, np.arange(pos + 1), k, pos, n_sink, window, align=64)
+        sinks = set(range(min(n_sink, pos + 1)))
+        first = max(0, pos - window + 1)
+        win = set(range(first - first % 64, pos + 1)) if window > 0 else set()
+        rest = [j for j in range(pos + 1) if j not in sinks and j not in win]
+        best = sorted(rest, key=lambda j: (-sc[j], j))[:k]
+        assert got.tolist() == sorted(sinks | win | set(best))
