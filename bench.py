@@ -368,21 +368,33 @@ def measure(name, args, rank, world, local_rank, headline):
                          "algorithmic_bytes_per_launch": idx_bytes})
     res["roofline"] = roof
 
-    # Attention of the first pass alone (every layer of the pass, as in the step), against the
-    # tensor roofline when its flops dominate (prefill), else HBM.
-    p0 = w.passes[0]
+    # Attention of the first pass alone, its layers on two streams as in the step (layer l on
+    # branch l mod 2), against the tensor roofline when its flops dominate (prefill), else HBM.
+    # Bytes: the rows of the union of a sequence's lists once per layer (as in the step's
+    # algorithmic bytes), plus q / o / lse; flops: every (query, selected row) pair.
     att_layers = sd0["layers"]
-    ws_att = torch.empty(max(256, 2 * lsa.attn_workspace_size(sd0["T"], w.H, w.Dv, sd0["n_split"])),
-                         dtype=torch.uint8, device=dev)
+    one = lsa.attn_workspace_size(sd0["T"], w.H, w.Dv, sd0["n_split"])
+    ws_att = [torch.empty(max(256, one), dtype=torch.uint8, device=dev) for _ in range(2)]
+    side = torch.cuda.Stream(device=dev)
+    ev_fork, ev_join = torch.cuda.Event(), torch.cuda.Event()
 
     def att_fn():
-        for L in att_layers:
+        ev_fork.record(stream)
+        side.wait_event(ev_fork)
+        for li, L in enumerate(att_layers):
             lsa.sparse_attn(sd0["batch"], L.q, L.kv, sd0["idx"], sd0["cnt"], w.sm_scale, L.o, L.lse, v=L.v,
-                            n_split=sd0["n_split"], ws=ws_att, stream=stream)
+                            n_split=sd0["n_split"], ws=ws_att[li & 1], stream=stream if li % 2 == 0 else side)
+        ev_join.record(side)
+        stream.wait_event(ev_join)
     ams = time_alone(att_fn, stream, n_alone)
-    rows = float(sd0["cnt"].sum().item())
+    p0 = w.passes[0]
+    idx_h, cnt_h = sd0["idx"].cpu().numpy(), sd0["cnt"].cpu().numpy()
+    rows = float(cnt_h.sum())
+    urows = sum(np.unique(np.concatenate([idx_h[t, :cnt_h[t]] for t in range(b * p0.q_per_seq,
+                                                                             (b + 1) * p0.q_per_seq)])).size
+                for b in range(w.B))
     rowb = w.D * (1 if w.kv_fp8 else 2) + (4 if w.kv_fp8 else 0)
-    att_bytes = len(att_layers) * (rows * rowb + sd0["T"] * (w.H * w.D * 2 + w.H * w.Dv * 2 + w.H * 4))
+    att_bytes = len(att_layers) * (urows * rowb + sd0["T"] * (w.H * w.D * 2 + w.H * w.Dv * 2 + w.H * 4))
     att_flops = 2.0 * w.H * (w.D + w.Dv) * rows * len(att_layers)
     a_roof = {"kernel": "sparse_attn (+ split merge)", "launch_ms": ams, "algorithmic_bytes_per_launch": att_bytes,
               "algorithmic_flops_per_launch": att_flops}

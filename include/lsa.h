@@ -62,6 +62,7 @@ typedef enum { LSA_BF16 = 0, LSA_FP8_E4M3 = 1, LSA_FP32 = 2 } lsa_dtype;
 /* lsa_topk flags */
 #define LSA_TOPK_RAW (1u << 0) /* output the selected COLUMN ids, no sink/window union (HI recall) */
 #define LSA_TOPK_EXCLUDES_FIXED (1u << 1) /* fixed-budget SI: top-k drawn outside sinks and window */
+#define LSA_TOPK_WINDOW_ALIGNED (1u << 2) /* SI window starts on a 64-row boundary */
 
 /* A per-sequence cache: row r of sequence b starts at
  *   data + b * seq_stride + r * tok_stride            (elements of `dtype`),
@@ -164,8 +165,12 @@ lsa_status lsa_block_score(const lsa_batch* batch, const void* q_idx, const floa
  *   candidates, so the k picks come from the other visible positions and the (disjoint) list
  *   holds min(k, those) + the sinks + the window ([release] SI bullet, read as a budget split
  *   between the contiguous part and the dynamic picks).  Not with LSA_TOPK_RAW.
+ *   LSA_TOPK_WINDOW_ALIGNED: the window starts at max(0, q_pos - window + 1) rounded down to a
+ *   multiple of 64, so it covers whole 64-row blocks up to the query (window .. window + 63
+ *   positions; [release] SI bullet: hardware-aligned contiguous reads).  Combines with
+ *   LSA_TOPK_EXCLUDES_FIXED; not with LSA_TOPK_RAW.
  *   idx [T][ld_idx] int32, entries beyond count[t] set to -1; count [T] int32.
- *   ld_idx >= k + n_sink + window. */
+ *   ld_idx >= k + n_sink + window (+ 63 with LSA_TOPK_WINDOW_ALIGNED and window > 0). */
 lsa_status lsa_topk(const lsa_batch* batch, const float* scores, int64_t ld_scores, int n_cols,
                     const int32_t* cand_blocks, int n_cand, int block_size,
                     int k, int n_sink, int window, uint32_t flags,
@@ -340,6 +345,8 @@ typedef struct {
     /* selection: 0 = top-k over all visible keys, then the union with sinks and window;
      * 1 = fixed budget (LSA_TOPK_EXCLUDES_FIXED) */
     int32_t          si_fixed_budget;
+    /* 1 = the SI window starts on a 64-row boundary (LSA_TOPK_WINDOW_ALIGNED) */
+    int32_t          si_window_aligned;
 } lsa_decode_params;
 
 /* Runs indexer (flat, or HI: block scores -> recall -> fine scores), top-k + union, then
@@ -354,6 +361,9 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
                             int32_t* dev_status, void* stream);
 
 size_t lsa_decode_workspace_size(const lsa_decode_params* p);
+/* Entries per token of the step's index list: k + n_sink + window, plus 63 with
+ * si_window_aligned and window > 0 (the minimum idx_ld). */
+int    lsa_decode_index_capacity(const lsa_decode_params* p);
 
 /* ---------------------------------------------------------------- pipelined host I/O
  * A decode driver for callers whose queries and outputs live in host memory (pinned, so that
@@ -404,6 +414,15 @@ lsa_status lsa_pipeline_destroy(lsa_pipeline* pl);
 lsa_status  lsa_read_device_status(const int32_t* dev_status, void* stream);
 const char* lsa_status_string(lsa_status s);
 int         lsa_version(void);
+
+/* Diagnostic: the wall-time limit, in nanoseconds, of the pipeline waits of the tensor-core
+ * indexer (lsa_index_score, lsa_index_score_q8, the indexer of lsa_decode_fused) and of the
+ * tensor-core block scores, for launches issued after the call; 0 restores the default (2 s).  A
+ * CTA whose wait runs out stops its pipeline, waits (with the 2 s bound) for its copies and MMAs
+ * in flight, frees its tensor memory and stores LSA_ERR_TIMEOUT in dev_status; its outputs are
+ * then incomplete.  A limit shorter than the kernel's own waits makes it give up on purpose: the
+ * way to check that path.  Process-wide; returns the previous setting. */
+uint64_t    lsa_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

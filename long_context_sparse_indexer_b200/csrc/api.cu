@@ -1,5 +1,6 @@
 // C ABI of the LSA library: host-side validation, workspace carving and kernel dispatch.
 // No device allocation, no synchronisation (except lsa_read_device_status), no exceptions.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -11,6 +12,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kMaxTokens = 65535;
+constexpr int kWindowAlign = 64;             // rows of the block the aligned SI window starts on
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 inline int elem_bytes(int dtype) { return dtype == LSA_FP8_E4M3 ? 1 : (dtype == LSA_BF16 ? 2 : 4); }
@@ -93,8 +95,11 @@ lsa_status topk_impl(const lsa_batch* batch, const float* scores, int64_t ld, in
     if (raw && (n_sink || window || cand)) return LSA_ERR_INVALID_ARG;
     if ((int64_t)k + n_sink + window > ld_idx) return LSA_ERR_INVALID_ARG;
     if (cand && (n_cand < 1 || block_size < 1 || n_cols > (int64_t)n_cand * block_size)) return LSA_ERR_INVALID_ARG;
-    if (flags & ~(LSA_TOPK_RAW | LSA_TOPK_EXCLUDES_FIXED)) return LSA_ERR_UNSUPPORTED;
-    if (raw && fixed) return LSA_ERR_INVALID_ARG;
+    const bool aligned = flags & LSA_TOPK_WINDOW_ALIGNED;
+    if (flags & ~(LSA_TOPK_RAW | LSA_TOPK_EXCLUDES_FIXED | LSA_TOPK_WINDOW_ALIGNED)) return LSA_ERR_UNSUPPORTED;
+    if (raw && (fixed || aligned)) return LSA_ERR_INVALID_ARG;
+    // The aligned window holds up to 63 positions more than `window`.
+    if (aligned && window > 0 && (int64_t)k + n_sink + window + kWindowAlign - 1 > ld_idx) return LSA_ERR_INVALID_ARG;
     if (batch->T == 0) return LSA_OK;
     if (!scores || !idx || !count) return LSA_ERR_INVALID_ARG;
     TopkArgs a{};
@@ -103,6 +108,7 @@ lsa_status topk_impl(const lsa_batch* batch, const float* scores, int64_t ld, in
     a.scores = scores; a.ld = ld; a.n_cols = n_cols;
     a.cand = cand; a.n_cand = n_cand; a.block_size = block_size;
     a.k = k; a.n_sink = n_sink; a.window = window; a.raw = raw; a.fixed_budget = fixed;
+    a.window_align = aligned ? kWindowAlign : 0;
     a.idx = idx; a.ld_idx = ld_idx; a.count = count; a.status = st;
     return cuda_status(launch_topk(a, stream));
 }
@@ -112,7 +118,16 @@ size_t attn_ws(int T, int H, int Dv, int n_split) {
     return align_up((size_t)T * n_split * H * Dv * 4) + align_up((size_t)T * n_split * H * 4);
 }
 
+// Limit of the pipeline waits of the tensor-core indexer and block-score kernels (0: the 2 s
+// default), set by lsa_set_wait_limit_ns.
+std::atomic<uint64_t> g_wait_limit_ns{0};
+
 }  // namespace
+
+uint64_t lsa::wait_limit_ns() {
+    const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+    return v ? v : 2000000000ull;
+}
 
 // Argument checks of lsa_sparse_attn that do not involve the workspace (shared with the
 // no-allocation entry point, which checks its own scratch size after these).
@@ -191,7 +206,7 @@ struct FusedPlan {
 
 bool plan_fused(const lsa_decode_params* p, FusedPlan& f) {
     const int T = p->batch.T;
-    f.cap = p->k + p->n_sink + p->window;
+    f.cap = p->k + p->n_sink + p->window + (p->si_window_aligned && p->window > 0 ? kWindowAlign - 1 : 0);
     size_t off = 0;
     if (p->hi) {
         f.nblk = (p->batch.L_alloc + p->block_size - 1) / p->block_size;
@@ -323,6 +338,11 @@ size_t lsa_attn_workspace_size(int T, int H, int Dv, int n_split) {
     return attn_ws(T, H, Dv, n_split);
 }
 
+int lsa_decode_index_capacity(const lsa_decode_params* p) {
+    if (!p) return 0;
+    return p->k + p->n_sink + p->window + (p->si_window_aligned && p->window > 0 ? kWindowAlign - 1 : 0);
+}
+
 size_t lsa_decode_workspace_size(const lsa_decode_params* p) {
     if (!p) return 0;
     FusedPlan f;
@@ -339,7 +359,7 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
     if (p->n_layers < 0 || (p->n_layers > 0 && !p->layers)) return LSA_ERR_INVALID_ARG;
     if (p->k < 0 || p->n_sink < 0 || p->window < 0) return LSA_ERR_INVALID_ARG;
     if (p->hi && (p->block_size < 1 || p->block_size > 1024 || p->n_recall < 1 || !p->kbar)) return LSA_ERR_INVALID_ARG;
-    if (p->idx_out && p->idx_ld < (int64_t)p->k + p->n_sink + p->window) return LSA_ERR_INVALID_ARG;
+    if (p->idx_out && p->idx_ld < (int64_t)lsa_decode_index_capacity(p)) return LSA_ERR_INVALID_ARG;
     if ((p->idx_out == nullptr) != (p->count_out == nullptr)) return LSA_ERR_INVALID_ARG;
     FusedPlan f;
     plan_fused(p, f);
@@ -351,7 +371,8 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
     int32_t* idx = p->idx_out ? p->idx_out : reinterpret_cast<int32_t*>(w + f.idx);
     int32_t* count = p->count_out ? p->count_out : reinterpret_cast<int32_t*>(w + f.count);
     const int64_t ld_idx = p->idx_out ? p->idx_ld : f.cap;
-    const uint32_t topk_flags = p->si_fixed_budget ? LSA_TOPK_EXCLUDES_FIXED : 0u;
+    const uint32_t topk_flags = (p->si_fixed_budget ? LSA_TOPK_EXCLUDES_FIXED : 0u) |
+                                (p->si_window_aligned ? LSA_TOPK_WINDOW_ALIGNED : 0u);
 
     if (!p->hi) {
         s = index_score_impl(batch, p->q_idx, p->w, p->H_I, &p->k_idx, nullptr, 0, 0, scores, f.ld, f.n_cols,
@@ -514,5 +535,7 @@ const char* lsa_status_string(lsa_status s) {
 }
 
 int lsa_version(void) { return 1; }
+
+uint64_t lsa_set_wait_limit_ns(uint64_t ns) { return g_wait_limit_ns.exchange(ns); }
 
 }  // extern "C"

@@ -242,7 +242,7 @@ block_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 
     if (warp == 0) {
         if (tc::elect_one()) {
-            if (tc::mbar_wait(&sm.full, 0, abort_flag)) {
+            if (tc::mbar_wait(&sm.full, 0, abort_flag, a.wait_ns)) {
                 tc::tc_fence_after();
                 const uint32_t idesc = tc::idesc_f16(128, N, 1);      // bf16 x bf16 -> f32, K-major
 #pragma unroll
@@ -261,7 +261,7 @@ block_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         }
         __syncwarp();
     }
-    const bool ok = tc::mbar_wait(&sm.done, 0, abort_flag);
+    const bool ok = tc::mbar_wait(&sm.done, 0, abort_flag, a.wait_ns);
     if (ok) {
         tc::tc_fence_after();
         const int j = j0 + tid;
@@ -340,6 +340,7 @@ static cudaError_t launch_block_score_tc(const BlockScoreArgs& a, int H_I, cudaS
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaSuccess;
     BtArgs pa{a, G, H_I};
+    pa.a.wait_ns = wait_limit_ns();
     *used = true;
     if (a.d_I == 128) {
         switch (N) {

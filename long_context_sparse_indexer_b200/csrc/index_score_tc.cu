@@ -291,6 +291,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool hi = a.cand != nullptr;
     volatile int* abort_flag = &sm.abort;
+    const uint64_t wlim = a.wait_ns;                     // pipeline waits; the drains keep tc::kWaitNs
 
     // ---- set-up: barriers, TMEM, active tiles per group and this CTA's share
     if (threadIdx.x == 0) {
@@ -358,7 +359,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
             int s = 0, ph = 0, issued = 0;
             for (int k = k_lo; k < k_hi; ++k) {
                 if (wk.to(k)) { t0 = (pa.group0 + wk.g) * G; bseq = max(a.q_seq[t0], 0); }
-                if (!tc::mbar_wait(&sm.empty_k[s], ph ^ 1, abort_flag)) break;
+                if (!tc::mbar_wait(&sm.empty_k[s], ph ^ 1, abort_flag, wlim)) break;
                 ++issued;
                 tc::mbar_expect_tx(&sm.full_k[s], NB * kBlockBytes + (pa.scale_tma ? TK * 4 : 0));
                 const int c = (k - sm.tstart[wk.g]) * TK;
@@ -393,11 +394,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
             const uint64_t dh1 = tc::sdesc_sw128(tc::smem_u32(sm.q[1][0])), dl1 = tc::sdesc_sw128(tc::smem_u32(sm.q[1][1]));
             Walk wk(sm.tstart, NG, k_lo);
             int s = 0, kph = 0, slot = 0, dph = 0, last_slot = -1, last_ph = 0;
-            bool alive = n_mine == 0 || tc::mbar_wait(&sm.q_full[0], 0, abort_flag);
+            bool alive = n_mine == 0 || tc::mbar_wait(&sm.q_full[0], 0, abort_flag, wlim);
             for (int k = k_lo; alive && k < k_hi; ++k) {
-                if (wk.to(k) && !tc::mbar_wait(&sm.q_full[wk.epoch & 1], (wk.epoch >> 1) & 1, abort_flag)) break;
-                if (!tc::mbar_wait(&sm.full_k[s], kph, abort_flag)) break;
-                if (!tc::mbar_wait(&sm.d_empty[slot], dph ^ 1, abort_flag)) break;
+                if (wk.to(k) && !tc::mbar_wait(&sm.q_full[wk.epoch & 1], (wk.epoch >> 1) & 1, abort_flag, wlim)) break;
+                if (!tc::mbar_wait(&sm.full_k[s], kph, abort_flag, wlim)) break;
+                if (!tc::mbar_wait(&sm.d_empty[slot], dph ^ 1, abort_flag, wlim)) break;
                 tc::tc_fence_after();
                 const uint64_t dh = (wk.epoch & 1) ? dh1 : dh0, dl = (wk.epoch & 1) ? dl1 : dl0;
 #pragma unroll
@@ -430,8 +431,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
             // Group epoch e: its queries go to buffer e & 1 once both epilogue warpgroups have
             // released the group that used the buffer before (epoch e - 2).
             const int e = wk.epoch, qb = e & 1;
-            if (e >= 2 && (!tc::mbar_wait(&sm.q_free[qb][0], ((e - 2) >> 1) & 1, abort_flag) ||
-                           !tc::mbar_wait(&sm.q_free[qb][1], ((e - 2) >> 1) & 1, abort_flag)))
+            if (e >= 2 && (!tc::mbar_wait(&sm.q_free[qb][0], ((e - 2) >> 1) & 1, abort_flag, wlim) ||
+                           !tc::mbar_wait(&sm.q_free[qb][1], ((e - 2) >> 1) & 1, abort_flag, wlim)))
                 break;
             const int t0 = (pa.group0 + wk.g) * G;
             if (ct < kMaxG) set_group_validity(a, t0, G, ct, sm.pos[qb], sm.ok[qb]);
@@ -457,7 +458,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
             for (; released < e - 1; ++released) tc::mbar_arrive(&sm.q_free[(released + 1) & 1][wg]);
             if ((j & 1) == wg) {
                 if (e != waited) {
-                    if (!tc::mbar_wait(&sm.q_full[qb], (e >> 1) & 1, abort_flag)) break;
+                    if (!tc::mbar_wait(&sm.q_full[qb], (e >> 1) & 1, abort_flag, wlim)) break;
                     waited = e;
                 }
                 int col[NB], row[NB];
@@ -472,7 +473,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                         row[b] = blk >= 0 ? blk * 64 + (col[b] & 63) : -1;
                     }
                 }
-                if (!tc::mbar_wait(&sm.full_k[s], kph, abort_flag)) break;
+                if (!tc::mbar_wait(&sm.full_k[s], kph, abort_flag, wlim)) break;
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
                     ks[b] = 1.f;
@@ -483,7 +484,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                     }
                 }
                 tc::mbar_arrive(&sm.empty_k[s]);
-                if (!tc::mbar_wait(&sm.d_full[slot], dph, abort_flag)) break;
+                if (!tc::mbar_wait(&sm.d_full[slot], dph, abort_flag, wlim)) break;
                 tc::tc_fence_after();
                 const uint32_t tb = d_col + slot * SW + lane_off;
                 const auto store = [&](int gi, int b, float tot) {
@@ -588,6 +589,7 @@ cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st) {
     if (a.n_cols <= 0 || a.T <= 0) return cudaSuccess;
     PArgs pa{};
     pa.a = a;
+    pa.a.wait_ns = wait_limit_ns();
     pa.H_I = H_I;
     pa.G = group_size(a, H_I);
     const int N = pa.G * H_I;

@@ -22,6 +22,7 @@ struct IndexArgs {
     int n_cols;              // columns to write
     int group;               // tokens per CTA (<= 4)
     int q_fp8;               // 1: FP8-query mode (queries rounded once to e4m3, tensor-core path only)
+    uint64_t wait_ns;        // limit of the tensor-core kernel's pipeline waits (drains keep 2 s)
     int32_t* status;
 };
 
@@ -53,6 +54,7 @@ struct BlockScoreArgs {
     float* scores;
     int64_t ld;
     int n_cols;
+    uint64_t wait_ns;        // limit of the tensor-core kernel's pipeline waits (drains keep 2 s)
     int32_t* status;
 };
 
@@ -69,6 +71,7 @@ struct TopkArgs {
     int k, n_sink, window;
     bool raw;
     bool fixed_budget;       // top-k drawn outside the sinks and the window
+    int window_align;        // 0, or the block the SI window's start is rounded down to (64)
     int32_t* idx;
     int64_t ld_idx;
     int32_t* count;
@@ -131,6 +134,9 @@ cudaError_t launch_kvp_local_index(int T, int B, const int32_t* q_seq, const int
                                    const int32_t* shard_len, const int32_t* idx, int64_t ld_idx,
                                    const int32_t* count, int32_t* local_idx, int64_t ld_local, int32_t* local_count,
                                    int32_t* status, cudaStream_t st);
+
+// Wait limit the tensor-core indexer and block-score kernels are launched with (api.cu).
+uint64_t wait_limit_ns();
 
 // Host-side checks of lsa_sparse_attn's arguments other than its workspace (api.cu).
 lsa_status attn_validate(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,

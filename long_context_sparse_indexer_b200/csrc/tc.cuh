@@ -64,18 +64,20 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-// Waits for the phase with the given parity.  Bounded: after kWaitNs of wall time (or once
-// another thread of the CTA has given up and set *abort) it sets *abort and returns false.
+// Waits for the phase with the given parity.  Bounded: after limit_ns of wall time (kWaitNs,
+// 2 s, unless the caller passes a shorter limit) or once another thread of the CTA has given up
+// and set *abort, it sets *abort and returns false.
 constexpr uint64_t kWaitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
         // The waiting thread sleeps until the phase completes (or 20 us pass), so waiting warps
         // leave the issue slots to working ones.
-        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (mbar_try_wait_sleep(bar, parity, limit_ns < 20000u ? (uint32_t)limit_ns : 20000u)) return true;
         if (*abort) return false;
-        if (global_ns() - t0 > kWaitNs) { *abort = 1; return false; }
+        if (global_ns() - t0 > limit_ns) { *abort = 1; return false; }
     }
 }
 

@@ -25,6 +25,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_DATA, 
 BF16, FP8_E4M3, FP32 = 0, 1, 2
 TOPK_RAW = 1
 TOPK_EXCLUDES_FIXED = 2
+TOPK_WINDOW_ALIGNED = 4
+WINDOW_ALIGN = 64
 
 c_i32, c_i64, c_u32, c_f32, c_vp, c_size = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float,
                                              ctypes.c_void_p, ctypes.c_size_t)
@@ -59,7 +61,7 @@ class CDecodeParams(ctypes.Structure):
                 ("H", c_i32), ("Dqk", c_i32), ("Dv", c_i32), ("sm_scale", c_f32), ("n_split", c_i32),
                 ("n_layers", c_i32), ("layers", ctypes.POINTER(CLayer)),
                 ("idx_out", c_vp), ("idx_ld", c_i64), ("count_out", c_vp), ("idx_q_fp8", c_i32),
-                ("si_fixed_budget", c_i32)]
+                ("si_fixed_budget", c_i32), ("si_window_aligned", c_i32)]
 
 
 _P = ctypes.POINTER
@@ -80,6 +82,8 @@ _lib.lsa_attn_workspace_size.restype = c_size
 _lib.lsa_decode_fused.argtypes = [_P(CDecodeParams), c_vp, c_size, c_vp, c_vp]
 _lib.lsa_decode_workspace_size.argtypes = [_P(CDecodeParams)]
 _lib.lsa_decode_workspace_size.restype = c_size
+_lib.lsa_decode_index_capacity.argtypes = [_P(CDecodeParams)]
+_lib.lsa_decode_index_capacity.restype = c_i32
 _lib.lsa_read_device_status.argtypes = [c_vp, c_vp]
 _lib.lsa_sparse_attn_partial.argtypes = [_P(CBatch), c_vp, c_i32, c_i32, _P(CCache), _P(CCache), c_i32, c_vp, c_i64,
                                          c_vp, c_f32, c_i32, c_vp, c_vp, c_vp, c_size, c_vp, c_vp]
@@ -105,6 +109,8 @@ _lib.lsa_pipeline_destroy.argtypes = [c_vp]
 _lib.lsa_status_string.argtypes = [c_i32]
 _lib.lsa_status_string.restype = ctypes.c_char_p
 _lib.lsa_version.restype = c_i32
+_lib.lsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+_lib.lsa_set_wait_limit_ns.restype = ctypes.c_uint64
 for _f in ("lsa_index_score", "lsa_index_score_q8", "lsa_block_keys", "lsa_block_score", "lsa_topk", "lsa_sparse_attn",
            "lsa_sparse_attn_noalloc", "lsa_decode_fused", "lsa_read_device_status", "lsa_sparse_attn_partial",
            "lsa_merge_partials", "lsa_kvp_shard_batch", "lsa_kvp_candidates", "lsa_kvp_select", "lsa_kvp_local_index"):
@@ -114,7 +120,8 @@ EXPORTS = ("lsa_index_score", "lsa_index_score_q8", "lsa_block_keys", "lsa_block
            "lsa_sparse_attn_noalloc", "lsa_attn_workspace_size", "lsa_decode_fused", "lsa_decode_workspace_size", "lsa_read_device_status",
            "lsa_status_string", "lsa_version", "lsa_pipeline_create", "lsa_pipeline_step", "lsa_pipeline_join",
            "lsa_pipeline_destroy", "lsa_sparse_attn_partial", "lsa_merge_partials", "lsa_kvp_shard_batch",
-           "lsa_kvp_candidates", "lsa_kvp_select_workspace_size", "lsa_kvp_select", "lsa_kvp_local_index")
+           "lsa_kvp_candidates", "lsa_kvp_select_workspace_size", "lsa_kvp_select", "lsa_kvp_local_index",
+           "lsa_set_wait_limit_ns", "lsa_decode_index_capacity")
 
 
 def library() -> ctypes.CDLL:
@@ -217,12 +224,14 @@ def block_score(batch: Batch, q_idx: torch.Tensor, w: torch.Tensor, kbar: torch.
 
 def topk(batch: Batch, scores: torch.Tensor, n_cols: int, k: int, n_sink: int, window: int, idx: torch.Tensor,
          count: torch.Tensor, cand_blocks: Optional[torch.Tensor] = None, block_size: int = 0, raw: bool = False,
-         dev_status: Optional[torch.Tensor] = None, stream=None, fixed_budget: bool = False) -> None:
+         dev_status: Optional[torch.Tensor] = None, stream=None, fixed_budget: bool = False,
+         window_aligned: bool = False) -> None:
     cb = batch.c()
     n_cand = int(cand_blocks.shape[1]) if cand_blocks is not None else 0
     _check(_lib.lsa_topk(ctypes.byref(cb), _ptr(scores), int(scores.stride(0)), int(n_cols), _ptr(cand_blocks),
                          n_cand, int(block_size), int(k), int(n_sink), int(window),
-                         (TOPK_RAW if raw else 0) | (TOPK_EXCLUDES_FIXED if fixed_budget else 0),
+                         (TOPK_RAW if raw else 0) | (TOPK_EXCLUDES_FIXED if fixed_budget else 0)
+                         | (TOPK_WINDOW_ALIGNED if window_aligned else 0),
                          _ptr(idx), int(idx.stride(0)), _ptr(count), _ptr(dev_status), _stream(stream)), "lsa_topk")
 
 
@@ -353,7 +362,7 @@ class DecodeStep:
                  window: int, layers: Sequence[Layer], H: int, Dqk: int, Dv: int, sm_scale: float, n_split: int = 1,
                  hi: bool = False, block_size: int = 64, n_recall: int = 0, kbar: Optional[torch.Tensor] = None,
                  idx_out: Optional[torch.Tensor] = None, count_out: Optional[torch.Tensor] = None,
-                 idx_q_fp8: bool = False, si_fixed_budget: bool = False):
+                 idx_q_fp8: bool = False, si_fixed_budget: bool = False, si_window_aligned: bool = False):
         self._keep = (batch, q_idx, w, k_idx, list(layers), kbar, idx_out, count_out)
         arr = (CLayer * max(1, len(layers)))()
         for i, L in enumerate(layers):
@@ -364,10 +373,13 @@ class DecodeStep:
                                int(kbar.stride(0)) if kbar is not None else 0, int(H), int(Dqk), int(Dv),
                                float(sm_scale), int(n_split), len(layers), arr, _ptr(idx_out),
                                int(idx_out.stride(0)) if idx_out is not None else 0, _ptr(count_out),
-                               int(bool(idx_q_fp8)), int(bool(si_fixed_budget)))
+                               int(bool(idx_q_fp8)), int(bool(si_fixed_budget)), int(bool(si_window_aligned)))
 
     def workspace_size(self) -> int:
         return int(_lib.lsa_decode_workspace_size(ctypes.byref(self.p)))
+
+    def index_capacity(self) -> int:
+        return int(_lib.lsa_decode_index_capacity(ctypes.byref(self.p)))
 
     def __call__(self, ws: torch.Tensor, dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
         _check(_lib.lsa_decode_fused(ctypes.byref(self.p), _ptr(ws), ws.numel() * ws.element_size(),
@@ -439,3 +451,8 @@ def status_string(status: int) -> str:
 
 def version() -> int:
     return int(_lib.lsa_version())
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    """lsa_set_wait_limit_ns (diagnostic): returns the previous limit (0 = the 2 s default)."""
+    return int(_lib.lsa_set_wait_limit_ns(int(ns)))

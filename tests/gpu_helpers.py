@@ -51,7 +51,7 @@ def block_key_values(kbar: torch.Tensor) -> np.ndarray:
 
 
 def decode_step(wt: D.WorkloadTensors, pi: int = 0, n_split: int = 1, kbar=None, cap_extra: int = 0,
-                idx_q_fp8: bool = False):
+                idx_q_fp8: bool = False, si_window_aligned: bool = False):
     """Builds lsa.DecodeStep for a pass plus its output tensors."""
     w = wt.w
     pt = wt.passes[pi]
@@ -70,7 +70,8 @@ def decode_step(wt: D.WorkloadTensors, pi: int = 0, n_split: int = 1, kbar=None,
         kbar = block_keys(wt, pi)
     step = lsa.DecodeStep(batch_of(wt, pi), pt.q_idx, pt.w, idx_cache(wt, pi), w.k, w.n_sink, w.window, layers,
                           w.H, w.D, w.Dv, w.sm_scale, n_split=n_split, hi=w.hi, block_size=w.block_size,
-                          n_recall=w.n_recall, kbar=kbar, idx_out=idx, count_out=cnt, idx_q_fp8=idx_q_fp8)
+                          n_recall=w.n_recall, kbar=kbar, idx_out=idx, count_out=cnt, idx_q_fp8=idx_q_fp8,
+                          si_window_aligned=si_window_aligned)
     ws = torch.empty(max(256, step.workspace_size()), dtype=torch.uint8, device=dev)
     return step, ws, idx, cnt, layers
 

@@ -13,7 +13,7 @@ HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), 
 
 def declared():
     txt = open(HDR).read()
-    return sorted(set(re.findall(r"^\s*(?:lsa_status|size_t|const char\*|int)\s+(lsa_\w+)\s*\(", txt, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:lsa_status|size_t|const char\*|int|uint64_t)\s+(lsa_\w+)\s*\(", txt, re.M)))
 
 
 def test_every_declared_symbol_is_exported():

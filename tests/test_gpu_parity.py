@@ -367,6 +367,64 @@ def test_topk_fixed_budget_candidate_blocks(cuda):
         assert got[t].tolist() == want.tolist()
 
 
+@pytest.mark.parametrize("fixed", [False, True])
+@pytest.mark.parametrize("n_cols", [5000, 70000])
+def test_topk_window_aligned(cuda, n_cols, fixed):
+    """Block-aligned SI window: the window starts on the 64-row boundary at or below
+    pos - window + 1; plain union and fixed budget, against the oracle's aligned reading."""
+    rng = np.random.default_rng(n_cols + 3 * fixed)
+    T, k, n_sink, window = 5, 300, 4, 100
+    s = _host_score_rows(rng, T, n_cols, 50)
+    pos = np.array([n_cols - 1, n_cols // 2 + 5, 130, 700, 63])
+    for t in range(T):
+        s[t, pos[t] + 1:] = -np.inf
+    batch = lsa.Batch(torch.tensor([n_cols], dtype=torch.int32, device="cuda"),
+                      torch.zeros(T, dtype=torch.int32, device="cuda"),
+                      torch.from_numpy(pos.astype(np.int32)).cuda(), n_cols)
+    cap = k + n_sink + window + lsa.WINDOW_ALIGN - 1
+    idx = torch.empty((T, cap), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(T, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.topk(batch, torch.from_numpy(s).cuda(), n_cols, k, n_sink, window, idx, cnt, dev_status=st,
+             fixed_budget=fixed, window_aligned=True)
+    assert lsa.read_device_status(st) == lsa.OK
+    got = H.index_lists(idx, cnt)
+    for t in range(T):
+        cols = np.nonzero(~np.isneginf(s[t]))[0]
+        sc = s[t, cols].astype(np.float64)
+        if fixed:
+            want = olsa.union_fixed_budget(sc, cols, k, int(pos[t]), n_sink, window, align=64)
+        else:
+            want = olsa.union_fixed(olsa.topk(sc, cols, k), int(pos[t]), n_sink, window, align=64)
+        assert got[t].tolist() == want.tolist(), t
+        assert np.all(idx[t, cnt[t]:].cpu().numpy() == -1)
+    # ld_idx must leave room for the 63 extra window positions
+    small = torch.empty((T, k + n_sink + window), dtype=torch.int32, device="cuda")
+    with pytest.raises(lsa.LsaError):
+        lsa.topk(batch, torch.from_numpy(s).cuda(), n_cols, k, n_sink, window, small, cnt, window_aligned=True)
+
+
+def test_fused_step_window_aligned(cuda):
+    w = SMALL["cli_small"]
+    wt = wt_of("cli_small")
+    p = w.passes[0]
+    sc = H.flat_scores(wt).cpu().numpy().astype(np.float64)
+    step, ws, idx, cnt, layers = H.decode_step(wt, 0, n_split=2, cap_extra=lsa.WINDOW_ALIGN - 1,
+                                               si_window_aligned=True)
+    assert step.index_capacity() == w.cap + lsa.WINDOW_ALIGN - 1
+    step(ws)
+    got = H.index_lists(idx, cnt)
+    _, q_pos = W.query_rows(w, p)
+    for t in range(w.T(p)):
+        pos = int(q_pos[t])
+        picks = olsa.topk(sc[t, :pos + 1], np.arange(pos + 1), w.k)
+        assert got[t].tolist() == olsa.union_fixed(picks, pos, w.n_sink, w.window, align=64).tolist()
+    t = w.T(p) - 1
+    o_ref, _ = run.attend(w, p, p.layers[0], t, got[t])
+    mx, rl2 = H.attn_errors(H.bf16_to_np(layers[0].o[t]), o_ref)
+    assert mx < 1e-2 and rl2 < 5e-3
+
+
 def test_topk_raw_and_candidate_blocks(cuda):
     rng = np.random.default_rng(1)
     T, bs, n_cand = 3, 64, 40
