@@ -70,7 +70,9 @@ __device__ __forceinline__ uint64_t global_ns() {
 constexpr uint64_t kWaitNs = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = kWaitNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // A shortened limit starts with a check that never suspends (try_wait may block for a
+    // while by itself, longer than the limit).
+    if (limit_ns < kWaitNs ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
         // The waiting thread sleeps until the phase completes (or 20 us pass), so waiting warps

@@ -607,14 +607,16 @@ topk_kernel(TopkArgs a) {
 //
 // Rows of at most kSmallCols columns (the HI recall over block scores and the HI fine stage over
 // the recalled blocks' tokens) fit in one CTA's shared memory: the row is cached as order keys,
-// the three radix passes (12 + 12 + 8 bits) sweep the cache with CTA barriers only, and the
-// emission walks the cache in column order.  Same selection and output as topk_kernel.
+// the radix passes (digits of at most 12 bits of the key's offset from the row's smallest key)
+// sweep the cache with CTA barriers only, and the emission walks the cache in column order.  Same
+// selection and output as topk_kernel.
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallWarps = kSmallThreads / 32;
 constexpr int kSmallCols = 20480;
-// The one-CTA kernel measured slower than the cluster kernel on 16,384-column rows (17.3 vs
-// 12.6 us for the HI recall, 24.8 vs 18.6 us for the HI fine top-k): off until it wins.
-constexpr bool kSmallRowsEnabled = false;
+// With digits of the key's top 12 bits the one-CTA kernel measured slower than the cluster kernel
+// on 16,384-column rows (17.3 vs 12.6 us, HI recall): the narrow score range piled every key into
+// a few bins; the range-adaptive digits remove that.
+constexpr bool kSmallRowsEnabled = true;
 
 // Inclusive prefix sum over a CTA of kSmallThreads threads.
 __device__ __forceinline__ int small_inclusive_scan(int v, int* s_warp, int& total) {
@@ -701,7 +703,9 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(TopkArgs a) {
         return p < a_lo || p >= b_hi;
     };
 
-    // ---- cache the row as order keys; pass 1 (top 12 bits)
+    // ---- cache the row as order keys, with their minimum and maximum
+    __shared__ uint32_t s_kmin[kSmallWarps], s_kmax[kSmallWarps];
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
     for (int i = threadIdx.x; i < 4096; i += kSmallThreads) hist[i] = 0;
     {
         constexpr int kB = 4;
@@ -727,15 +731,30 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(TopkArgs a) {
                     if (cc + e >= n) break;
                     const float x = f[u][e];
                     if (x != x) report(a.status, LSA_ERR_DEVICE_DATA);
-                    s_keys[cc + e] = (x != x || x == kNegInf || fixed_pos(cc + e)) ? 0u : order_key(x);
+                    const uint32_t key = (x != x || x == kNegInf || fixed_pos(cc + e)) ? 0u : order_key(x);
+                    s_keys[cc + e] = key;
+                    if (key) { kmin = min(kmin, key); kmax = max(kmax, key); }
                 }
             }
         }
     }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) { s_kmin[warp] = kmin; s_kmax[warp] = kmax; }
     __syncthreads();
+    kmin = __reduce_min_sync(0xffffffffu, s_kmin[lane]);
+    kmax = __reduce_max_sync(0xffffffffu, s_kmax[lane]);
+
+    // ---- radix select on d = key - kmin, digits of at most 12 bits from the top of the row's
+    // range (not of the key's 32 bits): scores in a narrow range then spread over the 4096 bins of
+    // the first pass instead of piling into a few (shared-memory atomics on one bin serialise).
+    // d is order-preserving, so the selection is the same.
+    const uint32_t span = kmax >= kmin ? kmax - kmin : 0u;
+    const int bits = span ? 32 - __clz(span) : 0;
+    const int s1 = max(0, bits - 12);
     for (int c = threadIdx.x; c < n; c += kSmallThreads) {
         const uint32_t key = s_keys[c];
-        if (key) atomicAdd(&hist[key >> 20], 1);
+        if (key) atomicAdd(&hist[(key - kmin) >> s1], 1);
     }
     __syncthreads();
     const int n_valid = small_threshold(hist, 4096, a.k, s_warp, &s_bin, &s_above);
@@ -743,32 +762,28 @@ __global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(TopkArgs a) {
     uint32_t vs = 0;
     int m_keep = 0, n_eq = 0;
     if (!take_all && a.k > 0) {
-        const uint32_t b1 = (uint32_t)s_bin;
-        int above = s_above;
-        // ---- pass 2: next 12 bits among keys with prefix b1
-        for (int i = threadIdx.x; i < 4096; i += kSmallThreads) hist[i] = 0;
-        __syncthreads();
-        for (int c = threadIdx.x; c < n; c += kSmallThreads) {
-            const uint32_t key = s_keys[c];
-            if (key && (key >> 20) == b1) atomicAdd(&hist[(key >> 8) & 0xfff], 1);
+        uint32_t pre = (uint32_t)s_bin;          // (key - kmin) >> s of the threshold bin
+        int above = s_above, s = s1;
+        int cnt = hist[s_bin];                   // keys in that bin
+        while (s > 0) {                          // at most two more passes (bits <= 32)
+            const int s_next = max(0, s - 12);
+            const int nb = 1 << (s - s_next);
+            for (int i = threadIdx.x; i < nb; i += kSmallThreads) hist[i] = 0;
+            __syncthreads();
+            for (int c = threadIdx.x; c < n; c += kSmallThreads) {
+                const uint32_t key = s_keys[c];
+                if (key && ((key - kmin) >> s) == pre) atomicAdd(&hist[((key - kmin) >> s_next) & (nb - 1)], 1);
+            }
+            __syncthreads();
+            small_threshold(hist, nb, a.k - above, s_warp, &s_bin, &s_above);
+            pre = (pre << (s - s_next)) | (uint32_t)s_bin;
+            above += s_above;
+            cnt = hist[s_bin];
+            s = s_next;
         }
-        __syncthreads();
-        small_threshold(hist, 4096, a.k - above, s_warp, &s_bin, &s_above);
-        const uint32_t pre = (b1 << 12) | (uint32_t)s_bin;
-        above += s_above;
-        // ---- pass 3: last 8 bits among keys with prefix (b1, b2)
-        for (int i = threadIdx.x; i < 256; i += kSmallThreads) hist[i] = 0;
-        __syncthreads();
-        for (int c = threadIdx.x; c < n; c += kSmallThreads) {
-            const uint32_t key = s_keys[c];
-            if (key && (key >> 8) == pre) atomicAdd(&hist[key & 0xff], 1);
-        }
-        __syncthreads();
-        small_threshold(hist, 256, a.k - above, s_warp, &s_bin, &s_above);
-        above += s_above;
-        vs = (pre << 8) | (uint32_t)s_bin;
+        vs = kmin + pre;
         m_keep = a.k - above;                        // keys == vs to keep, lowest columns first
-        n_eq = hist[s_bin];                          // keys == vs in the row
+        n_eq = cnt;                                  // keys == vs in the row
     }
     const bool every = take_all || a.k <= 0;         // every candidate is selected (none when k = 0)
     const bool ties_all = every || m_keep >= n_eq;
