@@ -581,9 +581,12 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
         float m_f = m_w, l_f = l_w;
         if constexpr (kSmx == 2) {
             sm.ml[wg][h] = make_float2(m_w, l_w);
-            // One barrier over both warpgroups.  (Per-quarter barriers over the two warps of a
-            // lane quarter, 64 threads each, let a warp read the other's pair before it was written
-            // in a fraction of launches.)
+            // One barrier over both warpgroups.  bar.sync is the aligned form: a warp's arrival
+            // counts all 32 threads, so the warp must be converged when it arrives -- after the
+            // lane-divergent code of the tile loop, __syncwarp makes sure of it.  (Per-quarter
+            // barriers of 64 threads without it let a warp read the other's pair before it was
+            // written in a fraction of launches.)
+            __syncwarp();
             named_bar_sync(6, 2 * 128);
             const float2 o = sm.ml[wg ^ 1][h];
             m_f = fmaxf(m_w, o.x);

@@ -70,14 +70,15 @@ __device__ __forceinline__ uint64_t global_ns() {
 constexpr uint64_t kWaitNs = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = kWaitNs) {
-    // A shortened limit starts with a check that never suspends (try_wait may block for a
-    // while by itself, longer than the limit).
-    if (limit_ns < kWaitNs ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    // Under a shortened limit the phase is polled with checks that never suspend: try_wait may
+    // block by itself, until the phase completes, for longer than the limit.
+    const bool poll = limit_ns < kWaitNs;
+    if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
         // The waiting thread sleeps until the phase completes (or 20 us pass), so waiting warps
         // leave the issue slots to working ones.
-        if (mbar_try_wait_sleep(bar, parity, limit_ns < 20000u ? (uint32_t)limit_ns : 20000u)) return true;
+        if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (*abort) return false;
         if (global_ns() - t0 > limit_ns) { *abort = 1; return false; }
     }
