@@ -331,21 +331,50 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* part_
             }
         }
     } else {
-        for (int s = 0; s < n_split; ++s) m = fmaxf(m, __ldcg(part_lse + row0 + (size_t)s * part_stride));
-        for (int s = 0; s < n_split; ++s) {
-            const float ls = __ldcg(part_lse + row0 + (size_t)s * part_stride);
-            wsum += m == kNegInf ? 0.f : expf(ls - m);
+        // More splits than registers: the same arithmetic in the same split order, with the loads
+        // of kMergeRegs splits issued together before their arithmetic (a round trip per chunk,
+        // not per split).
+        for (int s0 = 0; s0 < n_split; s0 += kMergeRegs) {
+            float l[kMergeRegs];
+#pragma unroll
+            for (int u = 0; u < kMergeRegs; ++u)
+                l[u] = s0 + u < n_split ? __ldcg(part_lse + row0 + (size_t)(s0 + u) * part_stride) : kNegInf;
+#pragma unroll
+            for (int u = 0; u < kMergeRegs; ++u) m = fmaxf(m, l[u]);
+        }
+        for (int s0 = 0; s0 < n_split; s0 += kMergeRegs) {
+            float l[kMergeRegs];
+#pragma unroll
+            for (int u = 0; u < kMergeRegs; ++u)
+                l[u] = s0 + u < n_split ? __ldcg(part_lse + row0 + (size_t)(s0 + u) * part_stride) : 0.f;
+#pragma unroll
+            for (int u = 0; u < kMergeRegs; ++u)
+                if (s0 + u < n_split) wsum += m == kNegInf ? 0.f : expf(l[u] - m);
         }
         const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
-        for (int s = 0; s < n_split; ++s) {
-            const size_t r = row0 + (size_t)s * part_stride;
-            const float ws = (m == kNegInf ? 0.f : expf(__ldcg(part_lse + r) - m)) * rs;
-            const float4* src = reinterpret_cast<const float4*>(part_o + r * DV + d);
-            const float4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
-            acc[0] = fmaf(ws, a0.x, acc[0]); acc[1] = fmaf(ws, a0.y, acc[1]);
-            acc[2] = fmaf(ws, a0.z, acc[2]); acc[3] = fmaf(ws, a0.w, acc[3]);
-            acc[4] = fmaf(ws, a1.x, acc[4]); acc[5] = fmaf(ws, a1.y, acc[5]);
-            acc[6] = fmaf(ws, a1.z, acc[6]); acc[7] = fmaf(ws, a1.w, acc[7]);
+        for (int s0 = 0; s0 < n_split; s0 += kMergeRegs) {
+            float l[kMergeRegs];
+            float4 x0[kMergeRegs], x1[kMergeRegs];
+#pragma unroll
+            for (int u = 0; u < kMergeRegs; ++u) {
+                if (s0 + u < n_split) {
+                    const size_t r = row0 + (size_t)(s0 + u) * part_stride;
+                    l[u] = __ldcg(part_lse + r);
+                    const float4* src = reinterpret_cast<const float4*>(part_o + r * DV + d);
+                    x0[u] = __ldcg(src);
+                    x1[u] = __ldcg(src + 1);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kMergeRegs; ++u) {
+                if (s0 + u < n_split) {
+                    const float ws = (m == kNegInf ? 0.f : expf(l[u] - m)) * rs;
+                    acc[0] = fmaf(ws, x0[u].x, acc[0]); acc[1] = fmaf(ws, x0[u].y, acc[1]);
+                    acc[2] = fmaf(ws, x0[u].z, acc[2]); acc[3] = fmaf(ws, x0[u].w, acc[3]);
+                    acc[4] = fmaf(ws, x1[u].x, acc[4]); acc[5] = fmaf(ws, x1[u].y, acc[5]);
+                    acc[6] = fmaf(ws, x1[u].z, acc[6]); acc[7] = fmaf(ws, x1[u].w, acc[7]);
+                }
+            }
         }
     }
     const size_t out = ((size_t)t * H + h) * DV + d;

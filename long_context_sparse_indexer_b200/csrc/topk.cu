@@ -235,6 +235,8 @@ __device__ void local_threshold(const int* hist, int nb, int need, int* s_warp, 
 
 // Segment length (columns) a CTA caches in shared memory as order keys.
 constexpr int kTopkCacheCols = 40960;
+// Candidate block ids of a row kept in shared memory (HI: the recalled blocks).
+constexpr int kTopkCandCache = 1024;
 // Candidate lists of the compacted finish: per CTA (in its `hsum` array) and merged in CTA 0.
 constexpr int kTopkLocalCap = 2048;
 constexpr int kTopkWarpCap = kTopkLocalCap / kTopkWarps;   // per warp
@@ -249,6 +251,7 @@ topk_kernel(TopkArgs a) {
     __shared__ int s_bin, s_above, s_slot[3], s_wmax;
     __shared__ int s_wcnt[kTopkWarps], s_wk[kTopkWarps];
     __shared__ int s_sup[64], s_red[130], s_total, hist3[256];
+    __shared__ int s_cand[kTopkCandCache];        // the row's candidate block ids (HI), when they fit
     extern __shared__ uint32_t s_keys[];          // CACHED: order key of each column of the segment, 0 = invalid
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
@@ -282,9 +285,21 @@ topk_kernel(TopkArgs a) {
     // Sinks [0, a_lo) and window [b_hi, pos] (positions), and the position of column cc.
     const int a_lo = a.raw ? 0 : min(a.n_sink, pos + 1);
     const int b_hi = a.raw ? 0x7fffffff : (a.window > 0 ? max(a_lo, window_start(pos, a.window, a.window_align)) : pos + 1);
+    // Column -> position through the candidate blocks: from shared memory when they fit (the
+    // emission maps every kept column; a dependent global load there would serialise its walks),
+    // with shifts for a power-of-two block size.
+    const bool cand_cached = !a.raw && a.cand && a.n_cand <= kTopkCandCache;
+    const int bs_log = (a.block_size > 0 && (a.block_size & (a.block_size - 1)) == 0) ? __ffs(a.block_size) - 1 : -1;
+    if (cand_cached) {                                // uniform over the CTA
+        for (int i = threadIdx.x; i < a.n_cand; i += kTopkThreads) s_cand[i] = a.cand[(size_t)t * a.n_cand + i];
+        __syncthreads();
+    }
     auto position = [&](int cc) -> int {
         if (a.raw || !a.cand) return cc;
-        return a.cand[(size_t)t * a.n_cand + cc / a.block_size] * a.block_size + cc % a.block_size;
+        const int bi = bs_log >= 0 ? cc >> bs_log : cc / a.block_size;
+        const int off = bs_log >= 0 ? cc & (a.block_size - 1) : cc % a.block_size;
+        const int blk = cand_cached ? s_cand[bi] : a.cand[(size_t)t * a.n_cand + bi];
+        return blk * a.block_size + off;
     };
     // Fixed-budget selection: a column at a sink or window position is no candidate.
     auto fixed_pos = [&](int cc) -> bool {
@@ -534,8 +549,7 @@ topk_kernel(TopkArgs a) {
             gt = take_all || key > vstar;
             eq = !take_all && key == vstar;
         }
-        if (a.raw || !a.cand) p = cc;
-        else p = a.cand[(size_t)t * a.n_cand + cc / a.block_size] * a.block_size + cc % a.block_size;
+        p = position(cc);
     };
     // A: ties per warp -> CTA prefix -> cluster prefix.
     int eq_w = 0;
@@ -603,260 +617,8 @@ topk_kernel(TopkArgs a) {
     if (threadIdx.x == 0) a.count[t] = n_out;
 }
 
-// ---------------------------------------------------------------- short rows: one CTA per row
-//
-// Rows of at most kSmallCols columns (the HI recall over block scores and the HI fine stage over
-// the recalled blocks' tokens) fit in one CTA's shared memory: the row is cached as order keys,
-// the radix passes (digits of at most 12 bits of the key's offset from the row's smallest key)
-// sweep the cache with CTA barriers only, and the emission walks the cache in column order.  Same
-// selection and output as topk_kernel.
-constexpr int kSmallThreads = 1024;
-constexpr int kSmallWarps = kSmallThreads / 32;
-constexpr int kSmallCols = 20480;
-// With digits of the key's top 12 bits the one-CTA kernel measured slower than the cluster kernel
-// on 16,384-column rows (17.3 vs 12.6 us, HI recall): the narrow score range piled every key into
-// a few bins; the range-adaptive digits remove that.
-constexpr bool kSmallRowsEnabled = true;
-
-// Inclusive prefix sum over a CTA of kSmallThreads threads.
-__device__ __forceinline__ int small_inclusive_scan(int v, int* s_warp, int& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += n;
-    }
-    if (lane == 31) s_warp[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int x = s_warp[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += n;
-        }
-        s_warp[lane] = x;
-    }
-    __syncthreads();
-    total = s_warp[kSmallWarps - 1];
-    const int res = v + (warp > 0 ? s_warp[warp - 1] : 0);
-    __syncthreads();
-    return res;
-}
-
-// The bin of hist[0..nb) where the count from the top first reaches `need` (run < need <=
-// run + hist[bin]) and the count above it, as local_threshold; returns the total count.
-__device__ int small_threshold(const int* hist, int nb, int need, int* s_warp, int* s_bin, int* s_above) {
-    const int per = (nb + kSmallThreads - 1) / kSmallThreads;
-    int local = 0;
-    for (int i = 0; i < per; ++i) {
-        const int bin = nb - 1 - ((int)threadIdx.x * per + i);
-        if (bin >= 0) local += hist[bin];
-    }
-    int total;
-    const int incl = small_inclusive_scan(local, s_warp, total);
-    int run = incl - local;
-    for (int i = 0; i < per; ++i) {
-        const int bin = nb - 1 - ((int)threadIdx.x * per + i);
-        if (bin < 0) break;
-        const int h = hist[bin];
-        if (run < need && run + h >= need) { *s_bin = bin; *s_above = run; }
-        run += h;
-    }
-    __syncthreads();
-    return total;
-}
-
-__global__ void __launch_bounds__(kSmallThreads) topk_small_kernel(TopkArgs a) {
-    __shared__ int hist[4096];
-    __shared__ int s_warp[kSmallWarps], s_wcnt[kSmallWarps], s_wk[kSmallWarps];
-    __shared__ int s_bin, s_above;
-    extern __shared__ uint32_t s_keys[];          // order key of every column, 0 = no candidate
-    const int t = blockIdx.x;
-    const float* row = a.scores + (size_t)t * a.ld;
-    int32_t* out = a.idx + (size_t)t * a.ld_idx;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt = (1u << lane) - 1;
-
-    const int b = a.q_seq[t];
-    const int pos = a.q_pos[t];
-    bool ok = b >= 0 && b < a.B;
-    if (ok) {
-        const int len = a.seq_len[b];
-        ok = len >= 1 && len <= a.L_alloc && pos >= 0 && pos < len;
-    }
-    if (!ok) {
-        if (threadIdx.x == 0) { report(a.status, LSA_ERR_DEVICE_DATA); a.count[t] = 0; }
-        for (int i = threadIdx.x; i < a.ld_idx; i += kSmallThreads) out[i] = -1;
-        return;
-    }
-    const int n = a.n_cols;
-    const int a_lo = a.raw ? 0 : min(a.n_sink, pos + 1);
-    const int b_hi = a.raw ? 0x7fffffff : (a.window > 0 ? max(a_lo, window_start(pos, a.window, a.window_align)) : pos + 1);
-    auto position = [&](int cc) -> int {
-        if (a.raw || !a.cand) return cc;
-        return a.cand[(size_t)t * a.n_cand + cc / a.block_size] * a.block_size + cc % a.block_size;
-    };
-    auto fixed_pos = [&](int cc) -> bool {
-        if (!a.fixed_budget) return false;
-        const int p = position(cc);
-        return p < a_lo || p >= b_hi;
-    };
-
-    // ---- cache the row as order keys, with their minimum and maximum
-    __shared__ uint32_t s_kmin[kSmallWarps], s_kmax[kSmallWarps];
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int i = threadIdx.x; i < 4096; i += kSmallThreads) hist[i] = 0;
-    {
-        constexpr int kB = 4;
-        const bool vec = (((uintptr_t)row) & 15) == 0;
-        for (int base = threadIdx.x * 4; base < n; base += kSmallThreads * 4 * kB) {
-            float f[kB][4];
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-                const int cc = base + u * kSmallThreads * 4;
-                if (vec && cc + 3 < n) {
-                    const float4 v4 = *reinterpret_cast<const float4*>(row + cc);
-                    f[u][0] = v4.x; f[u][1] = v4.y; f[u][2] = v4.z; f[u][3] = v4.w;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) f[u][e] = cc + e < n ? row[cc + e] : kNegInf;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-                const int cc = base + u * kSmallThreads * 4;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if (cc + e >= n) break;
-                    const float x = f[u][e];
-                    if (x != x) report(a.status, LSA_ERR_DEVICE_DATA);
-                    const uint32_t key = (x != x || x == kNegInf || fixed_pos(cc + e)) ? 0u : order_key(x);
-                    s_keys[cc + e] = key;
-                    if (key) { kmin = min(kmin, key); kmax = max(kmax, key); }
-                }
-            }
-        }
-    }
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    if (lane == 0) { s_kmin[warp] = kmin; s_kmax[warp] = kmax; }
-    __syncthreads();
-    kmin = __reduce_min_sync(0xffffffffu, s_kmin[lane]);
-    kmax = __reduce_max_sync(0xffffffffu, s_kmax[lane]);
-
-    // ---- radix select on d = key - kmin, digits of at most 12 bits from the top of the row's
-    // range (not of the key's 32 bits): scores in a narrow range then spread over the 4096 bins of
-    // the first pass instead of piling into a few (shared-memory atomics on one bin serialise).
-    // d is order-preserving, so the selection is the same.
-    const uint32_t span = kmax >= kmin ? kmax - kmin : 0u;
-    const int bits = span ? 32 - __clz(span) : 0;
-    const int s1 = max(0, bits - 12);
-    for (int c = threadIdx.x; c < n; c += kSmallThreads) {
-        const uint32_t key = s_keys[c];
-        if (key) atomicAdd(&hist[(key - kmin) >> s1], 1);
-    }
-    __syncthreads();
-    const int n_valid = small_threshold(hist, 4096, a.k, s_warp, &s_bin, &s_above);
-    const bool take_all = n_valid <= a.k;
-    uint32_t vs = 0;
-    int m_keep = 0, n_eq = 0;
-    if (!take_all && a.k > 0) {
-        uint32_t pre = (uint32_t)s_bin;          // (key - kmin) >> s of the threshold bin
-        int above = s_above, s = s1;
-        int cnt = hist[s_bin];                   // keys in that bin
-        while (s > 0) {                          // at most two more passes (bits <= 32)
-            const int s_next = max(0, s - 12);
-            const int nb = 1 << (s - s_next);
-            for (int i = threadIdx.x; i < nb; i += kSmallThreads) hist[i] = 0;
-            __syncthreads();
-            for (int c = threadIdx.x; c < n; c += kSmallThreads) {
-                const uint32_t key = s_keys[c];
-                if (key && ((key - kmin) >> s) == pre) atomicAdd(&hist[((key - kmin) >> s_next) & (nb - 1)], 1);
-            }
-            __syncthreads();
-            small_threshold(hist, nb, a.k - above, s_warp, &s_bin, &s_above);
-            pre = (pre << (s - s_next)) | (uint32_t)s_bin;
-            above += s_above;
-            cnt = hist[s_bin];
-            s = s_next;
-        }
-        vs = kmin + pre;
-        m_keep = a.k - above;                        // keys == vs to keep, lowest columns first
-        n_eq = cnt;                                  // keys == vs in the row
-    }
-    const bool every = take_all || a.k <= 0;         // every candidate is selected (none when k = 0)
-    const bool ties_all = every || m_keep >= n_eq;
-
-    // ---- emission in column order: warp w owns a contiguous range of columns, walked 32 at a time
-    const int cw = ((n + kSmallWarps - 1) / kSmallWarps + 31) / 32 * 32;
-    const int e0 = min(n, warp * cw), e1 = min(n, e0 + cw);
-    int eq_base = 0;
-    if (!ties_all) {                                 // ties at vs are cut: ranks among them needed
-        int c = 0;
-        for (int i = e0; i < e1; i += 32)
-            c += __popc(__ballot_sync(0xffffffffu, i + lane < e1 && s_keys[i + lane] == vs));
-        if (lane == 0) s_wcnt[warp] = c;
-        __syncthreads();
-        for (int w = 0; w < warp; ++w) eq_base += s_wcnt[w];
-    }
-    auto walk = [&](bool write, int o) -> int {
-        int eq_run = eq_base, cnt = 0;
-        for (int i = e0; i < e1; i += 32) {
-            const int ii = i + lane;
-            const bool in = ii < e1;
-            const uint32_t key = in ? s_keys[ii] : 0u;
-            bool keep;
-            if (every) {
-                keep = in && key != 0u && a.k > 0;
-            } else {
-                const bool eq = in && key == vs;
-                const uint32_t em = ties_all ? 0u : __ballot_sync(0xffffffffu, eq);
-                keep = in && key != 0u && (key > vs || (eq && (ties_all || eq_run + __popc(em & lt) < m_keep)));
-                eq_run += __popc(em);
-            }
-            int pv = 0;
-            if (keep) {
-                pv = a.raw ? ii : position(ii);
-                if (!a.raw) keep = pv >= a_lo && pv < b_hi;
-            }
-            const uint32_t km = __ballot_sync(0xffffffffu, keep);
-            if (write && keep) out[o + cnt + __popc(km & lt)] = pv;
-            cnt += __popc(km);
-        }
-        return cnt;
-    };
-    const int kept_w = walk(false, 0);
-    if (lane == 0) s_wk[warp] = kept_w;
-    __syncthreads();
-    int keep_base = 0, written = 0;
-    for (int w = 0; w < kSmallWarps; ++w) {
-        const int v = s_wk[w];
-        if (w < warp) keep_base += v;
-        written += v;
-    }
-    walk(true, a_lo + keep_base);
-    int n_out = a_lo + written;
-    if (!a.raw) {
-        for (int i = threadIdx.x; i < a_lo; i += kSmallThreads) out[i] = i;
-        const int tail = pos + 1 - b_hi;
-        for (int i = threadIdx.x; i < tail; i += kSmallThreads) out[n_out + i] = b_hi + i;
-        n_out += max(tail, 0);
-    }
-    for (int i = n_out + threadIdx.x; i < a.ld_idx; i += kSmallThreads) out[i] = -1;
-    if (threadIdx.x == 0) a.count[t] = n_out;
-}
-
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
     if (a.T <= 0) return cudaSuccess;
-    if (a.n_cols <= kSmallCols && kSmallRowsEnabled) {
-        const size_t smem = (size_t)std::max(a.n_cols, 4) * 4;
-        cudaError_t e = cudaFuncSetAttribute(topk_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmallCols * 4);
-        if (e != cudaSuccess) return e;
-        topk_small_kernel<<<a.T, kSmallThreads, smem, st>>>(a);
-        return cudaGetLastError();
-    }
     const int per_cta = ((a.n_cols + kTopkCluster - 1) / kTopkCluster + 31) / 32 * 32;
     const size_t cand_smem = (size_t)kTopkCap * 8;             // merged candidates (keys, columns) in CTA 0
     if (per_cta <= kTopkCacheCols) {
