@@ -312,14 +312,16 @@ def measure(name, args, rank, world, local_rank, headline):
     with ClockSampler(local_rank) as clk:
         torch.cuda.synchronize()
         time.sleep(0.05)                     # let the sampler start
-        # sustained untimed load of about args.load_ms, then the timed region
-        t_one = time_region(fn, 3, stream)
-        for _ in range(max(1, int(args.load_ms / max(t_one, 1e-3)))):
-            fn()
+        # The K timed steps, then a sustained window of about args.load_ms timed on its own: its
+        # rate is the steady state under the power cap, and the clock samples cover both.
         ms = time_region(fn, args.steps, stream)
+        n_sus = max(args.steps, int(args.load_ms / max(ms, 1e-3)))
+        ms_sus = time_region(fn, n_sus, stream) if args.load_ms > 0 else None
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(ms, world, dev)
+    if ms_sus is not None:
+        ms_sus = max_over_ranks(ms_sus, world, dev)
 
     q_per_step = w.queries_per_step()
     value = q_per_step * world / (ms / 1e3)
@@ -331,6 +333,9 @@ def measure(name, args, rank, world, local_rank, headline):
            "step_hbm_frac": total_bytes / (ms / 1e3) / 1e9 / hbm,
            "n_split": [sd["n_split"] for sd in sds], "launch": "cuda_graph" if graph is not None else "eager",
            "clocks": clk.summary()}
+    if ms_sus is not None:
+        res["sustained"] = {"steps": n_sus, "ms_per_step": ms_sus, "value": q_per_step * world / (ms_sus / 1e3),
+                            "step_hbm_frac": total_bytes / (ms_sus / 1e3) / 1e9 / hbm}
 
     # Dominant kernels timed alone on the same inputs, against their rooflines.
     sd0, pt0 = sds[0], wt.passes[0]
@@ -571,7 +576,8 @@ def main():
                     help="measure only --workload (by default a single-GPU run of the 128K decode also measures the "
                          "1M-context HI decode and the 32K prefill chunk)")
     ap.add_argument("--load-ms", type=float, default=250.0,
-                    help="untimed sustained load before each timed region (clock samples at steady state)")
+                    help="sustained window after each timed region, timed on its own (steady state under the "
+                         "power cap; the clock samples cover it); 0 = none")
     ap.add_argument("--slots", type=int, default=2, help="device buffer slots of the host-buffer pipeline")
     ap.add_argument("--idx-q8", action="store_true", help="indexer in FP8-query mode (lsa_index_score_q8)")
     ap.add_argument("--n-split", default="", help="override the split-KV chunk count: one value, or one per pass")
@@ -604,6 +610,8 @@ def main():
         "roofline": head["roofline"], "attention_roofline": head["attention_roofline"],
         "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
     }
+    if "sustained" in head:
+        res["sustained"] = head["sustained"]
     if world == 1 and not args.no_extras and args.workload == "decode_cli_128k" and not args.batch:
         # The metric names two context lengths (128K and 1M); the prefill chunk carries the tensor
         # roofline.  Each is measured the same way (graph, warm-up, sustained load, K timed steps).
