@@ -479,19 +479,24 @@ def e2e_rate(w, wt, sds, args, world, dev, stream, q_per_step):
 
 
 def indexer_traffic(kern: str, idx_bytes: float):
-    """DRAM bytes per launch of the flat tensor-core indexer, from the committed ncu figures.
+    """DRAM bytes per launch of the dominant kernel, from the committed ncu figures.
 
-    profiles/indexer_traffic.json records the ratio of measured DRAM traffic to algorithmic
-    bytes on a small case of the same kernel and the SHA-256 of the kernel source it was taken
-    on; the ratio is applied only while the source still has that hash (otherwise the counters
-    describe another kernel and the field is null)."""
+    profiles/indexer_traffic.json (flat tensor-core indexer) and profiles/block_score_traffic.json
+    (HI block scores) record the ratio of measured DRAM traffic to algorithmic bytes of a capture
+    of that kernel and the SHA-256 of the kernel source it was taken on; the ratio is applied only
+    while the source still has that hash (otherwise the counters describe another kernel and the
+    field is null)."""
     import hashlib
-    if not kern.startswith("index_score"):
+    if kern.startswith("index_score"):
+        rec, src_file = "indexer_traffic.json", "index_score_tc.cu"
+    elif kern.startswith("block_score"):
+        rec, src_file = "block_score_traffic.json", "hi_blocks.cu"
+    else:
         return None
     try:
-        with open(os.path.join(ROOT, "profiles", "indexer_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", rec)) as f:
             d = json.load(f)
-        src = open(os.path.join(ROOT, "long_context_sparse_indexer_b200", "csrc", "index_score_tc.cu"), "rb").read()
+        src = open(os.path.join(ROOT, "long_context_sparse_indexer_b200", "csrc", src_file), "rb").read()
     except (OSError, ValueError):
         return None
     if hashlib.sha256(src).hexdigest() != d.get("source_sha256"):
@@ -562,6 +567,76 @@ def run_reference(args, rank, world):
             "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_stages(args, local_rank):
+    """Each kernel of the workload's first pass timed alone: a CUDA graph of 20 back-to-back
+    launches, replayed 5 times after one replay of warm-up (CUDA events on the launching stream).
+    Prints one JSON line {"stages_us": {...}} -- a breakdown of the step, not the bench line."""
+    from lsa_synth import device as D
+    from long_context_sparse_indexer_b200 import launch, lsa
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS[args.workload]
+    if args.batch:
+        w = W.scaled(args.workload, B=args.batch)
+    wt = D.build_workload(w, dev)
+    p, pt = w.passes[0], wt.passes[0]
+    T = w.T(p)
+    ns = int(args.n_split.split(",")[0]) if args.n_split else launch.split_for(T, w.H, w.cap, layers=len(p.layers))
+    sd = build_step(w, wt, 0, ns, q8=args.idx_q8)
+    batch, kc = sd["batch"], lsa.Cache(pt.k_idx, pt.k_scale)
+    idx, cnt = sd["idx"], sd["cnt"]
+    stages = {}
+    if w.hi:
+        kbar = sd["kbar"]
+        nblk = kbar.shape[1]
+        bsc = torch.empty((T, (nblk + 3) // 4 * 4), dtype=torch.float32, device=dev)
+        cand = torch.empty((T, w.n_recall), dtype=torch.int32, device=dev)
+        ccnt = torch.empty((T,), dtype=torch.int32, device=dev)
+        ncols = w.n_recall * w.block_size
+        fsc = torch.empty((T, ncols), dtype=torch.float32, device=dev)
+        stages["block_score"] = lambda: lsa.block_score(batch, pt.q_idx, pt.w, kbar, w.block_size, bsc, nblk)
+        stages["recall_topk"] = lambda: lsa.topk(batch, bsc, nblk, w.n_recall, 0, 0, cand, ccnt, raw=True)
+        stages["fine_index_score"] = lambda: lsa.index_score(batch, pt.q_idx, pt.w, kc, fsc, cand_blocks=cand,
+                                                             block_size=w.block_size, q_fp8=args.idx_q8)
+        stages["fine_topk"] = lambda: lsa.topk(batch, fsc, ncols, w.k, w.n_sink, w.window, idx, cnt,
+                                               cand_blocks=cand, block_size=w.block_size)
+    else:
+        ld = (wt.L_alloc + 3) // 4 * 4
+        sc = torch.empty((T, ld), dtype=torch.float32, device=dev)
+        stages["index_score"] = lambda: lsa.index_score(batch, pt.q_idx, pt.w, kc, sc, n_cols=wt.L_alloc,
+                                                        q_fp8=args.idx_q8)
+        stages["topk"] = lambda: lsa.topk(batch, sc, wt.L_alloc, w.k, w.n_sink, w.window, idx, cnt)
+    L0 = sd["layers"][0]
+    ws = torch.empty(max(256, lsa.attn_workspace_size(T, w.H, w.Dv, ns)), dtype=torch.uint8, device=dev)
+    stages[f"attention_one_layer_n_split_{ns}"] = lambda: lsa.sparse_attn(batch, L0.q, L0.kv, idx, cnt, w.sm_scale,
+                                                                          L0.o, L0.lse, v=L0.v, n_split=ns, ws=ws)
+    stages["fused_step"] = lambda: sd["step"](sd["ws"])
+    sd["step"](sd["ws"])                          # index lists for the stages that read them
+    torch.cuda.synchronize()
+    out = {}
+    for name, f in stages.items():
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s_ = torch.cuda.Stream(device=dev)
+        s_.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s_):
+            with torch.cuda.graph(g, stream=s_):
+                for _ in range(20):
+                    f()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(5):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / 100 * 1e3
+    print(json.dumps({"workload": w.name, "n_split": ns, "stages_us": out}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -581,6 +656,8 @@ def main():
     ap.add_argument("--slots", type=int, default=2, help="device buffer slots of the host-buffer pipeline")
     ap.add_argument("--idx-q8", action="store_true", help="indexer in FP8-query mode (lsa_index_score_q8)")
     ap.add_argument("--n-split", default="", help="override the split-KV chunk count: one value, or one per pass")
+    ap.add_argument("--stages", action="store_true",
+                    help="print the time of each kernel of the step alone (CUDA graphs) instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -593,6 +670,9 @@ def main():
             print(json.dumps(res), flush=True)
         return
     torch.cuda.set_device(local_rank)
+    if args.stages:
+        run_stages(args, local_rank)
+        return
     if world > 1:
         import datetime
 
