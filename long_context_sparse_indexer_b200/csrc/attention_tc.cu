@@ -20,8 +20,7 @@
 // ring of 32-row KV tiles, read as the B operand of S (K-major) and of P V (MN-major): each
 // stage has its 4 swizzled 64-dim V-half atoms (16 KB), and two stages share one 64-dim rope
 // atom, each in the half of its 128-byte rows that the other leaves (only 32 rope dims are this
-// CTA's); two 16 KB buffers that receive the peer's partial S (the peer's send warps store into
-// them directly with st.async).
+// CTA's); two 16 KB staging buffers for this CTA's partial S and two that receive the peer's.
 //
 // Warp roles (512 threads).  With BF16 rows:
 //   warps 0,2,3: gather -- tile j by the (j mod 3)-th: the rows' indices (prefetched three tiles
@@ -32,9 +31,9 @@
 //   warp 1     : MMA issuer -- S_j (16 TS + 2 SS MMAs, N = 32) once tile j has landed, P V_{j-4}
 //                has been issued and S_{j-4} has been sent; O += P_j V_j (2 TS MMAs, N = 256) once
 //                the softmax of tile j is done; whichever is ready, each kind in order.
-//   warps 4..7 : send -- warp q (mod 4) pushes heads [32q, 32q + 32) of each partial S to the
-//                peer as soon as the MMA has produced it: each lane stores its head's 128 bytes
-//                into the peer's receive buffer with st.async, completing on the peer's barrier.
+//   warps 4..7 : send -- warp q (mod 4) stages heads [32q, 32q + 32) of each partial S in shared
+//                memory and pushes the 4 KB to the peer with one bulk shared-to-shared copy that
+//                completes on the peer's barrier, as soon as the MMA has produced it.
 //   warps 8..15: softmax -- two warpgroups taking alternate tiles; thread = head (TMEM lane).
 //                Each adds the peer's partial of its tile to its own, then runs the online
 //                softmax with lazy rescaling: the reference max is raised only when a tile's
@@ -61,7 +60,7 @@ namespace {
 constexpr int kAThreads = 512;
 constexpr int kRows = 32;                    // KV rows per tile
 constexpr int kStagesA = 8;                  // KV tile ring
-constexpr int kXB = 2;                       // partial-S exchange (receive) buffers
+constexpr int kXB = 2;                       // partial-S exchange buffers (staging and receive)
 constexpr int kSP = 4;                       // S / P buffers in TMEM (P overwrites its own S)
 constexpr int kD = 576, kDv = 512, kHalf = 256;
 constexpr int kKSteps = 4 * 4 + 2;           // 16-dim K steps of S per CTA (288 dims)
@@ -75,8 +74,9 @@ struct AttnSmem {
     alignas(1024) uint8_t kv[kStagesA][kVBytes];       // V-half atoms of each stage
     alignas(1024) uint8_t rope[kStagesA / 2][kRopeBytes];  // stage s: atom s / 2, chunk half (CTA half) ^ (s & 1)
     // Partial S exchange, per buffer [head][16-byte chunk ^ (head & 7)]; softmax warp q owns the
-    // 4 KB of heads [32q, 32q + 32) in each.  The peer's send warps store into it directly.
+    // 4 KB of heads [32q, 32q + 32) in each.
     alignas(1024) uint8_t xs[kXB][kXBytes];      // the peer's partial S
+    alignas(1024) uint8_t stg[kXB][kXBytes];     // this CTA's partial S, the source of the copy to the peer
     // The query's 32 rope dims of this CTA, K-major without swizzle: head h, 8-dim chunk c at
     // (h / 8) * 512 + c * 128 + (h % 8) * 16 -- the A operand of the two rope K steps of S.
     alignas(1024) uint8_t q_rope[128 * 64];
@@ -142,9 +142,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
     const float* kvs = KV_FP8 ? a.kv_scale + (size_t)max(b, 0) * a.kv_scale_seq : nullptr;
     const uint16_t* qt = a.q + (size_t)t * 128 * kD;
 
-    // The query's five 16 KB staging atoms: the two receive buffers and KV stages 5..7 (the gather
-    // warps fill those stages only once the query has moved to TMEM).
-    auto q_atom = [&](int at) -> uint8_t* { return at < 2 ? sm.xs[at] : sm.kv[3 + at]; };
+    auto q_atom = [&](int at) -> uint8_t* { return at < 2 ? sm.xs[at] : (at < 4 ? sm.stg[at - 2] : sm.kv[7]); };
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStagesA; ++i) {
             tc::mbar_init(&sm.kv_full[i], kAsync ? 33 : 32);   // async: 32 copy completions + 1 (scales)
@@ -167,9 +165,9 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
         tc::mbar_init(&sm.q_tma, 1);
         sm.abort = 0;
         tc::fence_barrier_init();
-        // Q[:, V half] as 4 swizzled 64-dim atoms into the two receive buffers and KV stages 5 and 6,
-        // its rope atom into KV stage 7, all idle until the softmax warps have moved Q to TMEM (the
-        // rope part to shared memory).
+        // Q[:, V half] as 4 swizzled 64-dim atoms into the exchange buffers and its rope atom into
+        // KV stage 7, all idle until the softmax warps have moved Q to TMEM (the rope part to
+        // shared memory).
         tc::prefetch_tmap(&qmap);
         tc::mbar_expect_tx(&sm.q_tma, 5 * 128 * 128);
         for (int at = 0; at < 5; ++at)
@@ -255,8 +253,8 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             nxt2 = nxt3;
             nxt3 = fetch_row(j + 3 * step);
             if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.kv_empty[g], ((j / kStagesA) + 1) & 1, abort_flag))) break;
-            // Stages 5..7 hold query atoms until the softmax warps have read them.
-            if (j >= 5 && j <= 7 && !__all_sync(0xffffffffu, tc::mbar_wait(&sm.q_ready, 0, abort_flag))) break;
+            // Stage 7 holds the query's rope atom until the softmax warps have read it.
+            if (j == 7 && !__all_sync(0xffffffffu, tc::mbar_wait(&sm.q_ready, 0, abort_flag))) break;
             const int nr = min(kRows, r_end - (r_beg + j * kRows));
             {
                 const bool v = cur >= 0 && cur < len;
@@ -464,7 +462,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                     x[4 * c + 3] = __uint_as_float(sv[4 * c + 3]) + __uint_as_float(pv.w);
                 }
             }
-            if (lane == 0 && j + kXB < n_tiles)      // buffer xb is ready for tile j + kXB
+            if (lane == 0 && j + kXB < n_tiles)      // buffer xb is ready for tile j + 2
                 tc::mbar_expect_tx(&sm.rx_full[xb][quarter], 4096);
             const float4* ks4 = reinterpret_cast<const float4*>(sm.kscale[st]);
             const float4* km4 = reinterpret_cast<const float4*>(sm.kmask[st]);
@@ -650,12 +648,11 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
         }
     } else if (send_warp) {
         // ---------------- send warps: warp q (mod 4) pushes heads [32q, 32q + 32) of every partial S
-        // to the peer as soon as the MMA has produced it, off the softmax's path: each lane stores
-        // its head's 128 bytes straight into the peer's receive buffer (st.async), completing as
-        // transaction bytes on the peer's rx_full.
+        // to the peer -- staged in shared memory, then one 4 KB bulk copy that completes on the
+        // peer's rx_full -- as soon as the MMA has produced it, off the softmax's path.
         const int quarter = warp & 3;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t xs_peer = tc::peer_smem(sm.xs[0], peer) + quarter * 4096 + lane * 128;
+        const uint32_t xs_peer = tc::peer_smem(sm.xs[0], peer) + quarter * 4096;
         for (int jj = 0; jj < n_tiles; ++jj) {
             const int b = jj % kSP, x = jj % kXB;
             if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.s_full[b], (jj / kSP) & 1, abort_flag))) break;
@@ -666,17 +663,22 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.s_sent[b]);          // buffer b may be overwritten
-            // The peer's buffer x is free once the peer has read tile jj - kXB out of it.
+            // Staging buffer x and the peer's buffer x are free once the peer has read tile jj - 2
+            // (which it received, so the copy out of staging buffer x is complete too).
             bool ok = true;
             if (jj >= kXB && lane == 0)
                 ok = tc::mbar_wait_cluster(&sm.tx_free[x][quarter], ((jj / kXB) - 1) & 1, abort_flag);
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-            const uint32_t dst = xs_peer + x * kXBytes;
-            const uint32_t bar = tc::peer_smem(&sm.rx_full[x][quarter], peer);
+            uint8_t* row = sm.stg[x] + quarter * 4096 + lane * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-                tc::st_async_v4(dst + ((c ^ (lane & 7)) << 4), make_uint4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]),
-                                bar);
+                *reinterpret_cast<uint4*>(row + ((c ^ (lane & 7)) << 4)) =
+                    make_uint4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                tc::bulk_copy_to_peer(xs_peer + x * kXBytes, sm.stg[x] + quarter * 4096, 4096,
+                                      tc::peer_smem(&sm.rx_full[x][quarter], peer));
         }
     }
 

@@ -287,14 +287,6 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar) {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar) : "memory");
 }
 
-// Asynchronous 16-byte store to shared::cluster address dst (a peer CTA's shared memory) whose
-// completion counts 16 transaction bytes on the mbarrier at shared::cluster address bar (in the
-// same CTA as dst).
-__device__ __forceinline__ void st_async_v4(uint32_t dst, uint4 v, uint32_t bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
-                 :: "r"(dst), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar) : "memory");
-}
-
 // 16-byte store to shared::cluster address dst (a peer CTA's shared memory).
 __device__ __forceinline__ void st_cluster_v4(uint32_t dst, uint4 v) {
     asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(dst), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
