@@ -347,10 +347,17 @@ typedef struct {
     int32_t          si_fixed_budget;
     /* 1 = the SI window starts on a 64-row boundary (LSA_TOPK_WINDOW_ALIGNED) */
     int32_t          si_window_aligned;
+    /* Optional cudaEvent_t (NULL: none) recorded by the caller once every layer's attention query
+     * `q` is written -- typically on another stream, at the end of the MLA prolog (norm,
+     * projections, RoPE).  The indexer and the top-k do not wait for it; the attention layers do.
+     * So the index selection runs while the prolog still computes the attention queries
+     * ([release] "推理 · 模型层面优化", Attention paragraph: the indexer computed in parallel with
+     * the MLA prolog).  The indexer's own inputs (q_idx, w) must be ready on `stream`. */
+    void*            attn_q_ready;
 } lsa_decode_params;
 
 /* Runs indexer (flat, or HI: block scores -> recall -> fine scores), top-k + union, then
- * attention for every layer, with no host synchronisation.  Everything is ordered after the
+ * attention for every layer (after attn_q_ready, when given), with no host synchronisation.  Everything is ordered after the
  * work already queued on `stream`, and work queued on `stream` afterwards runs after all of
  * it.  With two or more layers the layers alternate between `stream` and a second stream of
  * the calling thread (created on first use, with two events; forked from `stream` after

@@ -131,12 +131,6 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
     int len = 0;
     bool ok = b >= 0 && b < a.B;
     if (ok) { len = a.seq_len[b]; ok = len >= 1 && len <= a.L_alloc; }
-    int n = ok ? a.count[t] : 0;
-    if (n < 0 || n > a.ld_idx) { ok = false; n = 0; }
-    if (!ok && threadIdx.x == 0 && split == 0 && half == 0) report(a.status, LSA_ERR_DEVICE_DATA);
-    const int per = (n + a.n_split - 1) / a.n_split;
-    const int r_beg = min(n, split * per), r_end = min(n, r_beg + per);
-    const int n_tiles = (r_end - r_beg + kRows - 1) / kRows;
     const int32_t* irow = a.idx + (size_t)t * a.ld_idx;
     const uint8_t* kvb = a.kv + (size_t)max(b, 0) * a.kv_seq_b;
     const float* kvs = KV_FP8 ? a.kv_scale + (size_t)max(b, 0) * a.kv_scale_seq : nullptr;
@@ -177,6 +171,16 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    // The set-up above (barriers, TMEM, the query's load) needs nothing from the previous kernel;
+    // the index list does.
+    allow_dependents_early();
+    grid_dependency_wait();
+    int n = ok ? a.count[t] : 0;
+    if (n < 0 || n > a.ld_idx) { ok = false; n = 0; }
+    if (!ok && threadIdx.x == 0 && split == 0 && half == 0) report(a.status, LSA_ERR_DEVICE_DATA);
+    const int per = (n + a.n_split - 1) / a.n_split;
+    const int r_beg = min(n, split * per), r_end = min(n, r_beg + per);
+    const int n_tiles = (r_end - r_beg + kRows - 1) / kRows;
     const uint32_t tmem = sm.tmem_base;
     const uint32_t o_col = tmem, s_col = tmem + 256, qt_col = tmem + 256 + kSP * 32;   // O, S / P, Q slice
 
@@ -700,9 +704,7 @@ cudaError_t launch_t(const CUtensorMap& qm, const CUtensorMap& m, const AttnArgs
     auto kern = sparse_attn_tc_kernel<KV_FP8, TMA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.n_split, 2, a.T);
-    kern<<<grid, kAThreads, smem, st>>>(qm, m, a);
-    return cudaGetLastError();
+    return launch_maybe_pdl(a.pdl != 0, kern, dim3(a.n_split, 2, a.T), dim3(kAThreads), smem, st, qm, m, a);
 }
 
 // The BF16 cache as one 2-D tensor of rows (row of sequence b, token i = b * (kv_seq_b / kv_tok_b)

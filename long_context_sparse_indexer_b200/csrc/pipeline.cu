@@ -76,6 +76,9 @@ lsa_status decode_slot(lsa_pipeline* pl, int slot, const lsa_decode_params* cons
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (!ok(cudaStreamIsCapturing(pl->st, &cs)) || cs != cudaStreamCaptureStatusNone)
         return decode_eager(params, n, ws, ws_bytes, dev_status, pl->st);
+    // A wait on the caller's prolog event cannot be captured (the event lives outside the graph).
+    for (int i = 0; i < n; ++i)
+        if (params[i] && params[i]->attn_q_ready) return decode_eager(params, n, ws, ws_bytes, dev_status, pl->st);
     std::vector<unsigned char> sig = signature(params, n, ws, ws_bytes, dev_status);
     if (!pl->exec[slot] || sig != pl->sig[slot]) {
         if (pl->exec[slot]) {

@@ -61,7 +61,7 @@ class CDecodeParams(ctypes.Structure):
                 ("H", c_i32), ("Dqk", c_i32), ("Dv", c_i32), ("sm_scale", c_f32), ("n_split", c_i32),
                 ("n_layers", c_i32), ("layers", ctypes.POINTER(CLayer)),
                 ("idx_out", c_vp), ("idx_ld", c_i64), ("count_out", c_vp), ("idx_q_fp8", c_i32),
-                ("si_fixed_budget", c_i32), ("si_window_aligned", c_i32)]
+                ("si_fixed_budget", c_i32), ("si_window_aligned", c_i32), ("attn_q_ready", c_vp)]
 
 
 _P = ctypes.POINTER
@@ -362,8 +362,11 @@ class DecodeStep:
                  window: int, layers: Sequence[Layer], H: int, Dqk: int, Dv: int, sm_scale: float, n_split: int = 1,
                  hi: bool = False, block_size: int = 64, n_recall: int = 0, kbar: Optional[torch.Tensor] = None,
                  idx_out: Optional[torch.Tensor] = None, count_out: Optional[torch.Tensor] = None,
-                 idx_q_fp8: bool = False, si_fixed_budget: bool = False, si_window_aligned: bool = False):
-        self._keep = (batch, q_idx, w, k_idx, list(layers), kbar, idx_out, count_out)
+                 idx_q_fp8: bool = False, si_fixed_budget: bool = False, si_window_aligned: bool = False,
+                 attn_q_ready=None):
+        """attn_q_ready: a torch.cuda.Event recorded once the layers' attention queries are written
+        (the attention waits for it, the indexer and top-k do not), or None."""
+        self._keep = (batch, q_idx, w, k_idx, list(layers), kbar, idx_out, count_out, attn_q_ready)
         arr = (CLayer * max(1, len(layers)))()
         for i, L in enumerate(layers):
             arr[i] = CLayer(_ptr(L.q), L.kv.c(), L.v.c() if L.v is not None else _EMPTY_CACHE, _ptr(L.o), _ptr(L.lse))
@@ -373,7 +376,8 @@ class DecodeStep:
                                int(kbar.stride(0)) if kbar is not None else 0, int(H), int(Dqk), int(Dv),
                                float(sm_scale), int(n_split), len(layers), arr, _ptr(idx_out),
                                int(idx_out.stride(0)) if idx_out is not None else 0, _ptr(count_out),
-                               int(bool(idx_q_fp8)), int(bool(si_fixed_budget)), int(bool(si_window_aligned)))
+                               int(bool(idx_q_fp8)), int(bool(si_fixed_budget)), int(bool(si_window_aligned)),
+                               attn_q_ready.cuda_event if attn_q_ready is not None else None)
 
     def workspace_size(self) -> int:
         return int(_lib.lsa_decode_workspace_size(ctypes.byref(self.p)))

@@ -522,6 +522,41 @@ def test_fused_path_end_to_end(cuda, name):
                 assert mx < 1e-2 and rl2 < 5e-3, (t, li, mx, rl2, a == b)
 
 
+def test_fused_step_waits_for_the_prolog_event(cuda):
+    """attn_q_ready: the attention layers wait for the caller's event (the MLA prolog writing their
+    queries on another stream), the index selection does not need to.  The queries start as zeros
+    and are written on a side stream after a delay; the outputs must equal those of a step whose
+    queries were ready from the start, bit for bit, and so must the index lists."""
+    wt = wt_of("cli_small")
+    step, ws, idx_ref, cnt_ref, layers = H.decode_step(wt, 0, n_split=2)
+    step(ws)
+    torch.cuda.synchronize()
+    ref = [L.o.clone() for L in layers]
+    w = wt.w
+    pt = wt.passes[0]
+    q_late = [torch.zeros_like(L.q) for L in layers]
+    lay = [lsa.Layer(q, L.kv, torch.full_like(L.o, float("nan")), torch.empty_like(L.lse), L.v)
+           for q, L in zip(q_late, layers)]
+    idx = torch.full_like(idx_ref, -7)
+    cnt = torch.zeros_like(cnt_ref)
+    ev = torch.cuda.Event()
+    dec = lsa.DecodeStep(H.batch_of(wt), pt.q_idx, pt.w, H.idx_cache(wt), w.k, w.n_sink, w.window, lay, w.H, w.D,
+                         w.Dv, w.sm_scale, n_split=2, idx_out=idx, count_out=cnt, attn_q_ready=ev)
+    side = torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        torch.cuda._sleep(20_000_000)                       # the "prolog" takes a while
+        for q, L in zip(q_late, layers):
+            q.copy_(L.q)
+        ev.record(side)
+    dec(ws, stream=main)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_ref) and torch.equal(cnt, cnt_ref)
+    for a, b in zip(lay, ref):
+        assert torch.equal(a.o.view(torch.int16), b.view(torch.int16))
+
+
 @pytest.mark.parametrize("name", ["cli_small", "mtp_small"])
 def test_pipeline_host_io_matches_device_path(cuda, name):
     """lsa_pipeline_*: queries copied in from pinned host memory into two slots of device
