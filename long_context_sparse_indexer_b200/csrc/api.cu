@@ -63,7 +63,7 @@ IndexArgs make_index_args(const lsa_batch* batch, const void* q_idx, const float
 lsa_status index_score_impl(const lsa_batch* batch, const void* q_idx, const float* w, int H_I,
                             const lsa_cache* k_idx, const int32_t* cand, int n_cand, int block_size,
                             float* scores, int64_t ld, int n_cols, int32_t* st, cudaStream_t stream,
-                            bool q_fp8 = false, bool pdl = false) {
+                            bool q_fp8 = false) {
     lsa_status s = check_batch(batch);
     if (s != LSA_OK) return s;
     if ((s = check_cache(k_idx, 0)) != LSA_OK) return s;
@@ -78,7 +78,6 @@ lsa_status index_score_impl(const lsa_batch* batch, const void* q_idx, const flo
     }
     IndexArgs a = make_index_args(batch, q_idx, w, k_idx, cand, n_cand, block_size, scores, ld, n_cols, st);
     a.q_fp8 = q_fp8 ? 1 : 0;
-    a.pdl = pdl ? 1 : 0;
     // The FP8-query mode exists on the tensor-core path only.
     if (q_fp8 && !index_score_tc_supported(a, H_I, k_idx->dim, k_idx->dtype == LSA_FP8_E4M3)) return LSA_ERR_UNSUPPORTED;
     return cuda_status(launch_index_score(a, H_I, k_idx->dim, k_idx->dtype == LSA_FP8_E4M3, stream));
@@ -87,7 +86,7 @@ lsa_status index_score_impl(const lsa_batch* batch, const void* q_idx, const flo
 lsa_status topk_impl(const lsa_batch* batch, const float* scores, int64_t ld, int n_cols,
                      const int32_t* cand, int n_cand, int block_size, int k, int n_sink, int window,
                      uint32_t flags, int32_t* idx, int64_t ld_idx, int32_t* count, int32_t* st,
-                     cudaStream_t stream, bool pdl = false) {
+                     cudaStream_t stream) {
     lsa_status s = check_batch(batch);
     if (s != LSA_OK) return s;
     const bool raw = flags & LSA_TOPK_RAW;
@@ -110,7 +109,6 @@ lsa_status topk_impl(const lsa_batch* batch, const float* scores, int64_t ld, in
     a.cand = cand; a.n_cand = n_cand; a.block_size = block_size;
     a.k = k; a.n_sink = n_sink; a.window = window; a.raw = raw; a.fixed_budget = fixed;
     a.window_align = aligned ? kWindowAlign : 0;
-    a.pdl = pdl ? 1 : 0;
     a.idx = idx; a.ld_idx = ld_idx; a.count = count; a.status = st;
     return cuda_status(launch_topk(a, stream));
 }
@@ -159,8 +157,7 @@ namespace {
 lsa_status attn_impl(const lsa_batch* batch, const void* q, int H, int Dqk, const lsa_cache* kv,
                      const lsa_cache* v, int Dv, const int32_t* idx, int64_t ld_idx, const int32_t* count,
                      float sm_scale, int n_split, void* o, float* lse, void* ws, size_t ws_bytes,
-                     int32_t* st, cudaStream_t stream, float* o32 = nullptr, float* lse32 = nullptr,
-                     bool pdl = false) {
+                     int32_t* st, cudaStream_t stream, float* o32 = nullptr, float* lse32 = nullptr) {
     lsa_status s = attn_validate(batch, q, H, Dqk, kv, v, Dv, idx, ld_idx, count, sm_scale, n_split,
                                  o32 ? static_cast<const void*>(o32) : o);
     if (s != LSA_OK || batch->T == 0) return s;
@@ -190,7 +187,6 @@ lsa_status attn_impl(const lsa_batch* batch, const void* q, int H, int Dqk, cons
         a.part_o = static_cast<float*>(ws);
         a.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up((size_t)batch->T * n_split * H * Dv * 4));
     }
-    a.pdl = pdl ? 1 : 0;
     if (o32) {                    // FP32 result: one split writes it directly, more splits merge into it
         a.f32_out = 1;
         a.o32 = o32;
@@ -392,17 +388,14 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
         s = lsa_block_score(batch, p->q_idx, p->w, p->H_I, p->k_idx.dim, p->kbar, p->kbar_seq_stride,
                             p->block_size, bscores, f.bld, f.nblk, dev_status, st);
         if (s != LSA_OK) return s;
-        // The HI chain is six dependent kernels of a few microseconds each: every one after the
-        // block scores is launched programmatically dependent, so that its set-up (and its launch)
-        // overlaps the end of the previous one; it waits for that kernel before reading its output.
         s = topk_impl(batch, bscores, f.bld, f.nblk, nullptr, 0, 0, p->n_recall, 0, 0, LSA_TOPK_RAW, cand,
-                      p->n_recall, ccount, dev_status, st, true);
+                      p->n_recall, ccount, dev_status, st);
         if (s != LSA_OK) return s;
         s = index_score_impl(batch, p->q_idx, p->w, p->H_I, &p->k_idx, cand, p->n_recall, p->block_size, scores,
-                             f.ld, 0, dev_status, st, p->idx_q_fp8 != 0, true);
+                             f.ld, 0, dev_status, st, p->idx_q_fp8 != 0);
         if (s != LSA_OK) return s;
         s = topk_impl(batch, scores, f.ld, f.n_cols, cand, p->n_recall, p->block_size, p->k, p->n_sink, p->window,
-                      topk_flags, idx, ld_idx, count, dev_status, st, true);
+                      topk_flags, idx, ld_idx, count, dev_status, st);
         if (s != LSA_OK) return s;
     }
     // The attention queries may come from a prolog still running elsewhere: everything below
@@ -424,8 +417,7 @@ lsa_status lsa_decode_fused(const lsa_decode_params* p, void* ws, size_t ws_byte
         const int br = aux ? (l & 1) : 0;
         float* part = reinterpret_cast<float*>(w + f.attn + (size_t)(l & 1) * f.attn_one);
         s = attn_impl(batch, L.q, p->H, p->Dqk, &L.kv, L.v.data ? &L.v : nullptr, p->Dv, idx, ld_idx, count,
-                      p->sm_scale, p->n_split, L.o, L.lse, part, f.attn_one, dev_status, br ? aux->s : st, nullptr,
-                      nullptr, p->hi != 0 && !br);
+                      p->sm_scale, p->n_split, L.o, L.lse, part, f.attn_one, dev_status, br ? aux->s : st);
         if (s != LSA_OK) break;
     }
     if (aux) {                                   // join, also after an error, so the caller's stream waits

@@ -292,7 +292,6 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* part_
                                                               int n_split, int H, int DV, int64_t part_stride,
                                                               int64_t tok_stride, uint16_t* o, float* o32,
                                                               float* lse) {
-    grid_dependency_wait();                                         // the partials of the previous kernel
     const int per_row = DV / 8;
     const int i = blockIdx.x * kMergeThreads + threadIdx.x;       // (head, 8-dim chunk) of token t
     const int t = blockIdx.y;
@@ -395,24 +394,16 @@ cudaError_t launch_merge_partials(const float* part_o, const float* part_lse, in
                                   int64_t tok_stride, int T, int H, int DV, uint16_t* o, float* o32, float* lse,
                                   cudaStream_t st) {
     if (T <= 0) return cudaSuccess;
-    return launch_merge_partials_pdl(false, part_o, part_lse, n_part, part_stride, tok_stride, T, H, DV, o, o32, lse,
-                                     st);
-}
-
-cudaError_t launch_merge_partials_pdl(bool pdl, const float* part_o, const float* part_lse, int n_part,
-                                      int64_t part_stride, int64_t tok_stride, int T, int H, int DV, uint16_t* o,
-                                      float* o32, float* lse, cudaStream_t st) {
-    if (T <= 0) return cudaSuccess;
     dim3 mg((H * (DV / 8) + kMergeThreads - 1) / kMergeThreads, T);
-    return launch_maybe_pdl(pdl, merge_kernel, mg, dim3(kMergeThreads), 0, st, part_o, part_lse, n_part, H, DV,
-                            part_stride, tok_stride, o, o32, lse);
+    merge_kernel<<<mg, kMergeThreads, 0, st>>>(part_o, part_lse, n_part, H, DV, part_stride, tok_stride, o, o32, lse);
+    return cudaGetLastError();
 }
 
 // The merge of one call's split partials ([T][n_split][H]) into its BF16 (or FP32) result.
 static cudaError_t launch_merge(const AttnArgs& a, int DV, cudaStream_t st) {
-    return launch_merge_partials_pdl(a.pdl != 0, a.part_o, a.part_lse, a.n_split, a.H, (int64_t)a.n_split * a.H, a.T,
-                                     a.H, DV, a.f32_out ? nullptr : a.o, a.f32_out ? a.o32 : nullptr,
-                                     a.f32_out ? a.lse32 : a.lse, st);
+    return launch_merge_partials(a.part_o, a.part_lse, a.n_split, a.H, (int64_t)a.n_split * a.H, a.T, a.H, DV,
+                                 a.f32_out ? nullptr : a.o, a.f32_out ? a.o32 : nullptr,
+                                 a.f32_out ? a.lse32 : a.lse, st);
 }
 
 template <int DQK, int DV, int MT, bool KV_FP8, bool SEP_V>

@@ -171,10 +171,6 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    // The set-up above (barriers, TMEM, the query's load) needs nothing from the previous kernel;
-    // the index list does.
-    allow_dependents_early();
-    grid_dependency_wait();
     int n = ok ? a.count[t] : 0;
     if (n < 0 || n > a.ld_idx) { ok = false; n = 0; }
     if (!ok && threadIdx.x == 0 && split == 0 && half == 0) report(a.status, LSA_ERR_DEVICE_DATA);
@@ -704,7 +700,9 @@ cudaError_t launch_t(const CUtensorMap& qm, const CUtensorMap& m, const AttnArgs
     auto kern = sparse_attn_tc_kernel<KV_FP8, TMA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_maybe_pdl(a.pdl != 0, kern, dim3(a.n_split, 2, a.T), dim3(kAThreads), smem, st, qm, m, a);
+    dim3 grid(a.n_split, 2, a.T);
+    kern<<<grid, kAThreads, smem, st>>>(qm, m, a);
+    return cudaGetLastError();
 }
 
 // The BF16 cache as one 2-D tensor of rows (row of sequence b, token i = b * (kv_seq_b / kv_tok_b)

@@ -128,16 +128,6 @@ __device__ __forceinline__ uint4 ldg_nc16(const void* p) {
     return r;
 }
 
-// ---------------------------------------------------------------- programmatic dependent launch
-
-// Waits until the grids this one depends on programmatically have completed and their memory is
-// visible; a no-op when the kernel was launched without the programmatic attribute.
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-// Lets the next kernel of the stream, when launched with the programmatic attribute, start before
-// this grid completes (it still waits for the completion before reading this grid's outputs).
-__device__ __forceinline__ void allow_dependents_early() { asm volatile("griddepcontrol.launch_dependents;" :::); }
-
 // ---------------------------------------------------------------- reductions
 
 __device__ __forceinline__ float warp_max(float v) {

@@ -196,7 +196,6 @@ block_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     const int tid = threadIdx.x, warp = tid >> 5;
     const int t0 = blockIdx.y * G, j0 = blockIdx.x * kBtRows;
     volatile int* abort_flag = &sm.abort;
-    allow_dependents_early();
 
     if (tid < G) {
         int b;

@@ -351,11 +351,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         if (warp < 4) tc::mbar_arrive(&sm.q_full[0]);
     }
 
-    // Everything above read only this call's own inputs; the pipeline below reads what the
-    // previous kernel wrote (the recalled blocks) and writes what it may read.
-    allow_dependents_early();
-    grid_dependency_wait();
-
     if (warp == 0) {
         // ---------------- TMA producer
         if (tc::elect_one()) {
@@ -550,7 +545,8 @@ cudaError_t launch_n(const CUtensorMap& m, const CUtensorMap& sm, const PArgs& p
     auto kern = index_score_tc_kernel<N, NB, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_maybe_pdl(pa.a.pdl != 0, kern, dim3(num_sms()), dim3(kPThreads), smem, st, m, sm, pa);
+    kern<<<num_sms(), kPThreads, smem, st>>>(m, sm, pa);
+    return cudaGetLastError();
 }
 
 int group_size(const IndexArgs& a, int H_I) {

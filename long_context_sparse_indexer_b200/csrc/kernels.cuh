@@ -1,8 +1,6 @@
 // Internal kernel interfaces of the LSA library (argument blocks and host launchers).
 #pragma once
 
-#include <utility>
-
 #include "common.cuh"
 
 namespace lsa {
@@ -25,7 +23,6 @@ struct IndexArgs {
     int group;               // tokens per CTA (<= 4)
     int q_fp8;               // 1: FP8-query mode (queries rounded once to e4m3, tensor-core path only)
     uint64_t wait_ns;        // limit of the tensor-core kernel's pipeline waits (drains keep 2 s)
-    int pdl;                 // launch with the programmatic-dependent attribute (see launch_maybe_pdl)
     int32_t* status;
 };
 
@@ -75,7 +72,6 @@ struct TopkArgs {
     bool raw;
     bool fixed_budget;       // top-k drawn outside the sinks and the window
     int window_align;        // 0, or the block the SI window's start is rounded down to (64)
-    int pdl;                 // launch with the programmatic-dependent attribute
     int32_t* idx;
     int64_t ld_idx;
     int32_t* count;
@@ -106,32 +102,8 @@ struct AttnArgs {
     int f32_out;                // the result in FP32: o32 / lse32 instead of o / lse
     float* o32;                 // [T][H][DV] (f32_out)
     float* lse32;               // [T][H] (f32_out)
-    int pdl;                    // launch the attention (and the merge) programmatically dependent
     int32_t* status;
 };
-
-// Launches kern on st, with the programmatic-dependent-launch attribute when pdl is set: the
-// kernel may then start while the previous kernel of the stream is finishing, and must call
-// grid_dependency_wait() before reading that kernel's outputs or writing what it reads.
-template <typename... KArgs, typename... Args>
-inline cudaError_t launch_maybe_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                                    cudaStream_t st, Args&&... args) {
-    if (!pdl) {
-        kern<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
-        return cudaGetLastError();
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
 
 cudaError_t launch_index_score(IndexArgs a, int H_I, int D_I, bool fp8, cudaStream_t st);
 bool index_score_tc_supported(const IndexArgs& a, int H_I, int D_I, bool fp8);
@@ -148,9 +120,6 @@ cudaError_t launch_sparse_attn_tc(const AttnArgs& a, bool kv_fp8, cudaStream_t s
 cudaError_t launch_merge_partials(const float* part_o, const float* part_lse, int n_part, int64_t part_stride,
                                   int64_t tok_stride, int T, int H, int DV, uint16_t* o, float* o32, float* lse,
                                   cudaStream_t st);
-cudaError_t launch_merge_partials_pdl(bool pdl, const float* part_o, const float* part_lse, int n_part,
-                                      int64_t part_stride, int64_t tok_stride, int T, int H, int DV, uint16_t* o,
-                                      float* o32, float* lse, cudaStream_t st);
 
 // KVP helpers (kvp.cu).
 cudaError_t launch_kvp_shard_batch(int B, int T, int L_alloc_local, const int32_t* seq_len, const int32_t* q_seq,

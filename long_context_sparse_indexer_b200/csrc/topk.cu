@@ -259,8 +259,6 @@ topk_kernel(TopkArgs a) {
     const float* row = a.scores + (size_t)t * a.ld;
     int32_t* out = a.idx + (size_t)t * a.ld_idx;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    allow_dependents_early();
-    grid_dependency_wait();                       // the scores come from the previous kernel
 
     // Query position and its validity (identical in every CTA of the cluster).
     const int b = a.q_seq[t];
@@ -628,14 +626,12 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
         cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)std::max((size_t)kTopkCacheCols * 4, cand_smem));
         if (e != cudaSuccess) return e;
-        return launch_maybe_pdl(a.pdl != 0, topk_kernel<true>, dim3(a.T * kTopkCluster), dim3(kTopkThreads), smem,
-                                st, a);
+        topk_kernel<true><<<a.T * kTopkCluster, kTopkThreads, smem, st>>>(a);
     } else {
         cudaError_t e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)cand_smem);
         if (e != cudaSuccess) return e;
-        return launch_maybe_pdl(a.pdl != 0, topk_kernel<false>, dim3(a.T * kTopkCluster), dim3(kTopkThreads),
-                                cand_smem, st, a);
+        topk_kernel<false><<<a.T * kTopkCluster, kTopkThreads, cand_smem, st>>>(a);
     }
     return cudaGetLastError();
 }

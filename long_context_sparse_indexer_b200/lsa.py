@@ -377,7 +377,8 @@ class DecodeStep:
                                float(sm_scale), int(n_split), len(layers), arr, _ptr(idx_out),
                                int(idx_out.stride(0)) if idx_out is not None else 0, _ptr(count_out),
                                int(bool(idx_q_fp8)), int(bool(si_fixed_budget)), int(bool(si_window_aligned)),
-                               attn_q_ready.cuda_event if attn_q_ready is not None else None)
+                               None)
+        self._attn_q_ready = attn_q_ready
 
     def workspace_size(self) -> int:
         return int(_lib.lsa_decode_workspace_size(ctypes.byref(self.p)))
@@ -386,6 +387,9 @@ class DecodeStep:
         return int(_lib.lsa_decode_index_capacity(ctypes.byref(self.p)))
 
     def __call__(self, ws: torch.Tensor, dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+        if self._attn_q_ready is not None:
+            # torch creates an event's CUDA handle at its first record: read it at each call
+            self.p.attn_q_ready = self._attn_q_ready.cuda_event or None
         _check(_lib.lsa_decode_fused(ctypes.byref(self.p), _ptr(ws), ws.numel() * ws.element_size(),
                                      _ptr(dev_status), _stream(stream)), "lsa_decode_fused")
 
