@@ -250,8 +250,7 @@ topk_kernel(TopkArgs a) {
     __shared__ int s_warp[kTopkWarps];
     __shared__ int s_bin, s_above, s_slot[3], s_wmax;
     __shared__ int s_wcnt[kTopkWarps], s_wk[kTopkWarps];
-    __shared__ int s_sup[64], s_red[130], s_total;
-    __shared__ uint32_t s_mm[2], s_mmw[2][kTopkWarps];   // this CTA's smallest and largest key
+    __shared__ int s_sup[64], s_red[130], s_total, hist3[256];
     __shared__ int s_cand[kTopkCandCache];        // the row's candidate block ids (HI), when they fit
     extern __shared__ uint32_t s_keys[];          // CACHED: order key of each column of the segment, 0 = invalid
     cg::cluster_group cl = cg::this_cluster();
@@ -317,13 +316,7 @@ topk_kernel(TopkArgs a) {
         return (f != f || f == kNegInf || fixed_pos(cc)) ? 0u : order_key(f);
     };
 
-    // ---- the segment's keys (cached in shared memory when they fit) and the row's smallest and
-    // largest key.  The radix digits are those of d = key - kmin, 12 bits at a time from the top
-    // of the row's range (not of the key's 32 bits): scores in a narrow range then spread over the
-    // 4096 bins of the first pass instead of piling into a few (shared-memory atomics on one bin
-    // serialise, and a crowded threshold bin leaves too many candidates for CTA 0).  d preserves
-    // the order of the keys, so the selection is the same.
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    // ---- pass 1: top 12 bits (and, when cached, the segment's keys into shared memory)
     for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
     if (CACHED) {
         // Batches of 8 independent 16-byte loads per thread, then conversion to keys.
@@ -350,50 +343,22 @@ topk_kernel(TopkArgs a) {
                     if (cc + e >= c1) break;
                     const float x = f[u][e];
                     if (x != x) report(a.status, LSA_ERR_DEVICE_DATA);
-                    const uint32_t key = (x != x || x == kNegInf || fixed_pos(cc + e)) ? 0u : order_key(x);
-                    s_keys[cc + e - c0] = key;
-                    if (key) { kmin = min(kmin, key); kmax = max(kmax, key); }
+                    s_keys[cc + e - c0] = (x != x || x == kNegInf || fixed_pos(cc + e)) ? 0u : order_key(x);
                 }
             }
         }
-    } else {
-        for (int c = w0; c < w1; c += 32) {
-            const int cc = c + lane;
-            if (cc < w1) {
-                const float f = row[cc];
-                if (f != f) report(a.status, LSA_ERR_DEVICE_DATA);
-            }
-            const uint32_t key = key_at(cc);
-            if (key) { kmin = min(kmin, key); kmax = max(kmax, key); }
-        }
     }
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    if (lane == 0) { s_mmw[0][warp] = kmin; s_mmw[1][warp] = kmax; }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t lo = 0xffffffffu, hi = 0u;
-        for (int w = 0; w < kTopkWarps; ++w) { lo = min(lo, s_mmw[0][w]); hi = max(hi, s_mmw[1][w]); }
-        s_mm[0] = lo;
-        s_mm[1] = hi;
-    }
-    cl.sync();                                           // every CTA's extremes are written
-    kmin = 0xffffffffu;
-    kmax = 0u;
-#pragma unroll
-    for (int r = 0; r < kTopkCluster; ++r) {
-        const uint32_t* mm = cl.map_shared_rank(s_mm, r);
-        kmin = min(kmin, mm[0]);
-        kmax = max(kmax, mm[1]);
-    }
-    const uint32_t span = kmax >= kmin ? kmax - kmin : 0u;     // no valid key: kmin > kmax
-    const int s1 = max(0, (span ? 32 - __clz(span) : 0) - 12);
-    // ---- pass 1: the top digit of d
     for (int c = w0; c < w1; c += 32) {
-        const uint32_t key = key_at(c + lane);
-        hist_add(hist, key ? (int)((key - kmin) >> s1) : 0, key != 0u);
+        const int cc = c + lane;
+        if (!CACHED && cc < w1) {
+            const float f = row[cc];
+            if (f != f) report(a.status, LSA_ERR_DEVICE_DATA);
+        }
+        const uint32_t key = key_at(cc);
+        hist_add(hist, (int)(key >> 20), key != 0u);
     }
-    // Cluster histogram of the top digit; its total is the number of candidates.
+    // Cluster histogram of the top 12 bits; its total is the number of candidates.
     const int n_valid = cluster_threshold_4096(cl, hist, s_sup, a.k, s_red, &s_bin, &s_above, &s_total);
     const bool take_all = n_valid <= a.k;
 
@@ -402,7 +367,7 @@ topk_kernel(TopkArgs a) {
     // of `hsum`; when they fit, every warp stores them into CTA 0's merged list, and CTA 0
     // completes the selection and the emission alone.
     {
-        const uint32_t tb = a.k <= 0 ? 0xffffffffu : (take_all ? 1u : kmin + ((uint32_t)s_bin << s1));
+        const uint32_t tb = a.k <= 0 ? 0xffffffffu : (take_all ? 1u : ((uint32_t)s_bin << 20));
         // One pass: warp w appends its candidates (column order) to its own region of kTopkWarpCap
         // slots of the CTA's list in `hsum` (keys, then columns).
         uint32_t* lkey = reinterpret_cast<uint32_t*>(hsum);
@@ -448,44 +413,36 @@ topk_kernel(TopkArgs a) {
             }
             // No peer reads `hist` any more (the count barrier above): CTA 0 clears its
             // histograms for passes 2 and 3 while the candidates arrive.
-            if (rank == 0)
+            if (rank == 0) {
                 for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
+                if (threadIdx.x < 256) hist3[threadIdx.x] = 0;
+            }
             cl.sync();                                   // every candidate has reached CTA 0
             if (rank != 0) return;
             const int n = total;
             uint32_t vs = 0;
             int m_keep = 0, n_eq = 0;
             if (!take_all && a.k > 0) {
-                // The next digits of d among the candidates in the threshold bin, down to d itself.
-                uint32_t pre = (uint32_t)s_bin;          // d >> s of the threshold bin
-                int above = s_above, s = s1;
-                bool counted = false;
-                while (s > 0) {
-                    const int s_next = max(0, s - 12), nb = 1 << (s - s_next);
-                    for (int i = threadIdx.x; i < nb; i += kTopkThreads) hist[i] = 0;
-                    __syncthreads();
-                    for (int i = threadIdx.x; i < n; i += kTopkThreads) {
-                        const uint32_t d = ckey[i] - kmin;
-                        if ((d >> s) == pre) atomicAdd(&hist[(d >> s_next) & (nb - 1)], 1);
-                    }
-                    __syncthreads();
-                    local_threshold(hist, nb, a.k - above, s_warp, &s_bin, &s_above);
-                    pre = (pre << (s - s_next)) | (uint32_t)s_bin;
-                    above += s_above;
-                    n_eq = hist[s_bin];                  // keys in that bin (== vs once s_next is 0)
-                    counted = true;
-                    s = s_next;
+                const uint32_t b1 = (uint32_t)s_bin;
+                int above = s_above;
+                for (int i = threadIdx.x; i < n; i += kTopkThreads) {
+                    const uint32_t key = ckey[i];
+                    if ((key >> 20) == b1) atomicAdd(&hist[(key >> 8) & 0xfff], 1);
                 }
-                vs = kmin + pre;
-                if (!counted) {                          // d was exact in the first pass
-                    if (threadIdx.x == 0) hist[0] = 0;
-                    __syncthreads();
-                    for (int i = threadIdx.x; i < n; i += kTopkThreads)
-                        if (ckey[i] == vs) atomicAdd(&hist[0], 1);
-                    __syncthreads();
-                    n_eq = hist[0];
+                __syncthreads();
+                local_threshold(hist, 4096, a.k - above, s_warp, &s_bin, &s_above);
+                const uint32_t pre = (b1 << 12) | (uint32_t)s_bin;
+                above += s_above;
+                for (int i = threadIdx.x; i < n; i += kTopkThreads) {
+                    const uint32_t key = ckey[i];
+                    if ((key >> 8) == pre) atomicAdd(&hist3[key & 0xff], 1);
                 }
+                __syncthreads();
+                local_threshold(hist3, 256, a.k - above, s_warp, &s_bin, &s_above);
+                above += s_above;
+                vs = (pre << 8) | (uint32_t)s_bin;
                 m_keep = a.k - above;                    // keys == vs to keep, lowest columns first
+                n_eq = hist3[s_bin];                     // keys == vs among the candidates
             }
             const bool every = take_all || a.k <= 0;     // every candidate is selected (none when k = 0)
             const bool ties_all = every || m_keep >= n_eq;
@@ -556,28 +513,29 @@ topk_kernel(TopkArgs a) {
     uint32_t vstar = 0;
     int above = 0;
     if (!take_all && a.k > 0) {
-        // ---- full passes over the segments: the next digits of d among the keys of the threshold
-        // bin, down to d itself (cluster_threshold wants a multiple of kTopkCluster bins: the
-        // bins past the digit's range stay empty).
-        uint32_t pre = (uint32_t)s_bin;
+        const uint32_t b1 = (uint32_t)s_bin;
         above = s_above;
-        int s = s1;
-        while (s > 0) {
-            const int s_next = max(0, s - 12), nb = 1 << (s - s_next), nb_alloc = max(nb, kTopkCluster);
-            __syncthreads();
-            for (int i = threadIdx.x; i < nb_alloc; i += kTopkThreads) hist[i] = 0;
-            __syncthreads();
-            for (int c = w0; c < w1; c += 32) {
-                const uint32_t key = key_at(c + lane);
-                const uint32_t d = key - kmin;
-                hist_add(hist, (int)((d >> s_next) & (nb - 1)), key != 0u && (d >> s) == pre);
-            }
-            cluster_threshold(cl, rank, hist, hsum, nb_alloc, a.k - above, s_warp, &s_bin, &s_above);
-            pre = (pre << (s - s_next)) | (uint32_t)s_bin;
-            above += s_above;
-            s = s_next;
+        // ---- pass 2: next 12 bits among keys with prefix b1
+        for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
+        __syncthreads();
+        for (int c = w0; c < w1; c += 32) {
+            const uint32_t key = key_at(c + lane);
+            hist_add(hist, (int)((key >> 8) & 0xfff), key != 0u && (key >> 20) == b1);
         }
-        vstar = kmin + pre;
+        cluster_threshold(cl, rank, hist, hsum, 4096, a.k - above, s_warp, &s_bin, &s_above);
+        const uint32_t b2 = (uint32_t)s_bin;
+        above += s_above;
+        // ---- pass 3: last 8 bits among keys with prefix (b1, b2)
+        const uint32_t pre = (b1 << 12) | b2;
+        for (int i = threadIdx.x; i < 256; i += kTopkThreads) hist[i] = 0;
+        __syncthreads();
+        for (int c = w0; c < w1; c += 32) {
+            const uint32_t key = key_at(c + lane);
+            hist_add(hist, (int)(key & 0xff), key != 0u && (key >> 8) == pre);
+        }
+        cluster_threshold(cl, rank, hist, hsum, 256, a.k - above, s_warp, &s_bin, &s_above);
+        above += s_above;
+        vstar = (pre << 8) | (uint32_t)s_bin;
     }
     const int m_ties = a.k - above;           // keys == v* to keep (lowest columns first)
 
