@@ -490,7 +490,7 @@ def indexer_traffic(kern: str, idx_bytes: float):
     if kern.startswith("index_score"):
         rec, src_file = "indexer_traffic.json", "index_score_tc.cu"
     elif kern.startswith("block_score"):
-        rec, src_file = "block_score_traffic.json", "hi_blocks.cu"
+        rec, src_file = "block_score_traffic.json", "row_score_tc.cu"
     else:
         return None
     try:

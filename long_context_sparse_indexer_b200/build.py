@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT = os.path.join(HERE, "_lsa.so")
 BUILD = os.path.join(HERE, "_build")
 
-SOURCES = ["api.cu", "pipeline.cu", "index_score.cu", "index_score_tc.cu", "hi_blocks.cu", "topk.cu", "attention.cu", "attention_tc.cu", "noalloc.cu", "kvp.cu"]
+SOURCES = ["api.cu", "pipeline.cu", "index_score.cu", "index_score_tc.cu", "hi_blocks.cu", "topk.cu", "attention.cu", "attention_tc.cu", "noalloc.cu", "kvp.cu", "row_score_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
 

@@ -269,6 +269,16 @@ cudaError_t launch_index_score(IndexArgs a, int H_I, int D_I, bool fp8, cudaStre
                                                            : (a.q_group % 2 == 0 ? 2 : 1));
     if (a.n_cols <= 0 || a.T <= 0) return cudaSuccess;
     if (index_score_tc_supported(a, H_I, D_I, fp8)) return launch_index_score_tc(a, H_I, st);
+    if (!fp8 && !a.cand) {
+        // BF16 keys: the tensor-core row scorer (row_score_tc.cu), one key per row.
+        RowScoreArgs r{};
+        r.seq_len = a.seq_len; r.q_seq = a.q_seq; r.q_pos = a.q_pos;
+        r.B = a.B; r.T = a.T; r.L_alloc = a.L_alloc; r.q_group = a.q_group;
+        r.q = a.q; r.w = a.w; r.H_I = H_I; r.d_I = D_I; r.halves = 1; r.row_span = 1;
+        r.scores = a.scores; r.ld = a.ld; r.n_cols = a.n_cols; r.status = a.status;
+        if (row_score_tc_supported(r, D_I, a.tok_stride_b, a.seq_stride_b, a.kdata))
+            return launch_row_score_tc(r, a.L_alloc, a.tok_stride_b, a.seq_stride_b, a.kdata, st);
+    }
     if (fp8) return D_I == 64 ? launch_index_d<true, 64>(a, H_I, st) : launch_index_d<true, 128>(a, H_I, st);
     return D_I == 64 ? launch_index_d<false, 64>(a, H_I, st) : launch_index_d<false, 128>(a, H_I, st);
 }

@@ -58,6 +58,26 @@ struct BlockScoreArgs {
     int32_t* status;
 };
 
+// Indexer-form scores of BF16 rows on the tensor cores (row_score_tc.cu): HI block keys stored
+// as [hi | lo] pairs (halves = 2, row_span = block size) or BF16 indexer keys (halves = 1,
+// row_span = 1).  Row j of token t is visible when j * row_span <= q_pos[t].
+struct RowScoreArgs {
+    const int32_t* seq_len;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    int B, T, L_alloc, q_group;
+    const uint16_t* q;       // bf16 [T][H_I][d_I]
+    const float* w;          // [T][H_I]
+    int H_I, d_I;
+    int halves;              // row = halves x d_I BF16 values
+    int row_span;            // positions per row
+    float* scores;
+    int64_t ld;
+    int n_cols;
+    uint64_t wait_ns;
+    int32_t* status;
+};
+
 struct TopkArgs {
     const int32_t* seq_len;
     const int32_t* q_seq;
@@ -110,6 +130,11 @@ bool index_score_tc_supported(const IndexArgs& a, int H_I, int D_I, bool fp8);
 cudaError_t launch_index_score_tc(IndexArgs a, int H_I, cudaStream_t st);
 cudaError_t launch_block_keys(const BlockKeyArgs& a, cudaStream_t st);
 cudaError_t launch_block_score(const BlockScoreArgs& a, int H_I, cudaStream_t st);
+int row_score_group(int q_group, int H_I);
+bool row_score_tc_supported(const RowScoreArgs& a, int row_elems, int64_t row_stride_b, int64_t seq_stride_b,
+                            const void* rows);
+cudaError_t launch_row_score_tc(const RowScoreArgs& a, int n_rows, int64_t row_stride_b, int64_t seq_stride_b,
+                                const void* rows, cudaStream_t st);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int DQK, int DV, bool kv_fp8, bool sep_v, cudaStream_t st);
 bool sparse_attn_tc_supported(const AttnArgs& a, int DQK, int DV, bool sep_v);

@@ -35,8 +35,11 @@ SMALL = {
     # reads them directly instead of by TMA), and a 64-dim FP8 indexer (warp-MMA kernel).
     "cli_unaligned": W.scaled("decode_cli_128k", B=3, len_lo=2500, len_hi=5200, seed=12),
     "cli_d64": W.scaled("decode_cli_128k", B=2, len_lo=3000, len_hi=4100, d_I=64, seed=13),
+    # BF16 indexer keys at d_I = 128 (the tensor-core row scorer), query groups of 1 and of 4
+    "cli_bf16": W.scaled("decode_cli_128k", B=3, len_lo=2500, len_hi=5200, idx_fp8=False, seed=14),
+    "mtp_bf16": W.scaled("mtp_256k", B=2, len_lo=3001, len_hi=3001, idx_fp8=False, seed=15),
 }
-FLAT = ["tiny_decode", "cli_small", "mtp_small", "prefill_small", "cli_unaligned", "cli_d64"]
+FLAT = ["tiny_decode", "cli_small", "mtp_small", "prefill_small", "cli_unaligned", "cli_d64", "cli_bf16", "mtp_bf16"]
 L_ALLOC = {"cli_unaligned": 5203}
 
 _cache = {}
@@ -206,9 +209,15 @@ def test_hi_fine_scores_fp8_query(cuda):
             assert np.all(np.isneginf(cols[~vis]))
 
 
-def test_block_keys_and_block_scores(cuda):
-    w = SMALL["hi_small"]
-    wt = wt_of("hi_small")
+@pytest.mark.parametrize("heads", [64, 16])
+def test_block_keys_and_block_scores(cuda, heads):
+    """Block keys against the oracle's means, block scores against the indexer formula on them;
+    64 heads (32-column TMEM reads) and 16 heads (8-column reads, query rows padded to 32)."""
+    if heads == 64:
+        w, wt = SMALL["hi_small"], wt_of("hi_small")
+    else:
+        w = W.scaled("decode_hi_1m", B=2, len_lo=9000, len_hi=9000, H_I=16, seed=16)
+        wt = D.build_workload(w, "cuda")
     p = w.passes[0]
     kbar_dev = H.block_keys(wt)
     kbar = H.block_key_values(kbar_dev)
