@@ -194,3 +194,55 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(cls), cname
         for fname, _ in cls._fields_:
             assert got[(cname, fname)] == getattr(cls, fname).offset, (cname, fname)
+
+
+def test_kvp_and_partial_calls_reject_bad_arguments():
+    """The KVP calls, the FP32 partial attention and the merge validate on the host (no GPU: each of
+    these returns before any CUDA call)."""
+    lib = lsa.library()
+    b = _batch(T=2, B=1)
+    # lsa_merge_partials: sizes, alignment, the token limit
+    assert lib.lsa_merge_partials(16, 16, 0, 2, 128, 512, 16, None, None) == lsa.ERR_INVALID_ARG     # no parts
+    assert lib.lsa_merge_partials(16, 16, 2, 2, 128, 500, 16, None, None) == lsa.ERR_INVALID_ARG     # Dv % 8
+    assert lib.lsa_merge_partials(None, 16, 2, 2, 128, 512, 16, None, None) == lsa.ERR_INVALID_ARG
+    assert lib.lsa_merge_partials(24, 16, 2, 2, 128, 512, 16, None, None) == lsa.ERR_INVALID_ARG     # unaligned
+    assert lib.lsa_merge_partials(16, 16, 2, 70000, 128, 512, 16, None, None) == lsa.ERR_UNSUPPORTED
+    assert lib.lsa_merge_partials(16, 16, 2, 0, 128, 512, 16, None, None) == lsa.OK                  # nothing to do
+    # lsa_kvp_select: part counts, workspace
+    need = lsa.kvp_select_workspace_size(2, 4, 100)
+    assert need >= 2 * 4 * 100 * 8
+    sel = lambda n_parts=4, k_part=100, ws=4096, wsb=need: lib.lsa_kvp_select(  # noqa
+        ctypes.byref(b), 16, 16, n_parts, k_part, 100, 4, 16, 16, 200, 16, ws, wsb, None, None)
+    assert sel(n_parts=0) == lsa.ERR_INVALID_ARG
+    assert sel(k_part=0) == lsa.ERR_INVALID_ARG
+    assert sel(ws=None) == lsa.ERR_WORKSPACE
+    assert sel(wsb=need - 1) == lsa.ERR_WORKSPACE
+    assert sel(ws=4100) == lsa.ERR_WORKSPACE                                               # not 256-byte aligned
+    # lsa_kvp_local_index: the local list must be at least as wide as the global one
+    assert lib.lsa_kvp_local_index(ctypes.byref(b), 16, 16, 16, 200, 16, 16, 199, 16, None, None) == lsa.ERR_INVALID_ARG
+    # lsa_kvp_candidates: k >= 1, pointers
+    assert lib.lsa_kvp_candidates(ctypes.byref(b), 16, 16, 16, 100, 100, 0, 16, 16, 16, None, None) == lsa.ERR_INVALID_ARG
+    assert lib.lsa_kvp_candidates(ctypes.byref(b), None, 16, 16, 100, 100, 8, 16, 16, 16, None, None) == lsa.ERR_INVALID_ARG
+    # lsa_kvp_shard_batch
+    assert lib.lsa_kvp_shard_batch(ctypes.byref(b), 0, 16, 16, 16, 16, None, None) == lsa.ERR_INVALID_ARG
+    assert lib.lsa_kvp_shard_batch(ctypes.byref(b), 64, None, 16, 16, 16, None, None) == lsa.ERR_INVALID_ARG
+    # lsa_sparse_attn_partial: both FP32 outputs are required; otherwise lsa_sparse_attn's checks
+    kv = _cache(dtype=lsa.BF16, dim=576, scale=None)
+    part = lambda o=4096, l=4096, H=128: lib.lsa_sparse_attn_partial(  # noqa
+        ctypes.byref(b), 4096, H, 576, ctypes.byref(kv), None, 512, 16, 100, 16, 0.04, 1, o, l, None, 0, None, None)
+    assert part(o=None) == lsa.ERR_INVALID_ARG
+    assert part(l=None) == lsa.ERR_INVALID_ARG
+    assert part(H=100) == lsa.ERR_UNSUPPORTED
+
+
+def test_wait_limit_setter_and_index_capacity():
+    assert lsa.set_wait_limit_ns(5) == 0                  # the default is 0 (2 s)
+    assert lsa.set_wait_limit_ns(0) == 5
+    p = lsa.CDecodeParams()
+    p.k, p.n_sink, p.window = 2048, 4, 512
+    lib = lsa.library()
+    assert lib.lsa_decode_index_capacity(ctypes.byref(p)) == 2564
+    p.si_window_aligned = 1
+    assert lib.lsa_decode_index_capacity(ctypes.byref(p)) == 2564 + lsa.WINDOW_ALIGN - 1
+    p.window = 0
+    assert lib.lsa_decode_index_capacity(ctypes.byref(p)) == 2052
