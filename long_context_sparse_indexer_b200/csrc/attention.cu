@@ -5,8 +5,8 @@
 // attention is MLA in absorbed form, so all heads of a query share one latent KV row
 // (K = the 576-dim row, V = its first 512 dims).  Section "③ KVP 解码切分示意": each KV
 // shard computes a partial attention and the partial results are merged; here the shards
-// are contiguous chunks of one query's index list (n_split), merged in a fixed binary
-// tree, as the release post's section "确定性与可靠性" asks of reductions.
+// are contiguous chunks of one query's index list (n_split), merged in split order, a fixed
+// order, as the release post's section "确定性与可靠性" asks of reductions.
 //
 // CTA = (split, group of 16*MT heads, query token).  Warps 0..4*MT-1: warp w owns head
 // tile (w % MT) and quarter (w / MT).  For S = Q K^T each quarter computes a partial over
@@ -279,123 +279,122 @@ sparse_attn_kernel(AttnArgs a) {
     }
 }
 
-// Split merge: thread = 8 consecutive V dims of one (token, head).  With m = max_s lse_s and
-// w_s = exp(lse_s - m): o = sum_s (w_s / sum w) o_s and lse = m + log(sum w), sums in split
-// order.  Up to kMergeRegs splits are loaded before any arithmetic (one memory round trip).
+// Split merge.  With m = max_s lse_s and w_s = exp(lse_s - m): o = sum_s (w_s / sum w) o_s and
+// lse = m + log(sum w), both sums in split order (the values do not depend on the kernel below).
 // Partial s of (token t, head h) is row s * part_stride + t * tok_stride + h; the splits of one
 // call are [T][n_split][H] (part_stride = H, tok_stride = n_split * H), the per-rank partials of
 // KVP [n_part][T][H] (part_stride = T * H, tok_stride = H).
-constexpr int kMergeThreads = 256;
-constexpr int kMergeRegs = 8;
+//
+// Up to 32 splits: warp = 128 consecutive V dims of one (token, head), lane = 4 of them.  Lane s
+// loads lse_s and computes w_s; the others get it by shuffle, so the weights need no shared
+// memory and no block barrier, and the first kMergeNS partial rows are loaded together with the
+// lse values (one memory round trip).
+constexpr int kMergeThreads = 128;
+constexpr int kMergeNS = 24;
+
+__device__ __forceinline__ void merge_store(const float4& acc, size_t out, uint16_t* o, float* o32) {
+    if (o32) {
+        *reinterpret_cast<float4*>(o32 + out) = acc;
+    } else {
+        uint2 pk;
+        pk.x = pack_bf16x2(acc.x, acc.y);
+        pk.y = pack_bf16x2(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(o + out) = pk;
+    }
+}
+
+__device__ __forceinline__ void axpy4(float ws, const float4& x, float4& acc) {
+    acc.x = fmaf(ws, x.x, acc.x); acc.y = fmaf(ws, x.y, acc.y);
+    acc.z = fmaf(ws, x.z, acc.z); acc.w = fmaf(ws, x.w, acc.w);
+}
 
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* part_o, const float* part_lse,
                                                               int n_split, int H, int DV, int64_t part_stride,
                                                               int64_t tok_stride, uint16_t* o, float* o32,
                                                               float* lse) {
-    const int per_row = DV / 8;
-    const int i = blockIdx.x * kMergeThreads + threadIdx.x;       // (head, 8-dim chunk) of token t
+    const int lane = threadIdx.x & 31;
+    const int chunks = (DV + 127) / 128;
+    const int64_t gw = (int64_t)blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
     const int t = blockIdx.y;
-    if (i >= H * per_row) return;
-    const int h = i / per_row, d = (i % per_row) * 8;
+    if (gw >= (int64_t)H * chunks) return;                        // whole warps
+    const int h = (int)(gw / chunks), d = (int)(gw % chunks) * 128 + lane * 4;
+    const bool act = d < DV;
     const size_t row0 = (size_t)t * tok_stride + h;                // (split 0, head h)
+    auto src = [&](int s) {
+        return reinterpret_cast<const float4*>(part_o + (row0 + (size_t)s * part_stride) * DV + d);
+    };
+    float4 x[kMergeNS];
+    if (act) {
+#pragma unroll
+        for (int s = 0; s < kMergeNS; ++s)
+            if (s < n_split) x[s] = __ldcg(src(s));
+    }
+    const float l = lane < n_split ? __ldcg(part_lse + row0 + (size_t)lane * part_stride) : kNegInf;
+    const float m = warp_max(l);
+    const float e = lane < n_split && m != kNegInf ? expf(l - m) : 0.f;
+    float wsum = 0.f;
+    for (int s = 0; s < n_split; ++s) wsum += __shfl_sync(0xffffffffu, e, s);
+    const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < kMergeNS; ++s) {
+        const float ws = __shfl_sync(0xffffffffu, e, s) * rs;
+        if (s < n_split) axpy4(ws, x[s], acc);
+    }
+    for (int s = kMergeNS; s < n_split; ++s) {                     // 25..32 splits: a second round trip
+        const float ws = __shfl_sync(0xffffffffu, e, s) * rs;
+        if (act) axpy4(ws, __ldcg(src(s)), acc);
+    }
+    if (act) merge_store(acc, ((size_t)t * H + h) * DV + d, o, o32);
+    if (lse && lane == 0 && (gw % chunks) == 0) lse[(size_t)t * H + h] = wsum > 0.f ? m + logf(wsum) : kNegInf;
+}
+
+// More than 32 splits: block = one (token, head), thread = 4 consecutive V dims (and every 512th
+// dim after them); the lse values go through shared memory once, the rows in chunks of kMergeNS.
+__global__ void __launch_bounds__(kMergeThreads) merge_wide_kernel(const float* part_o, const float* part_lse,
+                                                                   int n_split, int DV, int64_t part_stride,
+                                                                   int64_t tok_stride, uint16_t* o, float* o32,
+                                                                   float* lse) {
+    extern __shared__ float s_l[];                                 // lse of every split of this (token, head)
+    const int h = blockIdx.x, t = blockIdx.y, H = gridDim.x;
+    const size_t row0 = (size_t)t * tok_stride + h;
+    for (int s = threadIdx.x; s < n_split; s += kMergeThreads)
+        s_l[s] = __ldcg(part_lse + row0 + (size_t)s * part_stride);
+    __syncthreads();
     float m = kNegInf, wsum = 0.f;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (n_split <= kMergeRegs) {
-        float l[kMergeRegs];
-        float4 x0[kMergeRegs], x1[kMergeRegs];
+    for (int s = 0; s < n_split; ++s) m = fmaxf(m, s_l[s]);
+    for (int s = 0; s < n_split; ++s) wsum += m == kNegInf ? 0.f : expf(s_l[s] - m);
+    const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
+    for (int d = 4 * threadIdx.x; d < DV; d += 4 * kMergeThreads) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < n_split; s0 += kMergeNS) {
+            float4 x[kMergeNS];
 #pragma unroll
-        for (int s = 0; s < kMergeRegs; ++s) {
-            if (s < n_split) {
-                const size_t r = row0 + (size_t)s * part_stride;
-                l[s] = __ldcg(part_lse + r);
-                const float4* src = reinterpret_cast<const float4*>(part_o + r * DV + d);
-                x0[s] = __ldcg(src);
-                x1[s] = __ldcg(src + 1);
-            }
+            for (int u = 0; u < kMergeNS; ++u)
+                if (s0 + u < n_split)
+                    x[u] = __ldcg(reinterpret_cast<const float4*>(part_o + (row0 + (size_t)(s0 + u) * part_stride) * DV + d));
+#pragma unroll
+            for (int u = 0; u < kMergeNS; ++u)
+                if (s0 + u < n_split) axpy4((m == kNegInf ? 0.f : expf(s_l[s0 + u] - m)) * rs, x[u], acc);
         }
-#pragma unroll
-        for (int s = 0; s < kMergeRegs; ++s) if (s < n_split) m = fmaxf(m, l[s]);
-#pragma unroll
-        for (int s = 0; s < kMergeRegs; ++s) {
-            if (s < n_split) { l[s] = m == kNegInf ? 0.f : expf(l[s] - m); wsum += l[s]; }
-        }
-        const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
-#pragma unroll
-        for (int s = 0; s < kMergeRegs; ++s) {
-            if (s < n_split) {
-                const float ws = l[s] * rs;
-                acc[0] = fmaf(ws, x0[s].x, acc[0]); acc[1] = fmaf(ws, x0[s].y, acc[1]);
-                acc[2] = fmaf(ws, x0[s].z, acc[2]); acc[3] = fmaf(ws, x0[s].w, acc[3]);
-                acc[4] = fmaf(ws, x1[s].x, acc[4]); acc[5] = fmaf(ws, x1[s].y, acc[5]);
-                acc[6] = fmaf(ws, x1[s].z, acc[6]); acc[7] = fmaf(ws, x1[s].w, acc[7]);
-            }
-        }
-    } else {
-        // More splits than registers: the same arithmetic in the same split order, with the loads
-        // of kMergeRegs splits issued together before their arithmetic (a round trip per chunk,
-        // not per split).
-        for (int s0 = 0; s0 < n_split; s0 += kMergeRegs) {
-            float l[kMergeRegs];
-#pragma unroll
-            for (int u = 0; u < kMergeRegs; ++u)
-                l[u] = s0 + u < n_split ? __ldcg(part_lse + row0 + (size_t)(s0 + u) * part_stride) : kNegInf;
-#pragma unroll
-            for (int u = 0; u < kMergeRegs; ++u) m = fmaxf(m, l[u]);
-        }
-        for (int s0 = 0; s0 < n_split; s0 += kMergeRegs) {
-            float l[kMergeRegs];
-#pragma unroll
-            for (int u = 0; u < kMergeRegs; ++u)
-                l[u] = s0 + u < n_split ? __ldcg(part_lse + row0 + (size_t)(s0 + u) * part_stride) : 0.f;
-#pragma unroll
-            for (int u = 0; u < kMergeRegs; ++u)
-                if (s0 + u < n_split) wsum += m == kNegInf ? 0.f : expf(l[u] - m);
-        }
-        const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
-        for (int s0 = 0; s0 < n_split; s0 += kMergeRegs) {
-            float l[kMergeRegs];
-            float4 x0[kMergeRegs], x1[kMergeRegs];
-#pragma unroll
-            for (int u = 0; u < kMergeRegs; ++u) {
-                if (s0 + u < n_split) {
-                    const size_t r = row0 + (size_t)(s0 + u) * part_stride;
-                    l[u] = __ldcg(part_lse + r);
-                    const float4* src = reinterpret_cast<const float4*>(part_o + r * DV + d);
-                    x0[u] = __ldcg(src);
-                    x1[u] = __ldcg(src + 1);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kMergeRegs; ++u) {
-                if (s0 + u < n_split) {
-                    const float ws = (m == kNegInf ? 0.f : expf(l[u] - m)) * rs;
-                    acc[0] = fmaf(ws, x0[u].x, acc[0]); acc[1] = fmaf(ws, x0[u].y, acc[1]);
-                    acc[2] = fmaf(ws, x0[u].z, acc[2]); acc[3] = fmaf(ws, x0[u].w, acc[3]);
-                    acc[4] = fmaf(ws, x1[u].x, acc[4]); acc[5] = fmaf(ws, x1[u].y, acc[5]);
-                    acc[6] = fmaf(ws, x1[u].z, acc[6]); acc[7] = fmaf(ws, x1[u].w, acc[7]);
-                }
-            }
-        }
+        merge_store(acc, ((size_t)t * H + h) * DV + d, o, o32);
     }
-    const size_t out = ((size_t)t * H + h) * DV + d;
-    if (o32) {
-        *reinterpret_cast<float4*>(o32 + out) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4*>(o32 + out + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    } else {
-        uint4 pk;
-        pk.x = pack_bf16x2(acc[0], acc[1]); pk.y = pack_bf16x2(acc[2], acc[3]);
-        pk.z = pack_bf16x2(acc[4], acc[5]); pk.w = pack_bf16x2(acc[6], acc[7]);
-        *reinterpret_cast<uint4*>(o + out) = pk;
-    }
-    if (lse && d == 0) lse[(size_t)t * H + h] = wsum > 0.f ? m + logf(wsum) : kNegInf;
+    if (lse && threadIdx.x == 0) lse[(size_t)t * H + h] = wsum > 0.f ? m + logf(wsum) : kNegInf;
 }
 
 cudaError_t launch_merge_partials(const float* part_o, const float* part_lse, int n_part, int64_t part_stride,
                                   int64_t tok_stride, int T, int H, int DV, uint16_t* o, float* o32, float* lse,
                                   cudaStream_t st) {
     if (T <= 0) return cudaSuccess;
-    dim3 mg((H * (DV / 8) + kMergeThreads - 1) / kMergeThreads, T);
-    merge_kernel<<<mg, kMergeThreads, 0, st>>>(part_o, part_lse, n_part, H, DV, part_stride, tok_stride, o, o32, lse);
+    if (n_part <= 32) {
+        const int64_t warps = (int64_t)H * ((DV + 127) / 128);
+        dim3 mg((unsigned)((warps + kMergeThreads / 32 - 1) / (kMergeThreads / 32)), T);
+        merge_kernel<<<mg, kMergeThreads, 0, st>>>(part_o, part_lse, n_part, H, DV, part_stride, tok_stride, o, o32,
+                                                   lse);
+    } else {
+        merge_wide_kernel<<<dim3(H, T), kMergeThreads, (size_t)n_part * sizeof(float), st>>>(
+            part_o, part_lse, n_part, DV, part_stride, tok_stride, o, o32, lse);
+    }
     return cudaGetLastError();
 }
 
