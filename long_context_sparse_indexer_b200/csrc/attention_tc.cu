@@ -84,7 +84,13 @@ struct AttnSmem {
     alignas(16) float kmask[kStagesA][kRows];    // 0, or -inf for masked rows (added to the scaled score)
     alignas(16) float vscale[kStagesA][kRows];   // per-row FP8 scale (1 for BF16)
     int rows[kStagesA][kRows];
-    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[kSP], p_full[kSP], o_done[2], q_ready, q_tma;
+    uint64_t kv_full[kStagesA], kv_empty[kStagesA], s_full[kSP], p_full[kSP], q_ready, q_tma;
+    // P V_k completes phase k / kSP of o_done[k % kSP].  A parity wait tells two phases apart only
+    // if the earlier one is complete: a thread that has seen S_j done knows P V_{j-4} done (the
+    // commit after S_j covers every earlier MMA, and S_j is issued after P V_{j-4}), so it may
+    // wait for P V_{j-1} on a ring of kSP barriers -- on two it could not, P V_{j-3} may still be
+    // pending.  mma_done: committed once, after the last MMA (the issuer's drain).
+    uint64_t o_done[kSP], mma_done;
     uint64_t s_sent[kSP];                        // the send warps have read S out of this buffer
     uint64_t hand[2][4];                         // softmax warpgroup w, quarter q: m_ref of its tile is out
     float m_ref[128];                            // the reference max after the latest decided tile
@@ -152,7 +158,8 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                 tc::mbar_init(&sm.rx_full[x][q], 1);     // the receiving warp's expect_tx + the copy's bytes
                 tc::mbar_init(&sm.tx_free[x][q], 1);     // one remote arrival from the peer's warp q
             }
-        for (int i = 0; i < 2; ++i) tc::mbar_init(&sm.o_done[i], 1);
+        for (int i = 0; i < kSP; ++i) tc::mbar_init(&sm.o_done[i], 1);
+        tc::mbar_init(&sm.mma_done, 1);
         for (int w = 0; w < 2; ++w)
             for (int q = 0; q < 4; ++q) tc::mbar_init(&sm.hand[w][q], 1);
         tc::mbar_init(&sm.q_ready, kSmx * 128);
@@ -408,7 +415,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                                        (npv > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit(&sm.kv_empty[npv % kStagesA]);
-                    tc::mma_commit(&sm.o_done[npv & 1]);
+                    tc::mma_commit(&sm.o_done[npv % kSP]);
                     ++npv;
                     progressed = true;
                 }
@@ -416,9 +423,10 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                     if (*abort_flag || tc::global_ns() - t0 > tc::kWaitNs * 4) { *abort_flag = 1; break; }
                 }
             }
-            if (npv > 0) {                          // drain before TMEM is freed
+            if (ns > 0) {                           // drain before TMEM is freed (every MMA issued)
+                tc::mma_commit(&sm.mma_done);
                 volatile int drain_abort = 0;
-                tc::mbar_wait(&sm.o_done[(npv - 1) & 1], ((npv - 1) >> 1) & 1, &drain_abort);
+                tc::mbar_wait(&sm.mma_done, 0, &drain_abort);
             }
         }
     } else if (smx_warp) {
@@ -557,7 +565,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             if (__any_sync(0xffffffffu, rescale)) {
                 // O must hold P V_{j-1} before it is rescaled.
                 if (j >= 1 &&
-                    !__all_sync(0xffffffffu, tc::mbar_wait(&sm.o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
+                    !__all_sync(0xffffffffu, tc::mbar_wait(&sm.o_done[(j - 1) % kSP], ((j - 1) / kSP) & 1, abort_flag))) {
                     alive = false;
                     break;
                 }
@@ -593,7 +601,8 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             l_f = (m_w == kNegInf ? 0.f : l_w * ex2(m_w - m_f)) + (o.x == kNegInf ? 0.f : o.y * ex2(o.x - m_f));
         }
         if (alive && n_tiles > 0 &&
-            !__all_sync(0xffffffffu, tc::mbar_wait(&sm.o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag)))
+            !__all_sync(0xffffffffu,
+                        tc::mbar_wait(&sm.o_done[(n_tiles - 1) % kSP], ((n_tiles - 1) / kSP) & 1, abort_flag)))
             alive = false;
         tc::tc_fence_after();
         const float kLn2 = 0.69314718055994530942f;
