@@ -282,6 +282,46 @@ def test_topk_matches_oracle_exactly(cuda, n_cols, k, n_sink, window, tie_levels
         assert np.all(idx[t, cnt[t]:].cpu().numpy() == -1)
 
 
+@pytest.mark.parametrize("T,n_cols,fixed_budget,tie_levels", [
+    (63, 30000, False, 40),        # fewer than 64 rows: clusters of 8
+    (64, 30000, False, 40),        # clusters of 2 (a row's half fits the shared-memory cache);
+                                   # a wide threshold bin: the full passes over the segments
+    (64, 30000, False, 100000),    # clusters of 2, few candidates: the compacted finish
+    (64, 30000, True, 40),
+    (64, 100000, False, 100000),   # clusters of 4 (a half does not fit, a quarter does)
+    (64, 200000, False, 100000),   # clusters of 8 (a quarter does not fit either)
+])
+def test_topk_cluster_sizes(cuda, T, n_cols, fixed_budget, tie_levels):
+    """The launch picks the cluster size per row from the row count and the row width; every
+    choice must give the oracle's lists.  Positions differ per row (several rows see only part
+    of the row), scores carry ties."""
+    rng = np.random.default_rng(T * 1000 + n_cols + int(fixed_budget) + tie_levels)
+    k, n_sink, window = 2048, 4, 512
+    s = _host_score_rows(rng, T, n_cols, tie_levels)
+    pos = rng.integers(n_cols // 3, n_cols, size=T)
+    pos[:3] = [n_cols - 1, 700, 3000]
+    for t in range(T):
+        s[t, pos[t] + 1:] = -np.inf
+    batch = lsa.Batch(torch.tensor([n_cols], dtype=torch.int32, device="cuda"),
+                      torch.zeros(T, dtype=torch.int32, device="cuda"),
+                      torch.from_numpy(pos.astype(np.int32)).cuda(), n_cols)
+    idx = torch.empty((T, k + n_sink + window), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(T, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.topk(batch, torch.from_numpy(s).cuda(), n_cols, k, n_sink, window, idx, cnt, dev_status=st,
+             fixed_budget=fixed_budget)
+    assert lsa.read_device_status(st) == lsa.OK
+    got = H.index_lists(idx, cnt)
+    for t in range(T):
+        cols = np.nonzero(~np.isneginf(s[t]))[0]
+        sc = s[t, cols].astype(np.float64)
+        if fixed_budget:
+            want = olsa.union_fixed_budget(sc, cols, k, int(pos[t]), n_sink, window)
+        else:
+            want = olsa.union_fixed(olsa.topk(sc, cols, k), int(pos[t]), n_sink, window)
+        assert got[t].tolist() == want.tolist(), t
+
+
 @pytest.mark.parametrize("n_cols", [3000, 70000])
 def test_topk_all_equal_scores(cuda, n_cols):
     """Every visible score equal (as when every weighted ReLU sum is 0): the selection is the
