@@ -156,22 +156,29 @@ __device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t v) {
 // i: row n = i / 8 (token
 // n / H_I, head n % H_I), 16-element chunk c = i % 8; the 8 chunks of a row sit in 8 consecutive
 // lanes, which reduce the row maximum by shuffles.  Loads are issued four items at a time.
-template <int N>
+// `mid` runs once, after the first batch's loads are issued (the caller's own loads then overlap
+// them).  The head weight is loaded with its row.
+template <int N, typename Mid>
 __device__ void prepare_queries(const IndexArgs& a, int t0, int H_I, int ct, int nthr, uint8_t* q_hi,
-                                uint8_t* q_lo, float* w_out) {
+                                uint8_t* q_lo, float* w_out, Mid mid) {
     constexpr int kB = 4;
+    bool first = true;
     for (int i0 = ct; i0 < N * 8; i0 += nthr * kB) {
         uint4 raw[kB][2];
+        float wv[kB];
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
             const int i = i0 + u * nthr;
             if (i < N * 8) {                                  // warp-uniform: N * 8 is a multiple of 32
                 const int n = i >> 3, c = i & 7;
-                const uint16_t* src = a.q + ((size_t)(t0 + n / H_I) * H_I + n % H_I) * 128 + c * 16;
+                const size_t row = (size_t)(t0 + n / H_I) * H_I + n % H_I;
+                const uint16_t* src = a.q + row * 128 + c * 16;
                 raw[u][0] = *reinterpret_cast<const uint4*>(src);
                 raw[u][1] = *reinterpret_cast<const uint4*>(src + 8);
+                wv[u] = c == 0 ? a.w[row] : 0.f;
             }
         }
+        if (first) { mid(); first = false; }
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
             const int i = i0 + u * nthr;
@@ -210,27 +217,33 @@ __device__ void prepare_queries(const IndexArgs& a, int t0, int H_I, int ct, int
             const int off = (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4);
             *reinterpret_cast<uint4*>(q_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             *reinterpret_cast<uint4*>(q_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            if (c == 0) w_out[n] = a.w[(size_t)(t0 + n / H_I) * H_I + n % H_I] * exp2i(-s);
+            if (c == 0) w_out[n] = wv[u] * exp2i(-s);
         }
     }
 }
 
 // Token gi (< kMaxG) of the group starting at t0: its position, and whether it is a valid query of
-// the group's sequence (a token of another sequence, or out of range, sees no key).
-__device__ __forceinline__ void set_group_validity(const IndexArgs& a, int t0, int G, int gi, int* pos, int* ok) {
-    int okv = 0, p = -1;
-    if (gi < G) {
-        const int b0 = a.q_seq[t0], sq = a.q_seq[t0 + gi];
-        p = a.q_pos[t0 + gi];
-        okv = sq == b0 && sq >= 0 && sq < a.B;
-        if (okv) {
-            const int len = a.seq_len[sq];
-            okv = len >= 1 && len <= a.L_alloc && p >= 0 && p < len;
-        }
+// the group's sequence (a token of another sequence, or out of range, sees no key).  In two
+// halves -- the token's sequence and position, then its sequence's length -- so that a caller can
+// put other loads between them.
+struct GroupValidity {
+    int b0 = -1, sq = -1, p = -1, len = 0;
+    bool in = false;
+    __device__ void load(const IndexArgs& a, int t0, int G, int gi) {
+        in = gi < G;
+        if (in) { b0 = a.q_seq[t0]; sq = a.q_seq[t0 + gi]; p = a.q_pos[t0 + gi]; }
     }
-    pos[gi] = okv ? p : -1;
-    ok[gi] = okv;
-}
+    __device__ void load_len(const IndexArgs& a) {
+        if (in && sq == b0 && sq >= 0 && sq < a.B) len = a.seq_len[sq];
+    }
+    __device__ void store(const IndexArgs& a, int gi, int* pos, int* ok) const {
+        const bool okv = in && sq == b0 && sq >= 0 && sq < a.B && len >= 1 && len <= a.L_alloc && p >= 0 && p < len;
+        if (in && !okv) report(a.status, LSA_ERR_DEVICE_DATA);
+        pos[gi] = okv ? p : -1;
+        ok[gi] = okv;
+    }
+};
+
 
 // Weighted ReLU head sums of two accumulator rows held by this thread: item a (columns
 // ca .. ca + H_I - 1 of the TMEM row, weights wa) and item b (cb, wb; skipped unless `two`).
@@ -315,12 +328,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         const int b0 = a.q_seq[t0];
         int max_pos = -1;
         for (int gi = 0; gi < G; ++gi) {
+            // The tile count needs no sequence length (one round trip less before the first key
+            // tile is requested): a position past its sequence only adds tiles whose columns the
+            // epilogue writes as -inf, and is reported where the group's queries are prepared.
             const int s = a.q_seq[t0 + gi], p = a.q_pos[t0 + gi];
-            bool ok = s == b0 && s >= 0 && s < a.B;
-            if (ok) {
-                const int len = a.seq_len[s];
-                ok = len >= 1 && len <= a.L_alloc && p >= 0 && p < len;
-            }
+            const bool ok = s == b0 && s >= 0 && s < a.B && p >= 0;
             if (ok) max_pos = max(max_pos, p);
             else if (blockIdx.x == 0) report(a.status, LSA_ERR_DEVICE_DATA);
         }
@@ -344,8 +356,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
         const int ct = threadIdx.x - 64;                                // 0..319
         const Walk w0(sm.tstart, NG, k_lo);
         const int t0 = (pa.group0 + w0.g) * G;
-        if (ct < kMaxG) set_group_validity(a, t0, G, ct, sm.pos[0], sm.ok[0]);
-        prepare_queries<N>(a, t0, H_I, ct, kPThreads - 64, sm.q[0][0], sm.q[0][1], sm.w[0]);
+        // The validity loads go out with the query loads; the length load, which needs the
+        // sequence, after them, so that it overlaps the query arithmetic.
+        GroupValidity gv;
+        if (ct < kMaxG) gv.load(a, t0, G, ct);
+        prepare_queries<N>(a, t0, H_I, ct, kPThreads - 64, sm.q[0][0], sm.q[0][1], sm.w[0],
+                           [&] { if (ct < kMaxG) gv.load_len(a); });
+        if (ct < kMaxG) gv.store(a, ct, sm.pos[0], sm.ok[0]);
         tc::fence_proxy_async_smem();
         asm volatile("bar.sync 2, %0;" :: "n"(kPThreads - 64) : "memory");
         if (warp < 4) tc::mbar_arrive(&sm.q_full[0]);
@@ -435,8 +452,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
                            !tc::mbar_wait(&sm.q_free[qb][1], ((e - 2) >> 1) & 1, abort_flag, wlim)))
                 break;
             const int t0 = (pa.group0 + wk.g) * G;
-            if (ct < kMaxG) set_group_validity(a, t0, G, ct, sm.pos[qb], sm.ok[qb]);
-            prepare_queries<N>(a, t0, H_I, ct, kPrepThreads, sm.q[qb][0], sm.q[qb][1], sm.w[qb]);
+            GroupValidity gv;
+            if (ct < kMaxG) gv.load(a, t0, G, ct);
+            prepare_queries<N>(a, t0, H_I, ct, kPrepThreads, sm.q[qb][0], sm.q[qb][1], sm.w[qb],
+                               [&] { if (ct < kMaxG) gv.load_len(a); });
+            if (ct < kMaxG) gv.store(a, ct, sm.pos[qb], sm.ok[qb]);
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(&sm.q_full[qb]);
         }
