@@ -57,6 +57,7 @@ constexpr int kBlock = 128;            // keys per MMA (M); a tile is NB such bl
 constexpr int kBlockBytes = kBlock * 128;
 constexpr int kMaxG = 4;
 constexpr int kMaxGroups = 2048;       // query-token groups one launch schedules
+constexpr int kEarlyTiles = 2;         // key tiles requested before the first queries are ready
 
 struct PArgs {
     IndexArgs a;
@@ -376,6 +377,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
             int s = 0, ph = 0, issued = 0;
             for (int k = k_lo; k < k_hi; ++k) {
                 if (wk.to(k)) { t0 = (pa.group0 + wk.g) * G; bseq = max(a.q_seq[t0], 0); }
+                // Two key tiles go out at once; the rest of the ring only once the first group's
+                // queries are prepared.  Every CTA starts its key stream at the same moment, and a
+                // full ring of them (≈24 MB over the GPU) queued ahead of the queries' own loads
+                // delayed the first MMA; the tensor pipe cannot start before the queries anyway.
+                if (k == k_lo + kEarlyTiles && !tc::mbar_wait(&sm.q_full[0], 0, abort_flag, wlim)) break;
                 if (!tc::mbar_wait(&sm.empty_k[s], ph ^ 1, abort_flag, wlim)) break;
                 ++issued;
                 tc::mbar_expect_tx(&sm.full_k[s], NB * kBlockBytes + (pa.scale_tma ? TK * 4 : 0));
