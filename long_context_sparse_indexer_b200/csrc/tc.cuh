@@ -276,21 +276,11 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uin
         : "memory");
 }
 
-// Arrives (release, cluster scope) on the mbarrier at shared::cluster address bar of a peer CTA.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar) : "memory");
-}
-
-// As mbar_arrive_remote without release semantics: orders none of this thread's earlier memory
-// accesses, so the caller must already know that the accesses it signals the end of are complete.
+// Arrives on the mbarrier at shared::cluster address bar of a peer CTA, without release
+// semantics: orders none of this thread's earlier memory accesses, so the caller must already know
+// that the accesses it signals the end of are complete.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar) {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar) : "memory");
-}
-
-// 16-byte store to shared::cluster address dst (a peer CTA's shared memory).
-__device__ __forceinline__ void st_cluster_v4(uint32_t dst, uint4 v) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(dst), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
 }
 
 // mbar_wait with acquire at cluster scope, for phases completed by a peer CTA's remote arrivals
