@@ -325,6 +325,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
     }
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
     for (int gl = threadIdx.x; gl < NG; gl += kPThreads) {
+        if (hi) {                                        // every group scores all n_cols candidates
+            sm.tstart[gl] = a.n_cols > 0 ? (a.n_cols + TK - 1) / TK : 0;
+            continue;
+        }
         const int t0 = (pa.group0 + gl) * G;
         const int b0 = a.q_seq[t0];
         int max_pos = -1;
@@ -337,7 +341,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_con
             if (ok) max_pos = max(max_pos, p);
             else if (blockIdx.x == 0) report(a.status, LSA_ERR_DEVICE_DATA);
         }
-        const int cols = hi ? a.n_cols : min(a.n_cols, max_pos + 1);
+        const int cols = min(a.n_cols, max_pos + 1);
         sm.tstart[gl] = (max_pos < 0 || cols <= 0) ? 0 : (cols + TK - 1) / TK;
     }
     __syncthreads();
