@@ -139,3 +139,64 @@ def test_partial_attention_and_merge_against_the_oracle(cuda):
         o_ref, _ = run.attend(w, p, p.layers[0], t, lists[t])
         mx, rl2 = H.attn_errors(on[t], o_ref)
         assert mx < 1e-2 and rl2 < 5e-3, (t, mx, rl2)
+
+
+@pytest.mark.parametrize("R,Dv", [(1, 512), (8, 512), (17, 512), (24, 512), (25, 512), (32, 512), (33, 512),
+                                  (100, 512), (17, 200), (40, 136)])
+def test_merge_partials_part_counts(cuda, R, Dv):
+    """lsa_merge_partials against the oracle's merge for every kernel path: up to 24 partials held in
+    registers, 25..32 with a second round trip, more than 32 through the block-per-head kernel; V
+    widths that are not a multiple of 128; empty partials (lse = -inf), a head with every partial
+    empty, and lse values far apart (one partial dominates)."""
+    rng = np.random.default_rng(R * 1000 + Dv)
+    T, H_ = 3, 24
+    o_parts = rng.normal(size=(R, T, H_, Dv)).astype(np.float32)
+    l_parts = (rng.normal(size=(R, T, H_)) * 3.0).astype(np.float32)
+    l_parts[rng.random(size=(R, T, H_)) < 0.2] = -np.inf           # empty partials
+    l_parts[:, 1, 5] = -np.inf                                     # a head with nothing at all
+    l_parts[0, 2, 7] = 60.0                                        # one partial dominates
+    o = torch.empty((T, H_, Dv), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((T, H_), dtype=torch.float32, device="cuda")
+    lsa.merge_partials(torch.from_numpy(o_parts).cuda(), torch.from_numpy(l_parts).cuda(), o, lse)
+    on, ln = H.bf16_to_np(o), lse.cpu().numpy()
+    for t in range(T):
+        om, lm = olsa.merge_partials([o_parts[i, t].astype(np.float64) for i in range(R)],
+                                     [l_parts[i, t].astype(np.float64) for i in range(R)])
+        assert np.abs(on[t] - om).max() <= 2.0 ** -8 * np.abs(om).max() + 1e-6, t
+        fin = np.isfinite(lm)
+        assert np.array_equal(fin, np.isfinite(ln[t]))
+        assert np.abs(ln[t][fin] - lm[fin]).max() < 1e-5 * max(1.0, np.abs(lm[fin]).max())
+    assert np.all(on[1, 5] == 0) and np.isneginf(ln[1, 5])
+
+
+def test_attention_with_many_splits(cuda):
+    """lsa_sparse_attn with 40 splits (the wide merge) agrees with one split within the attention
+    tolerance, on the oracle's own index lists."""
+    wt = D.build_workload(W.scaled("decode_cli_128k", B=2, len_lo=6000, len_hi=8000, seed=5), "cuda")
+    w = wt.w
+    p = w.passes[0]
+    T = w.T(p)
+    lists = {t: run.index_list(w, p, t, None)[0] for t in range(T)}
+    idx = torch.full((T, w.cap), -1, dtype=torch.int32)
+    cnt = torch.zeros(T, dtype=torch.int32)
+    for t, l in lists.items():
+        idx[t, :len(l)] = torch.from_numpy(l.astype(np.int32))
+        cnt[t] = len(l)
+    idx, cnt = idx.cuda(), cnt.cuda()
+    kv, _ = H.kv_cache(wt, 0, 0)
+    q = wt.passes[0].layers[0]["q"]
+    outs = {}
+    for ns in (1, 40):
+        o = torch.empty((T, w.H, w.Dv), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
+        ws = torch.empty(max(256, lsa.attn_workspace_size(T, w.H, w.Dv, ns)), dtype=torch.uint8, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        lsa.sparse_attn(H.batch_of(wt), q, kv, idx, cnt, w.sm_scale, o, lse, n_split=ns, ws=ws, dev_status=st)
+        assert lsa.read_device_status(st) == lsa.OK
+        outs[ns] = (H.bf16_to_np(o), lse.cpu().numpy())
+    for t in range(T):
+        o_ref, lse_ref = run.attend(w, p, p.layers[0], t, lists[t])
+        for ns in (1, 40):
+            mx, rl2 = H.attn_errors(outs[ns][0][t], o_ref)
+            assert mx < 1e-2 and rl2 < 5e-3, (ns, t, mx, rl2)
+            assert np.abs(outs[ns][1][t] - lse_ref).max() < 1e-3 * max(1.0, np.abs(lse_ref).max())
