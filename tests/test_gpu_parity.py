@@ -717,6 +717,17 @@ def test_device_data_errors_are_reported(cuda):
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     lsa.index_score(batch, pt.q_idx, pt.w, H.idx_cache(wt), sc, n_cols=wt.L_alloc, dev_status=st)
     assert lsa.read_device_status(st) == lsa.ERR_DEVICE_DATA
+    assert torch.isneginf(sc[1]).all()                        # the bad token sees no key
+    assert torch.isfinite(sc[0, :int(pt.q_pos[0]) + 1]).all()
+    # the same bad position in the HI fine stage (every group scores all candidate columns)
+    n_cand = 8
+    cand = torch.arange(n_cand, dtype=torch.int32, device="cuda").repeat(pt.q_idx.shape[0], 1).contiguous()
+    sc_hi = torch.empty((pt.q_idx.shape[0], n_cand * 64), dtype=torch.float32, device="cuda")
+    st.zero_()
+    lsa.index_score(batch, pt.q_idx, pt.w, H.idx_cache(wt), sc_hi, n_cols=n_cand * 64, cand_blocks=cand,
+                    block_size=64, dev_status=st)
+    assert lsa.read_device_status(st) == lsa.ERR_DEVICE_DATA
+    assert torch.isneginf(sc_hi[1]).all()
     # NaN score
     good = H.batch_of(wt)
     sc = H.flat_scores(wt)
