@@ -28,6 +28,7 @@
 #include <cooperative_groups.h>
 
 #include "kernels.cuh"
+#include "tc.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -257,6 +258,8 @@ topk_kernel(TopkArgs a) {
     __shared__ int s_sup[64], s_red[130], s_total, hist3[256];
     __shared__ int s_cand[kTopkCandCache];        // the row's candidate block ids (HI), when they fit
     extern __shared__ uint32_t s_keys[];          // CACHED: order key of each column of the segment, 0 = invalid
+    __shared__ uint64_t s_seg_full;               // CACHED: the segment's bulk copy has landed
+    __shared__ int s_abort;
     cg::cluster_group cl = cg::this_cluster();
     const int rank = (int)cl.block_rank();
     const int t = blockIdx.x / NC;
@@ -323,44 +326,48 @@ topk_kernel(TopkArgs a) {
     // ---- pass 1: top 12 bits (and, when cached, the segment's keys into shared memory)
     for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
     if (CACHED) {
-        // Batches of 8 independent 16-byte loads per thread, then conversion to keys.
-        constexpr int kB = 8;
+        // The segment comes into shared memory as raw scores by one bulk copy (its 16-byte
+        // multiple; the ragged tail, or a row not 16-byte aligned, by plain loads), then every
+        // thread turns its columns into order keys in place and counts them in the same sweep.
+        // One round trip instead of a register round trip per batch of loads, and one sweep of
+        // the segment instead of two.
+        const int n_seg = c1 - c0;
         const bool vec = (((uintptr_t)(row + c0)) & 15) == 0;
-        for (int base = c0 + threadIdx.x * 4; base < c1; base += kTopkThreads * 4 * kB) {
-            float f[kB][4];
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-                const int cc = base + u * kTopkThreads * 4;
-                if (vec && cc + 3 < c1) {
-                    const float4 v4 = *reinterpret_cast<const float4*>(row + cc);
-                    f[u][0] = v4.x; f[u][1] = v4.y; f[u][2] = v4.z; f[u][3] = v4.w;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) f[u][e] = cc + e < c1 ? row[cc + e] : kNegInf;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-                const int cc = base + u * kTopkThreads * 4;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if (cc + e >= c1) break;
-                    const float x = f[u][e];
-                    if (x != x) report(a.status, LSA_ERR_DEVICE_DATA);
-                    s_keys[cc + e - c0] = (x != x || x == kNegInf || fixed_pos(cc + e)) ? 0u : order_key(x);
-                }
+        const int n_bulk = vec ? (n_seg & ~3) : 0;
+        if (threadIdx.x == 0) {
+            s_abort = 0;
+            if (n_bulk > 0) {
+                tc::mbar_init(&s_seg_full, 1);
+                tc::fence_barrier_init();
             }
         }
-    }
-    __syncthreads();
-    for (int c = w0; c < w1; c += 32) {
-        const int cc = c + lane;
-        if (!CACHED && cc < w1) {
-            const float f = row[cc];
-            if (f != f) report(a.status, LSA_ERR_DEVICE_DATA);
+        __syncthreads();                                 // hist cleared, the barrier initialised
+        if (threadIdx.x == 0 && n_bulk > 0) {
+            tc::mbar_expect_tx(&s_seg_full, (uint32_t)n_bulk * 4);
+            tc::bulk_load(s_keys, row + c0, (uint32_t)n_bulk * 4, &s_seg_full);
         }
-        const uint32_t key = key_at(cc);
-        hist_add(hist, (int)(key >> 20), key != 0u);
+        for (int i = n_bulk + threadIdx.x; i < n_seg; i += kTopkThreads) s_keys[i] = __float_as_uint(row[c0 + i]);
+        if (n_bulk > 0 && !tc::mbar_wait(&s_seg_full, 0, &s_abort) && threadIdx.x == 0)
+            report(a.status, LSA_ERR_TIMEOUT);           // the keys are then not the row's; every CTA goes on
+        __syncthreads();                                 // the tail's plain stores
+        for (int i = threadIdx.x; i < n_seg; i += kTopkThreads) {
+            const float x = __uint_as_float(s_keys[i]);
+            if (x != x) report(a.status, LSA_ERR_DEVICE_DATA);
+            const uint32_t key = (x != x || x == kNegInf || fixed_pos(c0 + i)) ? 0u : order_key(x);
+            s_keys[i] = key;
+            hist_add(hist, (int)(key >> 20), key != 0u);
+        }
+    } else {
+        __syncthreads();
+        for (int c = w0; c < w1; c += 32) {
+            const int cc = c + lane;
+            if (cc < w1) {
+                const float f = row[cc];
+                if (f != f) report(a.status, LSA_ERR_DEVICE_DATA);
+            }
+            const uint32_t key = key_at(cc);
+            hist_add(hist, (int)(key >> 20), key != 0u);
+        }
     }
     // Cluster histogram of the top 12 bits; its total is the number of candidates.
     const int n_valid = cluster_threshold_4096<NC>(cl, hist, s_sup, a.k, s_red, &s_bin, &s_above, &s_total);
