@@ -243,12 +243,14 @@ constexpr int kTopkCacheCols = 40960;
 // Candidate block ids of a row kept in shared memory (HI: the recalled blocks).
 constexpr int kTopkCandCache = 1024;
 // Candidate lists of the compacted finish: per CTA (in its `hsum` array) and merged in CTA 0.
+// Above kTopkRefine expected candidates per warp the listing waits for the second radix digit.
+constexpr int kTopkRefine = 96;
 constexpr int kTopkLocalCap = 2048;
 constexpr int kTopkWarpCap = kTopkLocalCap / kTopkWarps;   // per warp
 constexpr int kTopkCap = 8192;
 
 template <bool CACHED, int NC>
-__global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(kTopkThreads)
+__global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(kTopkThreads, 2)
 topk_kernel(TopkArgs a) {
     __shared__ int hist[4096];
     __shared__ int hsum[4096];
@@ -372,13 +374,39 @@ topk_kernel(TopkArgs a) {
     // Cluster histogram of the top 12 bits; its total is the number of candidates.
     const int n_valid = cluster_threshold_4096<NC>(cl, hist, s_sup, a.k, s_red, &s_bin, &s_above, &s_total);
     const bool take_all = n_valid <= a.k;
+    uint32_t tb = a.k <= 0 ? 0xffffffffu : (take_all ? 1u : ((uint32_t)s_bin << 20));   // listing threshold
+
+    // ---- refinement before the listing.  When the keys at or above the threshold bin b1 would
+    // fill more than kTopkRefine slots per warp on average (a wide bin, few warps per row: the
+    // per-warp lists would overflow and the row would take the full passes), the next 12 bits
+    // are settled first over the cluster, and only keys at or above (b1, b2) are listed.  The
+    // counts are the cluster's, so every CTA takes the same branch.  CTA 0's finish then finds b2
+    // again from the candidates (all keys of bin b1 at or above it are among them).
+    if (!take_all && a.k > 0) {
+        const uint32_t b1 = (uint32_t)s_bin;
+        const int above1 = s_above;
+        const int b1_count = s_red[66 + (b1 & 63)];              // the cluster's keys in bin b1
+        if ((above1 + b1_count) / (NC * kTopkWarps) > kTopkRefine) {
+            cl.sync();                                           // peers are done reading hist / sup
+            for (int i = threadIdx.x; i < 4096; i += kTopkThreads) hist[i] = 0;
+            __syncthreads();
+            for (int c = w0; c < w1; c += 32) {
+                const uint32_t key = key_at(c + lane);
+                hist_add(hist, (int)((key >> 8) & 0xfff), key != 0u && (key >> 20) == b1);
+            }
+            cluster_threshold<NC>(cl, rank, hist, hsum, 4096, a.k - above1, s_warp, &s_bin, &s_above);
+            tb = (b1 << 20) | ((uint32_t)s_bin << 8);
+            __syncthreads();                                     // every thread has read b2
+            if (threadIdx.x == 0) { s_bin = (int)b1; s_above = above1; }   // pass 1's, for what follows
+            __syncthreads();
+        }
+    }
 
     // ---- compacted finish.  The top-k lies in the threshold bin b1 of pass 1 or above it, a few
     // thousand columns of the row: every warp lists its candidates (column order) in its region
     // of `hsum`; when they fit, every warp stores them into CTA 0's merged list, and CTA 0
     // completes the selection and the emission alone.
     {
-        const uint32_t tb = a.k <= 0 ? 0xffffffffu : (take_all ? 1u : ((uint32_t)s_bin << 20));
         // One pass: warp w appends its candidates (column order) to its own region of kTopkWarpCap
         // slots of the CTA's list in `hsum` (keys, then columns).
         uint32_t* lkey = reinterpret_cast<uint32_t*>(hsum);
