@@ -500,8 +500,15 @@ topk_kernel(TopkArgs a) {
                 for (int w = 0; w < warp; ++w) eq_base += s_wcnt[w];
             }
             // kept(i): selected, and (unless raw) its position outside the sinks and the window.
-            auto walk = [&](bool write, int o) -> int {
-                int eq_run = eq_base, cnt = 0;
+            // One walk: warp w stages its kept positions in shared memory from its own candidate
+            // offset e0 on (kept entries are a subset of its candidates, so the regions do not
+            // meet; `hsum` then `hist`, both free by now, hold kTopkCap entries), then copies them
+            // out once the warps' counts are known.
+            static_assert(kTopkCap <= 2 * 4096, "the staging spans hsum and hist");
+            auto stage = [&](int i) -> int& { return i < 4096 ? hsum[i] : hist[i - 4096]; };
+            int kept_w = 0;
+            {
+                int eq_run = eq_base;
                 for (int i = e0; i < e1; i += 32) {
                     const int ii = i + lane;
                     const bool in = ii < e1;
@@ -521,12 +528,10 @@ topk_kernel(TopkArgs a) {
                         if (!a.raw) keep = pv >= a_lo && pv < b_hi;
                     }
                     const uint32_t km = __ballot_sync(0xffffffffu, keep);
-                    if (write && keep) out[o + cnt + __popc(km & lt)] = pv;
-                    cnt += __popc(km);
+                    if (keep) stage(e0 + kept_w + __popc(km & lt)) = pv;
+                    kept_w += __popc(km);
                 }
-                return cnt;
-            };
-            const int kept_w = walk(false, 0);
+            }
             if (lane == 0) s_wk[warp] = kept_w;
             __syncthreads();
             int keep_base = 0, written = 0;
@@ -535,7 +540,7 @@ topk_kernel(TopkArgs a) {
                 if (w < warp) keep_base += v;
                 written += v;
             }
-            walk(true, a_lo + keep_base);
+            for (int j = lane; j < kept_w; j += 32) out[a_lo + keep_base + j] = stage(e0 + j);
             int n_out = a_lo + written;
             if (!a.raw) {
                 for (int i = threadIdx.x; i < a_lo; i += kTopkThreads) out[i] = i;
