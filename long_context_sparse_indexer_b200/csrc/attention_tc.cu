@@ -25,9 +25,11 @@
 // Warp roles (512 threads).  With BF16 rows:
 //   warps 0,2,3: gather -- tile j by the (j mod 3)-th: the rows' indices (prefetched three tiles
 //                of the warp ahead) and validity to shared memory, then the V-half atoms with
-//                tile::gather4 (4 rows x 64 dims per load) and the 4 rope chunks of each row with
-//                16-byte cp.async; both complete on the tile's barrier by themselves, so the warp
-//                moves on at once.  (Without a tensor map for the cache, cp.async does it all.)
+//                tile::gather4 (4 rows x 64 dims per load; a tile of 32 consecutive valid rows,
+//                as the window gives, with one TMA box of 32 rows per atom) and the 4 rope chunks
+//                of each row with 16-byte cp.async; both complete on the tile's barrier by
+//                themselves, so the warp moves on at once.  (Without a tensor map for the cache,
+//                cp.async does it all.)
 //   warp 1     : MMA issuer -- S_j (16 TS + 2 SS MMAs, N = 32) once tile j has landed, P V_{j-4}
 //                has been issued and S_{j-4} has been sent; O += P_j V_j (2 TS MMAs, N = 256) once
 //                the softmax of tile j is done; whichever is ready, each kind in order.
@@ -122,7 +124,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
 template <bool KV_FP8, bool TMA>
 __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
-                          AttnArgs a) {
+                          const __grid_constant__ CUtensorMap kvtile, AttnArgs a) {
     static_assert(!(KV_FP8 && TMA), "TMA gathers BF16 rows only");
     constexpr bool kAsync = !KV_FP8;             // gather by 3 warps that do not wait for their copies
     constexpr int kSmx = kAsync ? 2 : 1;         // softmax warpgroups
@@ -247,7 +249,10 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
             const int r0 = r_beg + j * kRows;
             return lane < min(kRows, r_end - r0) ? irow[r0 + lane] : -1;
         };
-        if (TMA && lane == 0) tc::prefetch_tmap(&kvmap);
+        if (TMA && lane == 0) {
+            tc::prefetch_tmap(&kvmap);
+            tc::prefetch_tmap(&kvtile);
+        }
         // Row coordinate of this sequence's row 0 in the map (TMA): the cache is B sequences of
         // kv_seq_b / kv_tok_b rows.
         const int row0 = TMA ? (int)((int64_t)max(b, 0) * (a.kv_seq_b / a.kv_tok_b)) : 0;
@@ -282,19 +287,29 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
                 // A masked row reads as zeros.  Each lane's cp.async arrive on the barrier when
                 // they complete (32 of its 33 arrivals); the 33rd is lane 0's, after the scales.
                 if constexpr (TMA) {
-                    // V half: 8 groups of 4 rows x 4 atoms, 512 B per tile::gather4 (coordinate
-                    // -1 is outside the map).
+                    // V half.  A tile of 32 valid consecutive rows (the window, or a context
+                    // shorter than the selection) is one box of 32 rows per atom; any other tile
+                    // is 8 groups of 4 rows x 4 atoms, 512 B per tile::gather4 (coordinate -1 is
+                    // outside the map).  Both land the same swizzled bytes.
                     const int grow = (cur >= 0 && cur < len) ? row0 + cur : -1;
-                    int rr[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) rr[i] = __shfl_sync(0xffffffffu, grow, ((lane & 7) << 2) + i);
+                    const int grow0 = __shfl_sync(0xffffffffu, grow, 0);
+                    const bool run = __all_sync(0xffffffffu, grow >= 0 && grow == grow0 + lane);
                     if (lane == 0) tc::mbar_expect_tx(&sm.kv_full[g], kVBytes);
                     __syncwarp();
-                    if (lane < 8) {
+                    if (run) {
+                        if (lane < 4)
+                            tc::tma_load_2d(sm.kv[g] + lane * (kRows * 128), &kvtile, &sm.kv_full[g],
+                                            half * kHalf + lane * 64, grow0);
+                    } else {
+                        int rr[4];
 #pragma unroll
-                        for (int la = 0; la < 4; ++la)
-                            tc::tma_gather4(sm.kv[g] + la * (kRows * 128) + lane * 512, &kvmap, &sm.kv_full[g],
-                                            half * kHalf + la * 64, rr[0], rr[1], rr[2], rr[3]);
+                        for (int i = 0; i < 4; ++i) rr[i] = __shfl_sync(0xffffffffu, grow, ((lane & 7) << 2) + i);
+                        if (lane < 8) {
+#pragma unroll
+                            for (int la = 0; la < 4; ++la)
+                                tc::tma_gather4(sm.kv[g] + la * (kRows * 128) + lane * 512, &kvmap, &sm.kv_full[g],
+                                                half * kHalf + la * 64, rr[0], rr[1], rr[2], rr[3]);
+                        }
                     }
                     // Rope: 4 chunks per row.
 #pragma unroll
@@ -704,18 +719,17 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(kAThreads, 1)
 }
 
 template <bool KV_FP8, bool TMA>
-cudaError_t launch_t(const CUtensorMap& qm, const CUtensorMap& m, const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_t(const CUtensorMap& qm, const CUtensorMap& m, const CUtensorMap& mt, const AttnArgs& a,
+                     cudaStream_t st) {
     const size_t smem = sizeof(AttnSmem) + 1024;
     auto kern = sparse_attn_tc_kernel<KV_FP8, TMA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_split, 2, a.T);
-    kern<<<grid, kAThreads, smem, st>>>(qm, m, a);
+    kern<<<grid, kAThreads, smem, st>>>(qm, m, mt, a);
     return cudaGetLastError();
 }
 
-// The BF16 cache as one 2-D tensor of rows (row of sequence b, token i = b * (kv_seq_b / kv_tok_b)
-// + i) for tile::gather4.  False when the layout or the driver does not allow it.
 // The queries [T][128][576] as a 2-D tensor of T * 128 rows, box 64 dims x 128 heads.
 bool make_q_map(const AttnArgs& a, CUtensorMap* m) {
     if (tc::encode_tiled() == nullptr || a.T < 1 || (int64_t)a.T * 128 >= ((int64_t)1 << 31)) return false;
@@ -728,14 +742,17 @@ bool make_q_map(const AttnArgs& a, CUtensorMap* m) {
                               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_kv_map(const AttnArgs& a, CUtensorMap* m) {
+// The BF16 cache as one 2-D tensor of rows (row of sequence b, token i = b * (kv_seq_b / kv_tok_b)
+// + i), box 64 dims x `box_rows` rows: 1 for tile::gather4, kRows for a tile of consecutive rows.
+// False when the layout or the driver does not allow it.
+bool make_kv_map(const AttnArgs& a, CUtensorMap* m, int box_rows) {
     if (tc::encode_tiled() == nullptr || a.B < 1 || a.kv_tok_b <= 0 || a.kv_seq_b % a.kv_tok_b != 0) return false;
     const int64_t rps = a.kv_seq_b / a.kv_tok_b;
     const int64_t rows = (int64_t)(a.B - 1) * rps + a.L_alloc;
     if (rows < 1 || rows >= ((int64_t)1 << 31) || (a.B > 1 && rps < 1)) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)a.kv_tok_b};
-    const cuuint32_t box[2] = {64, 1};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return tc::encode_tiled()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint8_t*>(a.kv), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -751,13 +768,15 @@ bool sparse_attn_tc_supported(const AttnArgs& a, int DQK, int DV, bool sep_v) {
 }
 
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, bool kv_fp8, cudaStream_t st) {
-    CUtensorMap qm, m;
+    CUtensorMap qm, m, mt;
     memset(&m, 0, sizeof(m));
+    memset(&mt, 0, sizeof(mt));
     if (!make_q_map(a, &qm)) return cudaErrorInvalidValue;
-    if (kv_fp8) return launch_t<true, false>(qm, m, a, st);
-    if (make_kv_map(a, &m)) return launch_t<false, true>(qm, m, a, st);
+    if (kv_fp8) return launch_t<true, false>(qm, m, mt, a, st);
+    if (make_kv_map(a, &m, 1) && make_kv_map(a, &mt, kRows)) return launch_t<false, true>(qm, m, mt, a, st);
     memset(&m, 0, sizeof(m));
-    return launch_t<false, false>(qm, m, a, st);
+    memset(&mt, 0, sizeof(mt));
+    return launch_t<false, false>(qm, m, mt, a, st);
 }
 
 }  // namespace lsa
