@@ -544,6 +544,56 @@ def test_attention_on_oracle_index(cuda, name, n_split):
             assert np.abs(ln[t] - lse_ref).max() < 1e-3 * max(1.0, np.abs(lse_ref).max())
 
 
+@pytest.mark.parametrize("n_split", [1, 3, 7])
+def test_attention_runs_of_consecutive_rows(cuda, n_split):
+    """Tiles of 32 consecutive valid rows (one TMA box per atom) next to scattered tiles (row
+    gathers): runs that start on and off a tile boundary, a run cut by the list's end, a run
+    that ends at the query's position (the window), and a short run inside a scattered tile."""
+    name = "cli_small"
+    w = SMALL[name]
+    wt = wt_of(name)
+    p = w.passes[0]
+    T = w.T(p)
+    q_seq, q_pos = W.query_rows(w, p)
+    rng = np.random.default_rng(7)
+    lists = {}
+    for t in range(T):
+        pos = int(q_pos[t])
+        scattered = np.sort(rng.choice(np.arange(200, 1500), size=45, replace=False))
+        parts = [np.arange(0, 96),                       # three whole tiles from list offset 0
+                 scattered[:5],                          # shifts the next run off the tile grid
+                 np.arange(1600, 1670),                  # a run across two tile boundaries
+                 scattered[5:],
+                 np.arange(1700, 1708),                  # a run shorter than a tile
+                 np.arange(pos - 99, pos + 1)]           # the window, ending at the query
+        l = np.unique(np.concatenate(parts))
+        l = l[l <= pos]
+        lists[t] = l.astype(np.int64)
+    cap = max(len(l) for l in lists.values())
+    idx = torch.full((T, cap), -1, dtype=torch.int32)
+    cnt = torch.zeros(T, dtype=torch.int32)
+    for t, l in lists.items():
+        idx[t, :len(l)] = torch.from_numpy(l.astype(np.int32))
+        cnt[t] = len(l)
+    idx, cnt = idx.cuda(), cnt.cuda()
+    batch = H.batch_of(wt)
+    layer = p.layers[0]
+    kv, v = H.kv_cache(wt, 0, 0)
+    q = wt.passes[0].layers[0]["q"]
+    o = torch.empty((T, w.H, w.Dv), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(256, lsa.attn_workspace_size(T, w.H, w.Dv, n_split)), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.sparse_attn(batch, q, kv, idx, cnt, w.sm_scale, o, lse, v=v, n_split=n_split, ws=ws, dev_status=st)
+    assert lsa.read_device_status(st) == lsa.OK
+    on, ln = H.bf16_to_np(o), lse.cpu().numpy()
+    for t in range(T):
+        o_ref, lse_ref = run.attend(w, p, layer, t, lists[t])
+        mx, rl2 = H.attn_errors(on[t], o_ref)
+        assert mx < 1e-2 and rl2 < 5e-3, (t, mx, rl2)
+        assert np.abs(ln[t] - lse_ref).max() < 1e-3 * max(1.0, np.abs(lse_ref).max())
+
+
 # ------------------------------------------------------------------ whole path
 
 @pytest.mark.parametrize("name", list(SMALL))
