@@ -9,17 +9,21 @@
 // Method: radix select on the order-preserving 32-bit key of each score, 12 + 12 + 8 bits.
 // One query row is handled by a cluster of NC CTAs (8 for a few rows, 2 or 4 for many: see
 // launch_topk); CTA r owns the r-th contiguous segment of the row (cached in shared memory as
-// order keys when it has at most 40960 columns, else re-read from global memory).  Histograms are integer shared-memory counts (atomics;
-// counts do not depend on atomic order).
+// order keys when it has at most 40960 columns, else re-read from global memory).  Histograms
+// are integer shared-memory counts (atomics; counts do not depend on atomic order).
 //   1. Top 12 bits over the cluster: each CTA folds its 4096 bins into 64 super-bins; after one
-//      cluster barrier every CTA reads the 8 x 64 super-bin counts, then the 8 x 64 bins inside
+//      cluster barrier every CTA reads the NC x 64 super-bin counts, then the NC x 64 bins inside
 //      the threshold super-bin, through distributed shared memory, and finds the same bin b1.
-//   2. The keys at or above b1 (usually a few thousand) are compacted, in column order, into
-//      CTA 0's shared memory; CTA 0 alone finds the next 12 and the last 8 bits, i.e. the k-th
-//      key v* and the number m of ties at v* to keep, and emits: every key > v* and the first
-//      m keys == v* (lowest columns first), ranks from per-warp counts, ballots and popcounts.
-//      When the candidates do not fit, the cluster runs passes 2 and 3 over its segments and
-//      emits with cluster-wide prefix counts instead.
+//      When the keys at or above b1 would overflow the per-warp candidate lists, the next 12
+//      bits are settled over the cluster as well, and the listing threshold becomes (b1, b2).
+//   2. The keys at or above the threshold (usually a few thousand, about k after the second
+//      digit) are compacted, in column order, into CTA 0's shared memory; CTA 0 alone finds the
+//      next 12 and the last 8 bits, i.e. the k-th key v* and the number m of ties at v* to keep,
+//      and emits every key > v* and the first m keys == v* (lowest columns first) in one walk:
+//      each warp stages its kept positions in shared memory, and they are copied out at their
+//      offsets after a prefix over the warps' counts.  When the candidates do not fit, the
+//      cluster runs passes 2 and 3 over its segments and emits with cluster-wide prefix counts
+//      instead.
 // Positions are written in ascending order and merged with the sinks [0, a) and the window
 // [b, pos], so the list comes out sorted and de-duplicated.  Fixed-budget mode: sink and window
 // positions are no candidates at all, so the top-k is drawn from the other positions and the
@@ -78,8 +82,8 @@ __device__ __forceinline__ void hist_add(int* hist, int bin, bool on) {
 
 // Sums the histograms of all CTAs of the cluster into `sum` in every CTA, then finds the bin
 // where the count from the top first reaches `need` (identical in every CTA).  CTA r adds up
-// the r-th eighth of the bins over the cluster (distributed shared memory loads) and writes
-// the sums into every CTA's `sum` (distributed shared memory stores).
+// the r-th of NC equal shares of the bins over the cluster (distributed shared memory loads)
+// and writes the sums into every CTA's `sum` (distributed shared memory stores).
 template <int NC>
 __device__ int cluster_threshold(cg::cluster_group& cl, int rank, int* hist, int* sum, int nb, int need,
                                  int* s_warp, int* s_bin, int* s_above) {
@@ -147,8 +151,8 @@ __device__ __forceinline__ void top_crossing(const int* c, int base, int need, i
 
 // Two-level form of cluster_threshold for the 4096-bin histogram of the top 12 bits, with one
 // cluster barrier.  Each CTA folds its histogram into 64 super-bins of 64 bins (`sup`); after
-// the barrier every CTA reads the cluster's 8 x 64 super-bin counts, finds the super-bin where
-// the count from the top reaches `need`, then reads the 8 x 64 bin counts inside it and finds
+// the barrier every CTA reads the cluster's NC x 64 super-bin counts, finds the super-bin where
+// the count from the top reaches `need`, then reads the NC x 64 bin counts inside it and finds
 // the bin (the same rule, so the same bin, as the one-level form).  Peers read `hist` and `sup`
 // after this returns: the caller must pass another cluster barrier before changing either.
 // Returns the cluster's total count; *s_bin / *s_above are left unchanged when no bin reaches
