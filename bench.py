@@ -478,15 +478,25 @@ def e2e_rate(w, wt, sds, args, world, dev, stream, q_per_step):
             "d2h_bytes_per_step": d2h_bytes, "ms_per_step": e2e_ms}
 
 
+def code_digest(src: bytes) -> str:
+    """SHA-256 of a C++/CUDA source's code: comments removed, whitespace runs collapsed, so that an
+    edit of the comments keeps the digest and any edit of the code changes it."""
+    import hashlib
+    import re
+    text = src.decode("utf-8")
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode("utf-8")).hexdigest()
+
+
 def indexer_traffic(kern: str, idx_bytes: float):
     """DRAM bytes per launch of the dominant kernel, from the committed ncu figures.
 
     profiles/indexer_traffic.json (flat tensor-core indexer) and profiles/block_score_traffic.json
     (HI block scores) record the ratio of measured DRAM traffic to algorithmic bytes of a capture
-    of that kernel and the SHA-256 of the kernel source it was taken on; the ratio is applied only
-    while the source still has that hash (otherwise the counters describe another kernel and the
-    field is null)."""
-    import hashlib
+    of that kernel and the digest of the kernel source's code it was taken on (code_digest); the
+    ratio is applied only while the source still has that digest (otherwise the counters describe
+    another kernel and the field is null)."""
     if kern.startswith("index_score"):
         rec, src_file = "indexer_traffic.json", "index_score_tc.cu"
     elif kern.startswith("block_score"):
@@ -499,7 +509,7 @@ def indexer_traffic(kern: str, idx_bytes: float):
         src = open(os.path.join(ROOT, "long_context_sparse_indexer_b200", "csrc", src_file), "rb").read()
     except (OSError, ValueError):
         return None
-    if hashlib.sha256(src).hexdigest() != d.get("source_sha256"):
+    if code_digest(src) != d.get("code_sha256"):
         return None
     return float(d["dram_bytes_over_algorithmic"]) * idx_bytes
 

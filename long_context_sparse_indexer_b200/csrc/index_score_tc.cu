@@ -19,17 +19,20 @@
 // tensor-core work.  Scores then differ from the BF16-query ones by the rounding of q.
 //
 // Scheduling.  Query tokens come in groups of G <= 4 tokens of one sequence (N = G*H_I <= 256
-// query rows share every key row).  A group's key range is cut into 128-key tiles; only tiles
-// holding a visible key are active.  Every CTA counts the active tiles of all groups, takes an
+// query rows share every key row).  A group's key range is cut into tiles of NB blocks of 128
+// keys (NB = 2, 256-key tiles, for N <= 128; NB = 1 at N = 256); only tiles holding a visible
+// key are active.  Every CTA counts the active tiles of all groups, takes an
 // equal contiguous share of the concatenated list and runs it through one pipeline.  Tiles of
 // one group reuse its prepared queries; a CTA prepares a group's queries once ("epoch"), into
 // one of two buffers, so the next group's preparation overlaps the current group's tiles.
 //
-//   warp 0      : TMA producer -- key tiles (two 64-row boxes, 128-byte swizzle, which is the
-//                 K-major operand layout) and their per-token scales into a KS-stage ring;
+//   warp 0      : TMA producer -- key tiles (64-row boxes, 128-byte swizzle, which is the
+//                 K-major operand layout) and their per-token scales into a KS-stage ring; the
+//                 first kEarlyTiles tiles are requested before the first queries are ready;
 //                 allocates / frees TMEM.
-//   warp 1      : MMA issuer -- per tile, 8 (FP8 queries: 4) x tcgen05.mma kind::f8f6f4 (M = 128 keys, N, K = 32)
-//                 into one of 512 / N accumulator slots; its commit frees the key stage.
+//   warp 1      : MMA issuer -- per 128-key block, 8 (FP8 queries: 4) x tcgen05.mma kind::f8f6f4
+//                 (M = 128 keys, N, K = 32) into one of min(8, 512 / (NB N)) accumulator slots;
+//                 its commit frees the key stage.
 //   warps 2..3  : query preparation, once per epoch (hi / lo split, 128-byte-swizzled K-major).
 //   warps 4..11 : epilogue, two warpgroups taking alternate tiles -- thread = key row (= TMEM
 //                 lane): load the accumulator row, apply ReLU, the weighted head sum (eight

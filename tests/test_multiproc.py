@@ -64,3 +64,13 @@ def test_single_rank_is_identity():
     w = W.WORKLOADS["decode_cli_128k"]
     assert bench.rank_workload(w, 0, 1) is w
     assert bench.max_over_ranks(3.25, 1, torch.device("cpu")) == 3.25
+
+
+def test_traffic_records_follow_the_code_not_the_comments():
+    """The committed DRAM-traffic ratios apply while the kernel's code is the one they were
+    captured on: a comment edit keeps the digest, a code edit (one token) changes it."""
+    src = b"// header\nint f(int x) {  /* block\n comment */ return x + 1; // tail\n}\n"
+    assert bench.code_digest(src) == bench.code_digest(b"int f(int x) { return x + 1;\n}")
+    assert bench.code_digest(src) == bench.code_digest(src.replace(b"// tail", b"// another note"))
+    assert bench.code_digest(src) != bench.code_digest(src.replace(b"x + 1", b"x + 2"))
+    assert bench.indexer_traffic("attention", 1.0) is None      # no record for that kernel
