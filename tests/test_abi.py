@@ -57,6 +57,35 @@ def test_index_score_rejects_bad_arguments():
         == lsa.ERR_INVALID_ARG
 
 
+def test_block_calls_reject_bad_arguments():
+    """lsa_block_keys / lsa_block_score: layout of the block-key buffer, supported shapes, and an
+    empty batch as a no-op (L_alloc = 100, block size 64: 2 blocks of 2 * 128 BF16 each)."""
+    lib = lsa.library()
+    b, c = _batch(), _cache()
+    keys = lambda bb=b, cc=c, bs=64, kbar=4096, stride=512: lib.lsa_block_keys(  # noqa: E731
+        ctypes.byref(bb) if bb is not None else None, ctypes.byref(cc), bs, kbar, stride, None, None)
+    assert keys(bb=None) == lsa.ERR_INVALID_ARG
+    assert keys(kbar=None) == lsa.ERR_INVALID_ARG
+    assert keys(bs=0) == lsa.ERR_INVALID_ARG and keys(bs=1025) == lsa.ERR_INVALID_ARG
+    assert keys(stride=504) == lsa.ERR_INVALID_ARG                          # below 2 blocks x 2 d_I
+    assert keys(stride=516) == lsa.ERR_INVALID_ARG                          # not 16-byte rows
+    assert keys(kbar=4104) == lsa.ERR_INVALID_ARG                           # kbar not 16-byte aligned
+    assert keys(cc=_cache(dtype=7)) == lsa.ERR_UNSUPPORTED
+    assert keys(cc=_cache(scale=None)) == lsa.ERR_INVALID_ARG
+    assert keys(bb=lsa.CBatch(1, 0, 1, 100, None, None, None)) == lsa.ERR_INVALID_ARG   # no lengths
+
+    score = lambda bb=b, H_I=64, d_I=128, kbar=4096, stride=512, bs=64, ld=2, n=2, q=16, w=16, sc=16:         lib.lsa_block_score(ctypes.byref(bb), q, w, H_I, d_I, kbar, stride, bs, sc, ld, n, None, None)  # noqa: E731
+    assert score(H_I=48) == lsa.ERR_UNSUPPORTED
+    assert score(d_I=96) == lsa.ERR_UNSUPPORTED
+    assert score(bs=0) == lsa.ERR_INVALID_ARG
+    assert score(n=3, ld=3) == lsa.ERR_INVALID_ARG                          # more columns than blocks
+    assert score(n=2, ld=1) == lsa.ERR_INVALID_ARG                          # n_cols > ld
+    assert score(stride=504) == lsa.ERR_INVALID_ARG
+    assert score(q=None) == lsa.ERR_INVALID_ARG and score(sc=None) == lsa.ERR_INVALID_ARG
+    assert score(q=24) == lsa.ERR_INVALID_ARG and score(kbar=4104) == lsa.ERR_INVALID_ARG
+    assert score(bb=lsa.CBatch(1, 0, 1, 100, 16, None, None)) == lsa.OK     # no query: nothing to do
+
+
 def test_topk_rejects_bad_arguments():
     lib = lsa.library()
     b = _batch()
