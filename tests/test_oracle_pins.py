@@ -144,6 +144,21 @@ def test_worked_topk_and_union():
     assert lsa.union_fixed(picks3, 3, 2, 2).tolist() == u["pos_3_k_1_sink_2_window_2"]
 
 
+def test_worked_si_variants():
+    """The fixed-budget selection and the block-aligned window on the hand-worked example."""
+    g = _g()
+    s = np.array(g["indexer"]["scores"], float)
+    v = g["si_variants"]
+    pos = v["pos"]
+    for c in v["cases"]:
+        if c["fixed_budget"]:
+            got = lsa.union_fixed_budget(s, np.arange(pos + 1), c["k"], pos, c["n_sink"], c["window"], c["align"])
+        else:
+            got = lsa.union_fixed(lsa.topk(s, np.arange(pos + 1), c["k"]), pos, c["n_sink"], c["window"], c["align"])
+        assert got.tolist() == c["index_list"], c["why"]
+        assert lsa.window_start(pos, c["window"], c["align"]) == c["window_start"]
+
+
 def test_worked_hi():
     g = _g()
     q, w, K = (np.array(g["indexer"][n], float) for n in ("q", "w", "keys"))
